@@ -1,0 +1,368 @@
+#!/usr/bin/env python
+"""SegPagedAttention prefill benchmark (visible-pair TFLOP/s on B200).
+
+One step = one pass of the whole hot path over the Mistral-7B-shaped 32K
+layer (Hq 32, Hkv 8, D 128, P 64; 7 cached 4096-token segments + 4096 tail;
+kv_head 0 global, 1-7 local with a 4096 window): rk_relocate_rope (K, and V
+page copies) -> rk_select_visible -> rk_segpaged_prefill, inputs resident in
+HBM, L2 flushed (256 MiB write) between timed steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (torchrun, one rank per GPU) every rank runs its own replica
+(the work items are independent: weak scaling, no collective on the data
+path); time is the max over ranks of the summed device step times.
+``--impl reference`` times the fp64 CPU oracle on a bounded row sample of the
+same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "SegPagedAttn prefill visible-pair TFLOP/s & % BF16 peak at 32K"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+SPEC_BF16_TFLOPS = 2250.0
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def _kernel_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("rk_prefill.cu", "sm100.cuh", "rk_internal.h"):
+        with open(os.path.join(ROOT, "head_aware_paged_prefill_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def _recorded_traffic(kernel: str, workload: str):
+    """Per-launch DRAM bytes from the committed ncu summary, if it was taken on
+    the current kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel, {})
+    if e.get("source_hash") != _kernel_hash() or e.get("workload") != workload:
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def _gpu_id(torch, dev) -> str:
+    try:
+        return "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        return str(dev.index or 0)
+
+
+def _oracle_sample_rows(lay, n_rows: int, seed: int):
+    """A seeded sample of computed (layer, q_head, token) rows and the number of
+    visible keys of each, for the CPU baseline."""
+    rng = np.random.default_rng(seed)
+    g = lay.hq // lay.hkv
+    W = int(lay.class_window[1])
+    out, pairs = [], 0
+    L = lay.req_len(0)
+    tail0 = int(lay.segments[lay.segments[:, 4] == 0][0, 1])
+    for _ in range(n_rows):
+        h = int(rng.integers(lay.hq))
+        cls = int(lay.class_map[h // g])
+        i = int(rng.integers(L)) if cls in (0, 3) else int(rng.integers(tail0, L))
+        out.append((0, h, i))
+        pairs += (i + 1) if cls in (0, 3) else min(i + 1, W)
+    return np.asarray(out, dtype=np.int32), pairs
+
+
+def _time_oracle(lay, q, k, v, rows):
+    import torch
+    import oracle
+
+    def u16(t):
+        return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+    idx = torch.from_numpy(rows).long()
+    qr = q[idx[:, 0], idx[:, 2], idx[:, 1]]
+    t0 = time.perf_counter()
+    oracle.attention(lay, u16(qr), u16(k), u16(v), rows)
+    return time.perf_counter() - t0
+
+
+def cpu_values(wl):
+    """(q, k, v) on the host for the oracle (drawn on the GPU when the workload's
+    recipe says so, then copied back)."""
+    import torch
+    dev = wl.value_device if (wl.value_device == "cpu" or torch.cuda.is_available()) else "cpu"
+    q, k, v = wl.materialize(dev)
+    return q.cpu(), k.cpu(), v.cpu()
+
+
+def run_reference(args, rank, world):
+    """The fp64 oracle on a bounded row sample per step (rank 0 only)."""
+    if rank != 0:
+        return 0
+    from head_aware_paged_prefill_b200 import synth
+    wl = synth.CONFIGS[args.config]()
+    lay = wl.layout
+    q, k, v = cpu_values(wl)
+    cores = os.cpu_count() or 1
+    # size the per-step sample so one step takes about args.ref_step_s seconds
+    rows, pairs = _oracle_sample_rows(lay, 64, seed=0)
+    dt = _time_oracle(lay, q, k, v, rows)
+    n_rows = int(max(16, min(4096, 64 * args.ref_step_s / max(dt, 1e-3))))
+    tot_t, tot_pairs = 0.0, 0
+    for s in range(args.warmup + args.steps):
+        rows, pairs = _oracle_sample_rows(lay, n_rows, seed=1 + s)
+        dt = _time_oracle(lay, q, k, v, rows)
+        if s >= args.warmup:
+            tot_t += dt
+            tot_pairs += pairs
+    value = 4 * lay.d * tot_pairs / tot_t / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "step": f"oracle on {n_rows} sampled rows"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{n_rows} seeded (layer, q head, row) samples per step, "
+                                   f"{args.steps} steps"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default="cfg2")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-sample-rows", type=int, default=2048)
+    ap.add_argument("--ref-step-s", type=float, default=0.25)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+    import torch.distributed as dist
+    from head_aware_paged_prefill_b200 import metrics, synth
+    from head_aware_paged_prefill_b200.api import SegPagedPrefill
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+
+    wl = synth.CONFIGS[args.config]()
+    lay = wl.layout
+    q, k, v = wl.materialize(str(dev))
+    pre = SegPagedPrefill(lay, dev)
+    pre.load(q, k, v)
+    flops = metrics.attention_flops(lay)
+    tokens = lay.total_tokens * lay.n_layers
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    for _ in range(args.warmup):
+        pre.compute()
+    torch.cuda.synchronize()
+    st = pre.status()
+    if st != 0:
+        raise SystemExit(f"device error word {st:#x} after warm-up")
+
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    ev3 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(K)]
+    sampler = ClockSampler(_gpu_id(torch, dev))
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for s in range(K):
+        flush.zero_()
+        ev[s][0].record(stream)
+        pre.compute(k3_events=ev3[s])
+        ev[s][1].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    k3_ms = [a.elapsed_time(b) for a, b in ev3]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    st = pre.status()
+    if st != 0:
+        raise SystemExit(f"device error word {st:#x} after the timed steps")
+    ms_per_step = total_ms / K
+    value = world * flops * K / (total_ms * 1e-3) / 1e12
+
+    # end to end through the public API: pinned host inputs in, o back to host
+    q_h = q.cpu().pin_memory()
+    k_h = k.cpu().pin_memory()
+    v_h = v.cpu().pin_memory()
+    o_h = torch.empty(pre.o.shape, dtype=pre.o.dtype, pin_memory=True)
+    for _ in range(2):
+        pre.run(q_h, k_h, v_h, out="host", host_out=o_h)
+    torch.cuda.synchronize()
+    E = args.e2e_steps
+    e2e_ms = 0.0
+    for _ in range(E):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        pre.run(q_h, k_h, v_h, out="host", host_out=o_h)
+        b.record(stream)
+        b.synchronize()
+        e2e_ms += a.elapsed_time(b)
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * flops * E / (e2e_ms * 1e-3) / 1e12
+    h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h))
+    d2h = o_h.numel() * o_h.element_size()
+
+    peaks, peak_kind = _peaks()
+    k3_mean = statistics.mean(k3_ms)
+    achieved = flops / (k3_mean * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    traffic = _recorded_traffic("segpaged_prefill_kernel", wl.name)
+
+    cpu_baseline = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
+        rows, pairs = _oracle_sample_rows(lay, args.cpu_sample_rows, seed=0)
+        dt = _time_oracle(lay, qc, kc, vc, rows)
+        cpu_baseline = {"value": 4 * lay.d * pairs / dt / 1e12, "unit": UNIT,
+                        "cores": os.cpu_count() or 1, "kind": "oracle",
+                        "sample": f"{args.cpu_sample_rows} seeded (layer, q head, row) samples "
+                                  f"of the same workload, {pairs} visible pairs, {dt:.1f} s"}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "layers": lay.n_layers, "seq_len": lay.total_tokens,
+                   "heads": f"Hq {lay.hq} / Hkv {lay.hkv}", "head_dim": lay.d,
+                   "page_size": lay.p, "visible_pairs": flops // (4 * lay.d),
+                   "parallelism": f"replicas x{world}",
+                   "l2": "flushed between timed steps (256 MiB write)"},
+        "pct_bf16_peak": 100.0 * value / world / peak,
+        "pct_bf16_spec": 100.0 * value / world / SPEC_BF16_TFLOPS,
+        "tokens_per_s": world * tokens * K / (total_ms * 1e-3),
+        "roofline": {"bound": "tensor", "kernel": "segpaged_prefill_kernel",
+                     "achieved": achieved, "peak": peak, "unit": UNIT, "frac": achieved / peak,
+                     "peak_kind": f"bf16 burst, {peak_kind}", "traffic": traffic,
+                     "k3_ms": k3_mean},
+        "cpu_baseline": cpu_baseline,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / E},
+        "gpu_launches": K * pre.launches_per_run,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

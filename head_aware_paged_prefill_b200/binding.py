@@ -1,0 +1,195 @@
+"""ctypes binding of librk.so (the C ABI declared in include/rk.h).
+
+Argument marshalling only: every step of the path runs in the library's
+CUDA kernels.  PyTorch supplies device memory and the current stream.  If the
+library is missing, every call raises; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "librk.so")
+
+RK_OK, RK_ERR_INVALID_ARG, RK_ERR_UNALIGNED, RK_ERR_CAPACITY, RK_ERR_CUDA, RK_ERR_DEVICE = range(6)
+RK_DEV_BAD_PAGE, RK_DEV_TIMEOUT, RK_DEV_CAPACITY = 1, 2, 4
+STATUS_NAMES = {0: "RK_OK", 1: "RK_ERR_INVALID_ARG", 2: "RK_ERR_UNALIGNED", 3: "RK_ERR_CAPACITY",
+                4: "RK_ERR_CUDA", 5: "RK_ERR_DEVICE"}
+
+
+class RkError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
+        self.status = status
+
+
+class RkDims(ctypes.Structure):
+    _fields_ = [("n_req", ctypes.c_int32), ("n_layers", ctypes.c_int32),
+                ("num_q_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("page_size", ctypes.c_int32),
+                ("n_pages", ctypes.c_int64), ("total_tokens", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
+
+
+class RkLayout(ctypes.Structure):
+    _fields_ = [("n_segments", ctypes.c_int32), ("segments", ctypes.c_void_p),
+                ("page_base", ctypes.c_void_p), ("cu_seqlens", ctypes.c_void_p),
+                ("class_map", ctypes.c_void_p), ("class_window", ctypes.c_void_p),
+                ("retr_indptr", ctypes.c_void_p), ("retr_pages", ctypes.c_void_p)]
+
+
+class RkVisible(ctypes.Structure):
+    _fields_ = [("entries", ctypes.c_void_p), ("entry_start", ctypes.c_void_p),
+                ("entry_count", ctypes.c_void_p), ("ranges", ctypes.c_void_p),
+                ("range_start", ctypes.c_void_p), ("range_count", ctypes.c_void_p),
+                ("entry_capacity", ctypes.c_int64), ("range_capacity", ctypes.c_int64)]
+
+
+class RkSizes(ctypes.Structure):
+    _fields_ = [("n_tables", ctypes.c_int64), ("entry_capacity", ctypes.c_int64),
+                ("range_capacity", ctypes.c_int64), ("item_capacity", ctypes.c_int64),
+                ("workspace_bytes", ctypes.c_int64)]
+
+
+EXPORTS = ("rk_query_sizes", "rk_select_visible", "rk_relocate_rope", "rk_segpaged_prefill",
+           "rk_get_device_status")
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Loads librk.so; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m head_aware_paged_prefill_b200.csrc.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+        L.rk_query_sizes.argtypes = [vp, vp, vp]
+        L.rk_select_visible.argtypes = [vp, vp, vp, vp, ctypes.c_size_t, vp]
+        L.rk_relocate_rope.argtypes = [vp, vp, vp, i32, i64, i32, i32, ctypes.c_double, vp, vp]
+        L.rk_segpaged_prefill.argtypes = [vp, vp, vp, vp, vp, i32, ctypes.c_double, ctypes.c_float,
+                                          vp, vp, vp, ctypes.c_size_t, vp]
+        L.rk_get_device_status.argtypes = [vp, vp, vp]
+        for name in EXPORTS:
+            getattr(L, name).restype = i32
+        _lib = L
+    return _lib
+
+
+def _check(status: int, where: str):
+    if status != RK_OK:
+        raise RkError(status, where)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+class HostLayout:
+    """ctypes view of a host-side layout (an object with the attributes of
+    ``synth.Layout``).  Keeps the contiguous arrays it points into alive."""
+
+    def __init__(self, lay):
+        self.lay = lay
+        seg = np.ascontiguousarray(lay.segments, dtype=np.int32).reshape(-1, 5)
+        pb = np.ascontiguousarray(lay.page_base, dtype=np.int32)
+        cu = np.ascontiguousarray(lay.cu_seqlens, dtype=np.int32)
+        cm = np.ascontiguousarray(lay.class_map, dtype=np.int8)
+        cw = np.ascontiguousarray(lay.class_window, dtype=np.int32)
+        ri = np.ascontiguousarray(lay.retr_indptr, dtype=np.int32)
+        rp = np.ascontiguousarray(np.concatenate([np.asarray(lay.retr_pages, np.int32),
+                                                  np.zeros(1, np.int32)]))
+        self._keep = (seg, pb, cu, cm, cw, ri, rp)
+        self.layout = RkLayout(seg.shape[0], seg.ctypes.data, pb.ctypes.data, cu.ctypes.data,
+                               cm.ctypes.data, cw.ctypes.data, ri.ctypes.data, rp.ctypes.data)
+        self.dims = RkDims(lay.n_req, lay.n_layers, lay.hq, lay.hkv, lay.d, lay.p, lay.n_pages,
+                           int(cu[-1]), 0)
+
+    def sizes(self) -> RkSizes:
+        s = RkSizes()
+        _check(lib().rk_query_sizes(ctypes.byref(self.dims), ctypes.byref(self.layout),
+                                    ctypes.byref(s)), "rk_query_sizes")
+        return s
+
+
+class Visible:
+    """Device buffers of rk_visible, sized by rk_query_sizes."""
+
+    def __init__(self, sizes: RkSizes, device):
+        nt = max(1, int(sizes.n_tables))
+        dev = torch.device(device)
+        self.entries = torch.zeros((max(1, int(sizes.entry_capacity)), 4), dtype=torch.int32,
+                                   device=dev)
+        self.entry_start = torch.zeros(nt, dtype=torch.int32, device=dev)
+        self.entry_count = torch.zeros(nt, dtype=torch.int32, device=dev)
+        self.ranges = torch.zeros((max(1, int(sizes.range_capacity)), 2), dtype=torch.int32,
+                                  device=dev)
+        self.range_start = torch.zeros(nt, dtype=torch.int32, device=dev)
+        self.range_count = torch.zeros(nt, dtype=torch.int32, device=dev)
+        self.struct = RkVisible(self.entries.data_ptr(), self.entry_start.data_ptr(),
+                                self.entry_count.data_ptr(), self.ranges.data_ptr(),
+                                self.range_start.data_ptr(), self.range_count.data_ptr(),
+                                self.entries.shape[0], self.ranges.shape[0])
+
+    def tables(self):
+        """Per-table (entries [n, 4], ranges [m, 2]) as numpy, in table order."""
+        es, ec = self.entry_start.cpu().numpy(), self.entry_count.cpu().numpy()
+        rs, rc = self.range_start.cpu().numpy(), self.range_count.cpu().numpy()
+        E, R = self.entries.cpu().numpy(), self.ranges.cpu().numpy()
+        return ([E[a:a + n] for a, n in zip(es, ec)], [R[a:a + n] for a, n in zip(rs, rc)])
+
+
+def workspace(sizes: RkSizes, device) -> torch.Tensor:
+    # torch's caching allocator returns 512-byte aligned blocks
+    return torch.zeros(int(sizes.workspace_bytes), dtype=torch.uint8, device=torch.device(device))
+
+
+def select_visible(hl: HostLayout, vis: Visible, ws: torch.Tensor, stream=None):
+    _check(lib().rk_select_visible(ctypes.byref(hl.dims), ctypes.byref(hl.layout),
+                                   ctypes.byref(vis.struct), _ptr(ws), ws.numel(),
+                                   _stream(stream)), "rk_select_visible")
+
+
+def relocate_rope(k_src: torch.Tensor, k_dst: torch.Tensor, jobs: torch.Tensor, theta: float,
+                  device_error: Optional[torch.Tensor] = None, stream=None):
+    n_pages, p, d = k_src.shape
+    assert k_dst.shape == k_src.shape and k_src.dtype == torch.bfloat16
+    assert jobs.dtype == torch.int32 and jobs.is_contiguous()
+    _check(lib().rk_relocate_rope(_ptr(k_src), _ptr(k_dst), _ptr(jobs), jobs.shape[0], n_pages,
+                                  p, d, float(theta), _ptr(device_error), _stream(stream)),
+           "rk_relocate_rope")
+
+
+def segpaged_prefill(hl: HostLayout, q: torch.Tensor, k_pool: torch.Tensor,
+                     v_pool: torch.Tensor, vis: Visible, ws: torch.Tensor, o: torch.Tensor,
+                     lse: Optional[torch.Tensor] = None, fuse_rope: bool = False,
+                     stream=None):
+    lay = hl.lay
+    for t in (q, k_pool, v_pool, o):
+        assert t.dtype == torch.bfloat16 and t.is_contiguous()
+    _check(lib().rk_segpaged_prefill(ctypes.byref(hl.dims), _ptr(q), _ptr(k_pool), _ptr(v_pool),
+                                     ctypes.byref(vis.struct), 1 if fuse_rope else 0,
+                                     float(lay.theta), float(lay.softmax_scale), _ptr(o),
+                                     _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)),
+           "rk_segpaged_prefill")
+
+
+def device_status(ws: torch.Tensor, stream=None) -> int:
+    v = ctypes.c_int32(0)
+    st = lib().rk_get_device_status(_ptr(ws), ctypes.byref(v), _stream(stream))
+    if st not in (RK_OK, RK_ERR_DEVICE):
+        raise RkError(st, "rk_get_device_status")
+    return int(v.value)

@@ -1,0 +1,338 @@
+// C-ABI entry points of librk.so: argument validation, workspace layout,
+// tensor-map set-up and kernel launches.  Every check that can be done on the
+// host is done here, synchronously, before any GPU work is enqueued.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+#include <vector>
+
+#include "rk_internal.h"
+
+namespace rk {
+
+cudaError_t launch_select(LayoutView* lv_dev, int n_tables, const rk_visible& vis, WsHeader* hdr,
+                          Item* items_tmp, Item* items, cudaStream_t stream);
+cudaError_t launch_relocate(const void* k_src, void* k_dst, const int32_t* jobs, int n_jobs,
+                            int64_t n_pages, int P, int D, double theta, int* device_error,
+                            cudaStream_t stream);
+
+cudaError_t launch_prefill_args(const PrefillLaunchArgs& a, cudaStream_t stream);
+
+namespace {
+
+constexpr int64_t kMaxI32 = 2147483647;
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+rk_status check_dims(const rk_dims* d) {
+  if (!d) return RK_ERR_INVALID_ARG;
+  if (d->n_req < 1 || d->n_layers < 1 || d->num_kv_heads < 1 || d->num_q_heads < 1)
+    return RK_ERR_INVALID_ARG;
+  if (d->num_q_heads % d->num_kv_heads != 0) return RK_ERR_INVALID_ARG;
+  if (d->head_dim != 64 && d->head_dim != 128) return RK_ERR_INVALID_ARG;
+  if (d->page_size != 16 && d->page_size != 64) return RK_ERR_INVALID_ARG;
+  if (d->n_pages < 1 || d->n_pages * d->page_size + kKeysPerTile >= kMaxI32)
+    return RK_ERR_INVALID_ARG;
+  if (d->total_tokens < 0 || d->reserved != 0) return RK_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(d->n_layers) * d->total_tokens + kRowsPerTile >= kMaxI32)
+    return RK_ERR_INVALID_ARG;
+  return RK_OK;
+}
+
+// Everything derived from a validated layout.
+struct Derived {
+  int64_t n_tables = 0, n_lh = 0, total_pages = 0;
+  int64_t entry_capacity = 0, range_capacity = 0, item_capacity = 0;
+  std::vector<int32_t> seg_indptr, page_prefix;
+  bool any_retrieval = false;
+  int64_t n_retr = 0;
+  WsMap map;
+  int32_t layout_words = 0;
+};
+
+rk_status check_layout(const rk_dims* d, const rk_layout* lay, Derived* out) {
+  if (!lay) return RK_ERR_INVALID_ARG;
+  if (lay->n_segments < 0) return RK_ERR_INVALID_ARG;
+  if ((lay->n_segments > 0 && (!lay->segments || !lay->page_base)) || !lay->cu_seqlens ||
+      !lay->class_map || !lay->class_window)
+    return RK_ERR_INVALID_ARG;
+  const int n_req = d->n_req, P = d->page_size;
+  const int64_t n_lh = static_cast<int64_t>(d->n_layers) * d->num_kv_heads;
+  out->n_lh = n_lh;
+  out->n_tables = n_lh * n_req;
+  if (out->n_tables >= kMaxI32 / 4) return RK_ERR_INVALID_ARG;
+  const int32_t* cu = lay->cu_seqlens;
+  if (cu[0] != 0) return RK_ERR_INVALID_ARG;
+  for (int r = 0; r < n_req; ++r)
+    if (cu[r + 1] < cu[r]) return RK_ERR_INVALID_ARG;
+  if (cu[n_req] != d->total_tokens) return RK_ERR_INVALID_ARG;
+  bool any_local = false;
+  for (int64_t k = 0; k < n_lh; ++k) {
+    const int c = lay->class_map[k];
+    if (c < RK_GLOBAL || c > RK_DENSE) return RK_ERR_INVALID_ARG;
+    any_local |= c == RK_LOCAL;
+    out->any_retrieval |= c == RK_RETRIEVAL;
+  }
+  if (any_local && lay->class_window[RK_LOCAL] < 1) return RK_ERR_INVALID_ARG;
+  // segments: grouped by request, tiling [0, L_r) in order
+  out->seg_indptr.assign(n_req + 1, 0);
+  int prev_req = -1, expect = 0;
+  for (int s = 0; s < lay->n_segments; ++s) {
+    const rk_segment& g = lay->segments[s];
+    if (g.req < 0 || g.req >= n_req || g.len < 1 || (g.cached != 0 && g.cached != 1))
+      return RK_ERR_INVALID_ARG;
+    if (g.req != prev_req) {
+      if (g.req < prev_req) return RK_ERR_INVALID_ARG;
+      if (prev_req >= 0 && expect != cu[prev_req + 1] - cu[prev_req]) return RK_ERR_INVALID_ARG;
+      for (int r = prev_req + 1; r < g.req; ++r)
+        if (cu[r + 1] != cu[r]) return RK_ERR_INVALID_ARG;  // skipped request must be empty
+      prev_req = g.req;
+      expect = 0;
+    }
+    if (g.logical_start != expect) return RK_ERR_INVALID_ARG;
+    const int L = cu[g.req + 1] - cu[g.req];
+    if (static_cast<int64_t>(g.logical_start) + g.len > L) return RK_ERR_INVALID_ARG;
+    const int64_t delta = static_cast<int64_t>(g.logical_start) - g.stored_pos_base;
+    if (g.cached && (delta > kMaxI32 || delta < -kMaxI32)) return RK_ERR_INVALID_ARG;
+    const bool last = g.logical_start + g.len == L;
+    if (!last && g.len % P != 0) return RK_ERR_UNALIGNED;
+    const int64_t npg = (g.len + P - 1) / P;
+    for (int64_t lh = 0; lh < n_lh; ++lh) {
+      const int64_t b = lay->page_base[s * n_lh + lh];
+      if (b < 0 || b + npg > d->n_pages) return RK_ERR_INVALID_ARG;
+    }
+    expect += g.len;
+    out->seg_indptr[g.req + 1] = s + 1;
+  }
+  if (prev_req >= 0 && expect != cu[prev_req + 1] - cu[prev_req]) return RK_ERR_INVALID_ARG;
+  for (int r = prev_req + 1; r < n_req; ++r)
+    if (cu[r + 1] != cu[r]) return RK_ERR_INVALID_ARG;
+  for (int r = 0; r < n_req; ++r)  // empty requests keep their predecessor's end
+    if (out->seg_indptr[r + 1] < out->seg_indptr[r]) out->seg_indptr[r + 1] = out->seg_indptr[r];
+  // retrieval lists
+  if (out->any_retrieval && !lay->retr_indptr) return RK_ERR_INVALID_ARG;
+  if (lay->retr_indptr) {
+    if (lay->retr_indptr[0] != 0) return RK_ERR_INVALID_ARG;
+    for (int64_t t = 0; t < out->n_tables; ++t)
+      if (lay->retr_indptr[t + 1] < lay->retr_indptr[t]) return RK_ERR_INVALID_ARG;
+    out->n_retr = lay->retr_indptr[out->n_tables];
+    if (out->n_retr > 0 && !lay->retr_pages) return RK_ERR_INVALID_ARG;
+    if (out->n_retr >= kMaxI32 / 4) return RK_ERR_INVALID_ARG;
+  }
+  // sizes
+  out->page_prefix.assign(n_req + 1, 0);
+  const int G = d->num_q_heads / d->num_kv_heads;
+  const int64_t npairs = (G + 1) / 2;
+  int64_t items = 0;
+  for (int r = 0; r < n_req; ++r) {
+    const int64_t L = cu[r + 1] - cu[r];
+    out->page_prefix[r + 1] =
+        static_cast<int32_t>(out->page_prefix[r] + (L + P - 1) / P);
+    const int64_t nseg = out->seg_indptr[r + 1] - out->seg_indptr[r];
+    items += n_lh * npairs * (L / kRowsPerTile + 1 + nseg);
+  }
+  out->total_pages = out->page_prefix[n_req];
+  out->entry_capacity = n_lh * out->total_pages;
+  out->range_capacity = n_lh * lay->n_segments;
+  out->item_capacity = items;
+  if (out->entry_capacity >= kMaxI32 || out->range_capacity >= kMaxI32 ||
+      out->item_capacity >= kMaxI32 / 2)
+    return RK_ERR_INVALID_ARG;
+  // workspace map
+  const int64_t words_fixed = (sizeof(LayoutView) + 3) / 4;
+  const int64_t words = words_fixed + 5 * static_cast<int64_t>(lay->n_segments) + (n_req + 1) +
+                        lay->n_segments * n_lh + (n_req + 1) + (n_req + 1) + n_lh +
+                        (out->n_tables + 1) + out->n_retr + (out->n_tables + 1) + 8;
+  if (words >= kMaxI32) return RK_ERR_INVALID_ARG;
+  out->layout_words = static_cast<int32_t>(words);
+  WsMap& m = out->map;
+  m.header = 0;
+  m.items = sizeof(WsHeader);
+  m.items_tmp = align_up(m.items + sizeof(Item) * out->item_capacity, 256);
+  m.layout = align_up(m.items_tmp + sizeof(Item) * out->item_capacity, 256);
+  m.total = align_up(m.layout + 4 * static_cast<size_t>(words), 256);
+  return RK_OK;
+}
+
+// Host image of the workspace's header + layout block.
+void build_layout_image(const rk_dims* d, const rk_layout* lay, const Derived& dv,
+                        std::vector<int32_t>* img) {
+  img->assign(dv.layout_words, 0);
+  LayoutView v{};
+  v.n_req = d->n_req;
+  v.n_layers = d->n_layers;
+  v.hq = d->num_q_heads;
+  v.hkv = d->num_kv_heads;
+  v.d = d->head_dim;
+  v.p = d->page_size;
+  v.n_seg = lay->n_segments;
+  v.n_retr = static_cast<int32_t>(dv.n_retr);
+  v.n_pages = d->n_pages;
+  v.total_tokens = d->total_tokens;
+  v.total_pages = static_cast<int32_t>(dv.total_pages);
+  v.window = lay->class_window[RK_LOCAL];
+  v.item_capacity = static_cast<int32_t>(dv.item_capacity);
+  int32_t off = static_cast<int32_t>((sizeof(LayoutView) + 3) / 4);
+  int32_t* w = img->data();
+  v.off_seg = off;
+  for (int s = 0; s < lay->n_segments; ++s) {
+    const rk_segment& g = lay->segments[s];
+    w[off + 5 * s + 0] = g.req;
+    w[off + 5 * s + 1] = g.logical_start;
+    w[off + 5 * s + 2] = g.len;
+    w[off + 5 * s + 3] = g.cached ? g.stored_pos_base : g.logical_start;
+    w[off + 5 * s + 4] = g.cached;
+  }
+  off += 5 * lay->n_segments;
+  v.off_seg_indptr = off;
+  for (int r = 0; r <= d->n_req; ++r) w[off + r] = dv.seg_indptr[r];
+  off += d->n_req + 1;
+  v.off_page_base = off;
+  if (lay->n_segments > 0)
+    std::memcpy(w + off, lay->page_base, 4 * static_cast<size_t>(lay->n_segments) * dv.n_lh);
+  off += static_cast<int32_t>(lay->n_segments * dv.n_lh);
+  v.off_cu = off;
+  for (int r = 0; r <= d->n_req; ++r) w[off + r] = lay->cu_seqlens[r];
+  off += d->n_req + 1;
+  v.off_page_prefix = off;
+  for (int r = 0; r <= d->n_req; ++r) w[off + r] = dv.page_prefix[r];
+  off += d->n_req + 1;
+  v.off_class = off;
+  for (int64_t k = 0; k < dv.n_lh; ++k) w[off + k] = lay->class_map[k];
+  off += static_cast<int32_t>(dv.n_lh);
+  v.off_retr_indptr = off;
+  for (int64_t t = 0; t <= dv.n_tables; ++t) w[off + t] = lay->retr_indptr ? lay->retr_indptr[t] : 0;
+  off += static_cast<int32_t>(dv.n_tables + 1);
+  v.off_retr_pages = off;
+  if (dv.n_retr > 0) std::memcpy(w + off, lay->retr_pages, 4 * static_cast<size_t>(dv.n_retr));
+  off += static_cast<int32_t>(dv.n_retr);
+  v.off_tile_prefix = off;
+  off += static_cast<int32_t>(dv.n_tables + 1);
+  v.layout_words = off;
+  std::memcpy(w, &v, sizeof(LayoutView));
+}
+
+}  // namespace
+}  // namespace rk
+
+using namespace rk;
+
+extern "C" rk_status rk_query_sizes(const rk_dims* dims, const rk_layout* layout, rk_sizes* out) {
+  if (!out) return RK_ERR_INVALID_ARG;
+  rk_status st = check_dims(dims);
+  if (st != RK_OK) return st;
+  Derived dv;
+  if ((st = check_layout(dims, layout, &dv)) != RK_OK) return st;
+  out->n_tables = dv.n_tables;
+  out->entry_capacity = dv.entry_capacity;
+  out->range_capacity = dv.range_capacity;
+  out->item_capacity = dv.item_capacity;
+  out->workspace_bytes = static_cast<int64_t>(dv.map.total);
+  return RK_OK;
+}
+
+extern "C" rk_status rk_select_visible(const rk_dims* dims, const rk_layout* layout,
+                                       const rk_visible* out, void* workspace,
+                                       size_t workspace_bytes, void* stream) {
+  rk_status st = check_dims(dims);
+  if (st != RK_OK) return st;
+  Derived dv;
+  if ((st = check_layout(dims, layout, &dv)) != RK_OK) return st;
+  if (!out || !workspace || !out->entries || !out->entry_start || !out->entry_count ||
+      !out->ranges || !out->range_start || !out->range_count)
+    return RK_ERR_INVALID_ARG;
+  if (!aligned(workspace, 256) || !aligned(out->entries, 16) || !aligned(out->ranges, 8) ||
+      !aligned(out->entry_start, 4) || !aligned(out->entry_count, 4) ||
+      !aligned(out->range_start, 4) || !aligned(out->range_count, 4))
+    return RK_ERR_INVALID_ARG;
+  if (out->entry_capacity < dv.entry_capacity || out->range_capacity < dv.range_capacity ||
+      workspace_bytes < dv.map.total)
+    return RK_ERR_CAPACITY;
+  // header + layout image, one host-to-device copy each
+  WsHeader hdr{};
+  hdr.n_tables = static_cast<int32_t>(dv.n_tables);
+  hdr.item_capacity = static_cast<int32_t>(dv.item_capacity);
+  std::vector<int32_t> img;
+  build_layout_image(dims, layout, dv, &img);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (cudaMemcpyAsync(ws, &hdr, sizeof hdr, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return RK_ERR_CUDA;
+  if (cudaMemcpyAsync(ws + dv.map.layout, img.data(), 4 * img.size(), cudaMemcpyHostToDevice, s) !=
+      cudaSuccess)
+    return RK_ERR_CUDA;
+  cudaError_t e = launch_select(reinterpret_cast<LayoutView*>(ws + dv.map.layout),
+                                static_cast<int>(dv.n_tables), *out,
+                                reinterpret_cast<WsHeader*>(ws),
+                                reinterpret_cast<Item*>(ws + dv.map.items_tmp),
+                                reinterpret_cast<Item*>(ws + dv.map.items), s);
+  return e == cudaSuccess ? RK_OK : RK_ERR_CUDA;
+}
+
+extern "C" rk_status rk_relocate_rope(const void* k_src, void* k_dst, const int32_t* jobs,
+                                      int32_t n_jobs, int64_t n_pages, int32_t page_size,
+                                      int32_t head_dim, double rope_theta, int32_t* device_error,
+                                      void* stream) {
+  if (n_jobs < 0 || n_pages < 1 || page_size < 1 || (head_dim != 64 && head_dim != 128))
+    return RK_ERR_INVALID_ARG;
+  if (!(rope_theta > 0.0) || !std::isfinite(rope_theta)) return RK_ERR_INVALID_ARG;
+  if (n_jobs > 0 && (!k_src || !k_dst || !jobs)) return RK_ERR_INVALID_ARG;
+  if (!aligned(k_src, 16) || !aligned(k_dst, 16) || !aligned(jobs, 4) ||
+      !aligned(device_error, 4))
+    return RK_ERR_INVALID_ARG;
+  cudaError_t e = launch_relocate(k_src, k_dst, jobs, n_jobs, n_pages, page_size, head_dim,
+                                  rope_theta, device_error, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? RK_OK : RK_ERR_CUDA;
+}
+
+extern "C" rk_status rk_segpaged_prefill(const rk_dims* dims, const void* q, const void* k_pool,
+                                         const void* v_pool, const rk_visible* vis,
+                                         int32_t fuse_rope, double rope_theta, float softmax_scale,
+                                         void* o, float* lse, void* workspace,
+                                         size_t workspace_bytes, void* stream) {
+  rk_status st = check_dims(dims);
+  if (st != RK_OK) return st;
+  if (!q || !k_pool || !v_pool || !vis || !vis->entries || !o || !workspace)
+    return RK_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k_pool, 16) || !aligned(v_pool, 16) || !aligned(o, 16) ||
+      !aligned(vis->entries, 16) || !aligned(workspace, 256) || !aligned(lse, 4))
+    return RK_ERR_INVALID_ARG;
+  if (fuse_rope != 0 && fuse_rope != 1) return RK_ERR_INVALID_ARG;
+  if (fuse_rope == 1) return RK_ERR_INVALID_ARG;  // fused relocation: not built yet
+  if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return RK_ERR_INVALID_ARG;
+  if (workspace_bytes < sizeof(WsHeader)) return RK_ERR_CAPACITY;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
+  PrefillLaunchArgs a;
+  a.q = q;
+  a.k_pool = k_pool;
+  a.v_pool = v_pool;
+  a.n_layers = dims->n_layers;
+  a.hq = dims->num_q_heads;
+  a.d = dims->head_dim;
+  a.p = dims->page_size;
+  a.n_pages = dims->n_pages;
+  a.total_tokens = dims->total_tokens;
+  a.items = reinterpret_cast<const Item*>(ws + sizeof(WsHeader));
+  a.n_items = &hdr->n_items;
+  a.error_word = &hdr->error;
+  a.timeout_site = &hdr->timeout_site;
+  a.entries = vis->entries;
+  a.o = o;
+  a.lse = lse;
+  a.scale_log2 = softmax_scale * 1.4426950408889634f;
+  if (dims->total_tokens == 0) return RK_OK;
+  cudaError_t e = launch_prefill_args(a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? RK_OK : RK_ERR_CUDA;
+}
+
+extern "C" rk_status rk_get_device_status(const void* workspace, int32_t* status, void* stream) {
+  if (!workspace || !status) return RK_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return RK_ERR_CUDA;
+  int32_t v = 0;
+  if (cudaMemcpy(&v, workspace, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess)
+    return RK_ERR_CUDA;
+  *status = v;
+  return v == 0 ? RK_OK : RK_ERR_DEVICE;
+}

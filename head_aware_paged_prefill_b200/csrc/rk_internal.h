@@ -1,0 +1,93 @@
+// Internal layout of the workspace and the work list shared by the
+// library's translation units.  Not part of the C ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/rk.h"
+
+namespace rk {
+
+constexpr int kRowsPerTile = 128;  // query rows per Q tile (one TMEM lane per row)
+constexpr int kKeysPerTile = 128;  // keys per KV tile (N of the QK^T MMA)
+
+// Workspace header (first 256 bytes of the workspace).
+struct WsHeader {
+  int32_t error;          // RK_DEV_* bits, reset by rk_select_visible
+  int32_t n_items;        // attention work items written by the select kernels
+  int32_t n_tables;
+  int32_t item_capacity;
+  int32_t timeout_site;   // first bounded wait that gave up (diagnostics)
+  int32_t pad[59];
+};
+static_assert(sizeof(WsHeader) == 256, "header size");
+
+// One attention work item: up to two q heads of one kv head over the same
+// block of <= 128 rows, hence the same visible keys (GQA sharing).
+struct Item {
+  int32_t q_row0;     // layer * T + first token of the request
+  int32_t row_begin;  // request-local rows [row_begin, row_end)
+  int32_t row_end;
+  int32_t e_begin;    // entries [e_begin, e_end) of the rk_visible arrays
+  int32_t e_end;
+  int32_t qh0;        // first q head
+  int32_t nh;         // 1 or 2 q heads
+  int32_t window;     // key window (local class), -1 = unbounded
+  int32_t layer;
+  int32_t req;
+  int32_t table;
+  int32_t cost;       // KV tiles
+};
+static_assert(sizeof(Item) == 48, "item size");
+
+// Layout copy inside the workspace, as written by the host (all int32).
+struct LayoutView {
+  int32_t n_req, n_layers, hq, hkv, d, p, n_seg, n_retr;
+  int64_t n_pages;
+  int32_t total_tokens, total_pages;  // total_pages = sum_r ceil(L_r / P)
+  int32_t window;                     // class_window[RK_LOCAL]
+  int32_t item_capacity;
+  // offsets (in int32 elements from the start of the layout block)
+  int32_t off_seg;          // [n_seg][5]
+  int32_t off_seg_indptr;   // [n_req + 1]
+  int32_t off_page_base;    // [n_seg][n_layers * hkv]
+  int32_t off_cu;           // [n_req + 1]
+  int32_t off_page_prefix;  // [n_req + 1]
+  int32_t off_class;        // [n_layers * hkv]
+  int32_t off_retr_indptr;  // [n_tables + 1]
+  int32_t off_retr_pages;   // [n_retr]
+  int32_t off_tile_prefix;  // [n_tables + 1] scratch: items per table, scanned
+  int32_t layout_words;
+};
+
+// Workspace map (byte offsets), computed on the host.
+struct WsMap {
+  size_t header = 0;
+  size_t items = 0;      // Item[item_capacity], sorted by cost (longest first)
+  size_t items_tmp = 0;  // Item[item_capacity], unsorted
+  size_t layout = 0;     // LayoutView followed by the int32 arrays
+  size_t total = 0;
+};
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Arguments of one attention launch (device pointers).
+struct PrefillLaunchArgs {
+  const void* q;
+  const void* k_pool;
+  const void* v_pool;
+  int n_layers, hq, d, p;
+  int64_t n_pages;
+  int total_tokens;
+  const Item* items;
+  const int32_t* n_items;
+  int* error_word;
+  int* timeout_site;
+  const rk_entry* entries;
+  void* o;
+  float* lse;
+  float scale_log2;
+};
+
+}  // namespace rk

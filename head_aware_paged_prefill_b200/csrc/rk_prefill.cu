@@ -1,0 +1,516 @@
+// K3: SegPagedAttention prefill on sm_100a.
+//
+// RedKnot (paooo page, "technical principles"): KV is stored per head in
+// pages and a fused varlen kernel attends over exactly the pages each head
+// may see, with no attn_mask; global heads recompute every row causally,
+// local heads compute the uncached rows over a window of reused KV (README
+// excerpt, "Head Classification" and "SegPagedAttention Runtime").
+//
+// One CTA per SM, persistent over the work list of rk_select_visible.  A work
+// item is <= 128 rows of one request and up to two q heads of the same kv
+// head: both heads see identical pages, so each K/V tile loaded into shared
+// memory feeds two Q tiles.
+//
+//   warp 0      TMA producer: Q tiles (3-D box out of [rows][Hq][D]) and, per
+//               KV tile, one box per page and 64-column block out of the pool.
+//   warp 1      tcgen05 issuer and TMEM owner.  S_t = Q_t K^T (M=128, N=128,
+//               K=D) into TMEM; O_t += P_t V (M=128, N=D, K=128) with P_t read
+//               from TMEM and V from shared memory (MN-major operand).
+//   warps 2-5   softmax warpgroup of Q tile 0, warps 6-9 of Q tile 1: one
+//               TMEM lane (= one query row) per thread; online softmax in the
+//               log2 domain, O rescaled in TMEM only when the running max
+//               grows by more than 2^8, P written back over S as bf16.
+//
+// Invisible pages are never loaded: the item's entry range already excludes
+// them.  Element masks are evaluated only on tiles that straddle the causal
+// diagonal, a window start or a partial page.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "rk_internal.h"
+#include "sm100.cuh"
+
+namespace rk {
+
+constexpr int kPrefillThreads = 320;
+constexpr float kRescaleLog2 = 8.0f;
+
+template <int D, int P>
+struct PrefillCfg {
+  static constexpr int KB = D / 64;  // 128-byte column blocks of a row
+  static constexpr int kQTileBytes = kRowsPerTile * D * 2;
+  static constexpr int kKVTileBytes = kKeysPerTile * D * 2;
+  static constexpr int kBlockBytes = kKeysPerTile * 128;  // one column block of a tile
+  static constexpr int kStages = D == 128 ? 2 : 4;
+  static constexpr int EPT = kKeysPerTile / P;  // pages per KV tile
+  static constexpr int kDataBytes = 2 * kQTileBytes + 2 * kStages * kKVTileBytes;
+  static constexpr int kSmemBytes = kDataBytes + 1024 + 1024;
+  static constexpr uint32_t kTmemCols = 512;
+  // TMEM columns: S_t (fp32, P_t as bf16 over its first 64 columns) and O_t
+  __host__ __device__ static constexpr uint32_t col_s(int t) { return t ? 128u : 0u; }
+  __host__ __device__ static constexpr uint32_t col_o(int t) { return t ? 256u + D : 256u; }
+};
+
+struct PrefillParams {
+  const Item* items;
+  const int32_t* n_items;
+  int* error_word;
+  int* timeout_site;
+  const rk_entry* entries;
+  __nv_bfloat16* o;
+  float* lse;
+  int hq;
+  int total_tokens;
+  int64_t n_pages;
+  float scale_log2;
+};
+
+// barrier slots
+enum : int {
+  kBarQFull = 0,
+  kBarQEmpty = 1,
+  kBarSFull = 2,   // [2]
+  kBarPFull = 4,   // [2]
+  kBarOFull = 6,   // [2]
+  kBarOEmpty = 8,  // [2]
+  kBarDrain = 10,  // MMA completion before TMEM is released
+  kBarKFull = 11,  // [kStages] x 4 groups follow
+};
+
+template <int D, int P>
+__global__ void __launch_bounds__(kPrefillThreads, 1)
+    segpaged_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
+                            const __grid_constant__ CUtensorMap tm_k,
+                            const __grid_constant__ CUtensorMap tm_v, const PrefillParams prm) {
+  using C = PrefillCfg<D, P>;
+  constexpr int S = C::kStages;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sK = sQ + 2 * C::kQTileBytes;
+  uint8_t* sV = sK + S * C::kKVTileBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + S * C::kKVTileBytes);
+  uint64_t* k_full = bars + kBarKFull;
+  uint64_t* k_empty = k_full + S;
+  uint64_t* v_full = k_empty + S;
+  uint64_t* v_empty = v_full + S;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 64);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars[kBarQFull], 1);
+    mbar_init(&bars[kBarQEmpty], 1);
+    mbar_init(&bars[kBarDrain], 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&bars[kBarSFull + t], 1);
+      mbar_init(&bars[kBarPFull + t], 128);
+      mbar_init(&bars[kBarOFull + t], 1);
+      mbar_init(&bars[kBarOEmpty + t], 128);
+    }
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tm_q);
+    prefetch_tensormap(&tm_k);
+    prefetch_tensormap(&tm_v);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int n_items = *prm.n_items;
+  const WaitCtx wc{abort_flag, prm.error_word, prm.timeout_site};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t k_issued = 0, v_issued = 0, q_uses = 0;
+      bool ok = true;
+      const int32_t oob_row = static_cast<int32_t>(prm.n_pages * P);
+      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+        const Item w = prm.items[it];
+        const int n_tiles = (w.e_end - w.e_begin + C::EPT - 1) / C::EPT;
+        if (n_tiles == 0) continue;
+        if (q_uses > 0 && !(ok = mbar_wait(&bars[kBarQEmpty], (q_uses - 1) & 1, wc, 1))) break;
+        mbar_arrive_expect_tx(&bars[kBarQFull], w.nh * C::kQTileBytes);
+        for (int t = 0; t < w.nh; ++t)
+          for (int cb = 0; cb < C::KB; ++cb)
+            tma_load_3d(sQ + t * C::kQTileBytes + cb * C::kBlockBytes, &tm_q, &bars[kBarQFull],
+                        cb * 64, w.qh0 + t, w.q_row0 + w.row_begin);
+        ++q_uses;
+        for (int j = 0; j < n_tiles; ++j) {
+          int32_t rows[C::EPT];
+#pragma unroll
+          for (int e = 0; e < C::EPT; ++e) {
+            const int idx = w.e_begin + j * C::EPT + e;
+            rows[e] = oob_row;
+            if (idx < w.e_end) {
+              const int32_t pg = prm.entries[idx].phys_page;
+              if (pg >= 0 && pg < prm.n_pages) rows[e] = pg * P;
+              else atomicOr(prm.error_word, static_cast<int>(RK_DEV_BAD_PAGE));
+            }
+          }
+          {
+            const int st = k_issued % S;
+            const uint32_t u = k_issued / S;
+            if (u > 0 && !(ok = mbar_wait(&k_empty[st], (u - 1) & 1, wc, 2))) break;
+            mbar_arrive_expect_tx(&k_full[st], C::kKVTileBytes);
+#pragma unroll
+            for (int e = 0; e < C::EPT; ++e)
+#pragma unroll
+              for (int cb = 0; cb < C::KB; ++cb)
+                tma_load_2d(sK + st * C::kKVTileBytes + cb * C::kBlockBytes + e * P * 128, &tm_k,
+                            &k_full[st], cb * 64, rows[e]);
+            ++k_issued;
+          }
+          {
+            const int st = v_issued % S;
+            const uint32_t u = v_issued / S;
+            if (u > 0 && !(ok = mbar_wait(&v_empty[st], (u - 1) & 1, wc, 3))) break;
+            mbar_arrive_expect_tx(&v_full[st], C::kKVTileBytes);
+#pragma unroll
+            for (int e = 0; e < C::EPT; ++e)
+#pragma unroll
+              for (int cb = 0; cb < C::KB; ++cb)
+                tma_load_2d(sV + st * C::kKVTileBytes + cb * C::kBlockBytes + e * P * 128, &tm_v,
+                            &v_full[st], cb * 64, rows[e]);
+            ++v_issued;
+          }
+        }
+      }
+      if (!ok) {
+        // drain: let every copy this thread started land before the CTA exits
+        for (uint32_t k = (k_issued > S ? k_issued - S : 0); k < k_issued; ++k)
+          mbar_wait_drain(&k_full[k % S], (k / S) & 1);
+        for (uint32_t k = (v_issued > S ? v_issued - S : 0); k < v_issued; ++k)
+          mbar_wait_drain(&v_full[k % S], (k / S) & 1);
+        if (q_uses > 0) mbar_wait_drain(&bars[kBarQFull], (q_uses - 1) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // -------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(kRowsPerTile, kKeysPerTile, false);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(kRowsPerTile, D, true);
+      const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
+      uint32_t kv_iter = 0, q_uses = 0;
+      uint32_t p_phase[2] = {0, 0}, o_uses[2] = {0, 0};
+      bool ok = true;
+      auto issue_s = [&](int t, int st) {
+        const uint32_t d = tmem + C::col_s(t);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::kBlockBytes + (kk & 3) * 32;
+          const uint64_t a = desc_sw128(sQa + t * C::kQTileBytes + off, 16, 1024);
+          const uint64_t b = desc_sw128(sKa + st * C::kKVTileBytes + off, 16, 1024);
+          mma_bf16_ss(d, a, b, idesc_s, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int t, int st, bool acc) {
+        const uint32_t d = tmem + C::col_o(t);
+        const uint32_t a = tmem + C::col_s(t);
+#pragma unroll
+        for (int kk = 0; kk < kKeysPerTile / 16; ++kk) {
+          const uint64_t b =
+              desc_sw128(sVa + st * C::kKVTileBytes + kk * 16 * 128, C::kBlockBytes, 1024);
+          mma_bf16_ts(d, a + kk * 8, b, idesc_o, (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+        const Item w = prm.items[it];
+        const int n_tiles = (w.e_end - w.e_begin + C::EPT - 1) / C::EPT;
+        if (n_tiles == 0) continue;
+        if (!(ok = mbar_wait(&bars[kBarQFull], q_uses & 1, wc, 10))) break;
+        ++q_uses;
+        {
+          const int st = kv_iter % S;
+          if (!(ok = mbar_wait(&k_full[st], (kv_iter / S) & 1, wc, 11))) break;
+          tc_fence_after();
+          for (int t = 0; t < w.nh; ++t) {
+            issue_s(t, st);
+            tc_commit(&bars[kBarSFull + t]);
+          }
+          tc_commit(&k_empty[st]);
+        }
+        for (int j = 0; j < n_tiles && ok; ++j) {
+          const uint32_t kj = kv_iter + j;
+          const int st = kj % S;
+          const int stn = (kj + 1) % S;
+          const bool more = j + 1 < n_tiles;
+          for (int t = 0; t < w.nh && ok; ++t) {
+            if (!(ok = mbar_wait(&bars[kBarPFull + t], p_phase[t], wc, 12))) break;
+            p_phase[t] ^= 1;
+            if (j == 0 && o_uses[t] > 0 &&
+                !(ok = mbar_wait(&bars[kBarOEmpty + t], (o_uses[t] - 1) & 1, wc, 13)))
+              break;
+            if (t == 0 && !(ok = mbar_wait(&v_full[st], (kj / S) & 1, wc, 14))) break;
+            tc_fence_after();
+            issue_pv(t, st, j > 0);
+            if (more) {
+              if (t == 0 && !(ok = mbar_wait(&k_full[stn], ((kj + 1) / S) & 1, wc, 15))) break;
+              tc_fence_after();
+              issue_s(t, stn);
+              tc_commit(&bars[kBarSFull + t]);
+            }
+          }
+          if (!ok) break;
+          tc_commit(&v_empty[st]);
+          if (more) tc_commit(&k_empty[stn]);
+        }
+        if (!ok) break;
+        for (int t = 0; t < w.nh; ++t) {
+          tc_commit(&bars[kBarOFull + t]);
+          ++o_uses[t];
+        }
+        tc_commit(&bars[kBarQEmpty]);
+        kv_iter += n_tiles;
+      }
+      // make sure no MMA still writes TMEM when it is released
+      tc_commit(&bars[kBarDrain]);
+      mbar_wait_drain(&bars[kBarDrain], 0);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int t = (warp - 2) >> 2;
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_base + C::col_s(t);
+    const uint32_t tO = tmem + lane_base + C::col_o(t);
+    const float sl2 = prm.scale_log2;
+    const int T = prm.total_tokens;
+    uint32_t s_phase = 0, o_uses = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+      const Item w = prm.items[it];
+      if (t >= w.nh) continue;
+      const int n_tiles = (w.e_end - w.e_begin + C::EPT - 1) / C::EPT;
+      const int i = w.row_begin + row;
+      const bool valid = i < w.row_end;
+      const int h = w.qh0 + t;
+      const int64_t orow = static_cast<int64_t>(w.q_row0 + i) * prm.hq + h;
+      const int64_t lse_idx =
+          (static_cast<int64_t>(w.layer) * prm.hq + h) * T + (w.q_row0 - w.layer * T) + i;
+      if (n_tiles == 0) {
+        if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(prm.o + orow * D);
+          for (int k = 0; k < D / 8; ++k) dst[k] = make_uint4(0, 0, 0, 0);
+          if (prm.lse) prm.lse[lse_idx] = -INFINITY;
+        }
+        continue;
+      }
+      const int window = w.window;
+      float m_ref = -INFINITY, l = 0.f;
+      for (int j = 0; j < n_tiles && ok; ++j) {
+        if (!(ok = mbar_wait(&bars[kBarSFull + t], s_phase, wc, 20))) break;
+        s_phase ^= 1;
+        tc_fence_after();
+        float s[kKeysPerTile];
+#pragma unroll
+        for (int c = 0; c < kKeysPerTile / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld_x32(tS + 32 * c, r);
+          tmem_ld_wait(r);
+#pragma unroll
+          for (int k = 0; k < 32; ++k) s[32 * c + k] = __uint_as_float(r[k]);
+        }
+        // pages of this tile
+        int lp[C::EPT], nv[C::EPT];
+        bool full = true;
+#pragma unroll
+        for (int e = 0; e < C::EPT; ++e) {
+          const int idx = w.e_begin + j * C::EPT + e;
+          if (idx < w.e_end) {
+            const int4 en = *reinterpret_cast<const int4*>(prm.entries + idx);
+            lp[e] = en.y;
+            nv[e] = en.w;
+          } else {
+            lp[e] = 0;
+            nv[e] = 0;
+          }
+          full = full && nv[e] == P;
+        }
+        full = full && lp[C::EPT - 1] + P - 1 <= i && (window < 0 || lp[0] > i - window);
+        if (!full) {
+#pragma unroll
+          for (int c = 0; c < kKeysPerTile; ++c) {
+            const int e = c / P, r = c % P;
+            const int jpos = lp[e] + r;
+            const bool vis = r < nv[e] && jpos <= i && (window < 0 || jpos > i - window);
+            s[c] = vis ? s[c] : -INFINITY;
+          }
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < kKeysPerTile; ++c) mx = fmaxf(mx, s[c]);
+        const float m_new = fmaxf(m_ref, mx * sl2);
+        const bool resc = m_new > m_ref + kRescaleLog2;
+        if (j > 0 && __any_sync(0xffffffffu, resc)) {
+          const float alpha = resc ? ex2_approx(m_ref - m_new) : 1.f;
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld_x32(tO + 32 * c, r);
+            tmem_ld_wait(r);
+#pragma unroll
+            for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * alpha);
+            tmem_st_x32(tO + 32 * c, r);
+          }
+          tmem_st_wait();
+          if (resc) l *= alpha;
+        }
+        if (resc) m_ref = m_new;
+        const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
+        float rs = 0.f;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            const float p0 = ex2_approx(fmaf(s[64 * half + 2 * k], sl2, -m_use));
+            const float p1 = ex2_approx(fmaf(s[64 * half + 2 * k + 1], sl2, -m_use));
+            rs += p0 + p1;
+            pk[k] = pack_bf16x2(p0, p1);
+          }
+          tmem_st_x32(tS + 32 * half, pk);
+        }
+        l += rs;
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bars[kBarPFull + t]);
+      }
+      if (!ok) break;
+      // epilogue: O / l -> bf16
+      if (!(ok = mbar_wait(&bars[kBarOFull + t], o_uses & 1, wc, 21))) break;
+      ++o_uses;
+      tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld_x32(tO + 32 * c, r);
+        tmem_ld_wait(r);
+        if (valid) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int k = 0; k < 16; ++k)
+            pk[k] = pack_bf16x2(__uint_as_float(r[2 * k]) * inv, __uint_as_float(r[2 * k + 1]) * inv);
+          uint4* dst = reinterpret_cast<uint4*>(prm.o + orow * D + 32 * c);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            dst[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+        }
+      }
+      if (valid && prm.lse)
+        prm.lse[lse_idx] = l > 0.f ? (m_ref + __log2f(l)) * 0.6931471805599453f : -INFINITY;
+      tc_fence_before();
+      mbar_arrive(&bars[kBarOEmpty + t]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+template <int D, int P>
+static cudaError_t launch_typed(const PrefillLaunchArgs& a, cudaStream_t stream) {
+  using C = PrefillCfg<D, P>;
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  CUtensorMap tq, tk, tv;
+  {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(a.hq),
+                                static_cast<cuuint64_t>(a.n_layers) * a.total_tokens};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
+                                   static_cast<cuuint64_t>(a.hq) * D * 2};
+    const cuuint32_t box[3] = {64, 1, kRowsPerTile};
+    const cuuint32_t es[3] = {1, 1, 1};
+    if (enc(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(a.q), dims, strides, box,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  const cuuint64_t pdims[2] = {static_cast<cuuint64_t>(D),
+                               static_cast<cuuint64_t>(a.n_pages) * P};
+  const cuuint64_t pstrides[1] = {static_cast<cuuint64_t>(D) * 2};
+  const cuuint32_t pbox[2] = {64, static_cast<cuuint32_t>(P)};
+  const cuuint32_t pes[2] = {1, 1};
+  if (enc(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.k_pool), pdims, pstrides,
+          pbox, pes, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  if (enc(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.v_pool), pdims, pstrides,
+          pbox, pes, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(segpaged_prefill_kernel<D, P>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return e;
+  PrefillParams prm;
+  prm.items = a.items;
+  prm.n_items = a.n_items;
+  prm.error_word = a.error_word;
+  prm.timeout_site = a.timeout_site;
+  prm.entries = a.entries;
+  prm.o = static_cast<__nv_bfloat16*>(a.o);
+  prm.lse = a.lse;
+  prm.hq = a.hq;
+  prm.total_tokens = a.total_tokens;
+  prm.n_pages = a.n_pages;
+  prm.scale_log2 = a.scale_log2;
+  segpaged_prefill_kernel<D, P><<<sms, kPrefillThreads, C::kSmemBytes, stream>>>(tq, tk, tv, prm);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prefill_args(const PrefillLaunchArgs& a, cudaStream_t stream) {
+  if (a.d == 128 && a.p == 64) return launch_typed<128, 64>(a, stream);
+  if (a.d == 128 && a.p == 16) return launch_typed<128, 16>(a, stream);
+  if (a.d == 64 && a.p == 64) return launch_typed<64, 64>(a, stream);
+  if (a.d == 64 && a.p == 16) return launch_typed<64, 16>(a, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace rk

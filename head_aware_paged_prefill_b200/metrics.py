@@ -1,0 +1,63 @@
+"""Work counts used to report throughput.
+
+visible_pairs(layout): sum over layers, q heads and computed rows of the
+number of keys the row attends to, counted from each class's rule in closed
+form.  Algorithmic FLOPs of the attention are 4 * D per visible pair
+(2 D for q.k, 2 D for p.v); exp, masking and rotation are not counted.
+
+relocate_bytes(jobs, p, d): bytes an rk_relocate_rope pass must move
+(read + write of every page it touches).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+LOCAL, RETRIEVAL = 1, 2
+
+
+def _uncached_mask(lay, r):
+    L = lay.req_len(r)
+    m = np.zeros(L, dtype=bool)
+    for seg in lay.segments[lay.segments[:, 0] == r]:
+        if not seg[4]:
+            m[int(seg[1]):int(seg[1] + seg[2])] = True
+    return m
+
+
+def visible_pairs(lay) -> int:
+    g = lay.hq // lay.hkv
+    W = int(lay.class_window[LOCAL])
+    P = lay.p
+    total = 0
+    for r in range(lay.n_req):
+        L = lay.req_len(r)
+        unc = _uncached_mask(lay, r)
+        rows = np.nonzero(unc)[0].astype(np.int64)
+        n_unc_le = np.cumsum(unc.astype(np.int64))  # uncached keys at positions <= i
+        for layer in range(lay.n_layers):
+            for kvh in range(lay.hkv):
+                c = int(lay.class_map[layer * lay.hkv + kvh])
+                if c == LOCAL:
+                    total += g * int(np.minimum(rows + 1, W).sum())
+                elif c == RETRIEVAL:
+                    t = lay.table_index(r, layer, kvh)
+                    pages = np.unique(lay.retr_pages[lay.retr_indptr[t]:lay.retr_indptr[t + 1]])
+                    pages = pages[(pages >= 0) & (pages * P < L)]
+                    pages = pages[~unc[pages * P]]
+                    cnt = n_unc_le[rows].sum() if rows.size else 0
+                    for k in pages:
+                        first, last = int(k) * P, min(int(k) * P + P, L) - 1
+                        # keys first..last visible to rows i >= first: min(i, last) - first + 1
+                        cnt += int(np.clip(rows - first + 1, 0, last - first + 1).sum())
+                    total += g * int(cnt)
+                else:
+                    total += g * L * (L + 1) // 2
+    return int(total)
+
+
+def attention_flops(lay) -> int:
+    return 4 * lay.d * visible_pairs(lay)
+
+
+def relocate_bytes(n_jobs: int, p: int, d: int) -> int:
+    return 2 * n_jobs * p * d * 2

@@ -379,3 +379,54 @@ def random_tiny(rng: np.random.Generator, *, p: Optional[int] = None, d: int = 8
 
 def tiny_workload(lay: Layout, seed: int = 0) -> Workload:
     return Workload("tiny", seed, lay, "cpu")
+
+
+def random_small(rng: np.random.Generator, *, p: Optional[int] = None, d: Optional[int] = None,
+                 max_pages: int = 24, n_req: Optional[int] = None) -> Layout:
+    """Random layout with the library's page sizes and head dims: 1-3
+    requests of up to max_pages pages (last page possibly partial), every
+    class, odd and even GQA groups, shared and private cached segments,
+    uncached segments anywhere, windows from 1 to 4 pages."""
+    p = p or int(rng.choice([16, 64]))
+    d = d or int(rng.choice([64, 128]))
+    n_req = n_req or int(rng.integers(1, 4))
+    n_layers = int(rng.integers(1, 3))
+    hkv = int(rng.integers(1, 4))
+    g = int(rng.choice([1, 2, 3, 4]))
+    shared = [(f"sh{i}", p * int(rng.integers(1, 4))) for i in range(2)]
+    requests = []
+    for r in range(n_req):
+        L = int(rng.integers(1, max_pages * p + 1))
+        segs, pos, k = [], 0, 0
+        while pos < L:
+            ln = p * int(rng.integers(1, 6))
+            if pos + ln >= L:
+                cached = bool(rng.random() < 0.3) and (L - pos) % p == 0
+                segs.append((f"t{r}_{k}", L - pos, int(rng.integers(0, 5000)), cached))
+                break
+            u = rng.random()
+            if u < 0.25:
+                name, ln = shared[int(rng.integers(2))]
+                if pos + ln > L:
+                    segs.append((f"t{r}_{k}", L - pos, 0, False))
+                    break
+                segs.append((name, ln, int(rng.integers(0, 5000)), True))
+            elif u < 0.45:
+                segs.append((f"u{r}_{k}", ln, 0, False))
+            else:
+                segs.append((f"c{r}_{k}", ln, int(rng.integers(0, 5000)), True))
+            pos += ln
+            k += 1
+        requests.append(segs)
+    cmap = rng.integers(0, 4, size=n_layers * hkv).astype(np.int8)
+    n_tables = n_req * n_layers * hkv
+    retrieval = {}
+    lens = [sum(s[1] for s in segs) for segs in requests]
+    for t in range(n_tables):
+        r = t // (n_layers * hkv)
+        npg = -(-lens[r] // p)
+        k = int(rng.integers(0, min(6, npg) + 1))
+        retrieval[t] = np.sort(rng.choice(npg, size=k, replace=False)).tolist()
+    return _make_layout(n_layers=n_layers, hq=hkv * g, hkv=hkv, d=d, p=p,
+                        theta=float(rng.choice([1e4, 1e6])), requests=requests, class_map=cmap,
+                        window=int(rng.integers(1, 4 * p + 1)), retrieval=retrieval)

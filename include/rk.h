@@ -1,0 +1,206 @@
+/*
+ * rk.h — C ABI of the SegPagedAttention prefill library (librk.so, sm_100a).
+ *
+ * The operations follow the RedKnot pages:
+ *   - rk_select_visible   <- SELECTVISIBLESTATE (paooo page, "how to use":
+ *                            choose which reused KV each head sees), built on
+ *                            the per-(layer, kv_head) head class map and the
+ *                            "per-head page table + segmented KV store" of the
+ *                            README excerpt ("SegPagedAttention Runtime").
+ *   - rk_relocate_rope    <- "Offline KV Reuse + RoPE Relocation" (README
+ *                            excerpt): re-rotate cached K from the position it
+ *                            was stored at to its new absolute position.
+ *   - rk_segpaged_prefill <- EXECUTE's attention (paooo page, "how to use" and
+ *                            "technical principles": a fused varlen kernel over
+ *                            per-head pages that never builds an attn_mask).
+ *
+ * Conventions shared by every call
+ *   - All pointers are caller-owned.  The library never allocates or frees
+ *     memory; device buffers are passed in, sized by rk_query_sizes().
+ *   - "host" pointers are read during the call only.  "device" pointers must
+ *     address memory of the current CUDA device.
+ *   - stream: a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Every device-side effect is ordered on that stream; calls return before
+ *     the GPU work finishes, except rk_get_device_status().
+ *   - Argument errors are detected on the host, synchronously, before any
+ *     GPU work is enqueued; nothing is written in that case.
+ *   - Kernels never trap.  A fault they detect (a page id outside the pool, a
+ *     bounded wait that ran out) sets a bit in the device error word inside
+ *     the workspace; read it with rk_get_device_status().
+ *   - bf16 tensors are passed as raw 16-bit storage (const void*).
+ *
+ * Notation: T = total tokens of the batch, L_r = length of request r,
+ * Hq / Hkv = query / key-value heads (G = Hq / Hkv, q head h reads kv head
+ * h / G), D = head_dim, P = page_size.  A "table" is one
+ * (request, layer, kv_head); its index is t = (r * n_layers + layer) * Hkv + kvh.
+ */
+#ifndef RK_H_
+#define RK_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t rk_status;
+#define RK_OK 0
+#define RK_ERR_INVALID_ARG 1 /* null pointer, bad dims, D not in {64,128}, P not in {16,64}, ... */
+#define RK_ERR_UNALIGNED 2   /* a segment other than a request's last has len % P != 0 */
+#define RK_ERR_CAPACITY 3    /* a buffer or the workspace is smaller than rk_query_sizes() says */
+#define RK_ERR_CUDA 4        /* a CUDA runtime / driver call failed */
+#define RK_ERR_DEVICE 5      /* rk_get_device_status(): the device error word is non-zero */
+
+/* bits of the device error word (reported through rk_get_device_status) */
+#define RK_DEV_BAD_PAGE 1u   /* a page id outside [0, n_pages): the access was skipped */
+#define RK_DEV_TIMEOUT 2u    /* a bounded wait inside a kernel gave up: outputs are invalid */
+#define RK_DEV_CAPACITY 4u   /* a work list would not fit the workspace: outputs are invalid */
+
+/* head classes (README excerpt, "Head Classification") */
+#define RK_GLOBAL 0    /* every row; key j visible to row i iff j <= i */
+#define RK_LOCAL 1     /* uncached rows; visible iff i - W < j <= i (W = class_window[RK_LOCAL]) */
+#define RK_RETRIEVAL 2 /* uncached rows; visible iff j <= i and (j uncached or page(j) listed) */
+#define RK_DENSE 3     /* same visibility as RK_GLOBAL (its KV is recomputed upstream) */
+
+typedef struct {
+  int32_t n_req;        /* requests in the batch, >= 1 */
+  int32_t n_layers;     /* attention layers covered by one call, >= 1 */
+  int32_t num_q_heads;  /* Hq, a multiple of num_kv_heads */
+  int32_t num_kv_heads; /* Hkv */
+  int32_t head_dim;     /* D: 64 or 128 */
+  int32_t page_size;    /* P: 16 or 64 */
+  int64_t n_pages;      /* pages in k_pool / v_pool; n_pages * P < 2^31 */
+  int32_t total_tokens; /* T = cu_seqlens[n_req] */
+  int32_t reserved;     /* must be 0 */
+} rk_dims;
+
+/* One segment instance of a request.  Segments of a request are listed in
+ * ascending logical_start and tile [0, L_r) exactly.  Cached segments hold KV
+ * computed offline at positions stored_pos_base .. stored_pos_base + len - 1
+ * and reused here at logical_start (delta = logical_start - stored_pos_base);
+ * uncached segments hold KV computed for this request at its own positions
+ * (their stored_pos_base is ignored, delta = 0). */
+typedef struct {
+  int32_t req;
+  int32_t logical_start;
+  int32_t len;
+  int32_t stored_pos_base;
+  int32_t cached; /* 1 = reused from the offline store, 0 = computed online */
+} rk_segment;
+
+/* Host-side description of the batch (all pointers are host memory). */
+typedef struct {
+  int32_t n_segments;
+  const rk_segment* segments; /* [n_segments], grouped by request */
+  /* [n_segments][n_layers * Hkv]: physical page of the segment's first page
+   * for (layer, kv_head); its pages for that pair are consecutive ids. */
+  const int32_t* page_base;
+  const int32_t* cu_seqlens;   /* [n_req + 1], cu_seqlens[0] = 0, non-decreasing */
+  const int8_t* class_map;     /* [n_layers * Hkv], RK_GLOBAL .. RK_DENSE */
+  const int32_t* class_window; /* [4]; class_window[RK_LOCAL] = W >= 1, others unused */
+  /* retrieval page lists, CSR over tables ([n_tables + 1] and the values):
+   * request-logical page numbers k (positions [kP, kP + P)); listed pages that
+   * are uncached or past the request are ignored.  Both may be NULL when no
+   * table has class RK_RETRIEVAL. */
+  const int32_t* retr_indptr;
+  const int32_t* retr_pages;
+} rk_layout;
+
+/* One page-table entry (16 bytes). */
+typedef struct {
+  int32_t phys_page;   /* page id in the pool */
+  int32_t logical_pos; /* absolute position (within the request) of the page's first key */
+  int32_t delta;       /* RoPE relocation of the page's keys: logical - stored position */
+  int32_t n_valid;     /* keys in the page, P except for the last page of a request */
+} rk_entry;
+
+typedef struct {
+  int32_t begin, end; /* half-open range of request-local row positions */
+} rk_range;
+
+/* Visible state produced by rk_select_visible (all device memory, written
+ * by the call).  Table t's entries are entries[entry_start[t] ..
+ * entry_start[t] + entry_count[t]), ascending logical_pos: every page of the
+ * request that holds at least one key visible to at least one row of the
+ * table.  Its rows are the merged ranges ranges[range_start[t] ..
+ * + range_count[t]).  The start offsets are fixed by the layout:
+ *   entry_start[t] = (layer * Hkv + kvh) * sum_r ceil(L_r / P) + sum_{r'<r} ceil(L_r' / P)
+ *   range_start[t] = (layer * Hkv + kvh) * n_segments + (first segment index of r) */
+typedef struct {
+  rk_entry* entries;    /* [entry_capacity] */
+  int32_t* entry_start; /* [n_tables] */
+  int32_t* entry_count; /* [n_tables] */
+  rk_range* ranges;     /* [range_capacity] */
+  int32_t* range_start; /* [n_tables] */
+  int32_t* range_count; /* [n_tables] */
+  int64_t entry_capacity;
+  int64_t range_capacity;
+} rk_visible;
+
+typedef struct {
+  int64_t n_tables;
+  int64_t entry_capacity;  /* rk_entry elements rk_visible.entries must hold */
+  int64_t range_capacity;  /* rk_range elements rk_visible.ranges must hold */
+  int64_t item_capacity;   /* attention work items the workspace reserves */
+  int64_t workspace_bytes; /* device workspace for select + prefill (256-byte aligned) */
+} rk_sizes;
+
+/* Validates dims + layout and reports the buffer sizes the other calls need.
+ * Host only: touches no GPU.  Errors: RK_ERR_INVALID_ARG, RK_ERR_UNALIGNED. */
+rk_status rk_query_sizes(const rk_dims* dims, const rk_layout* layout, rk_sizes* out);
+
+/* SELECTVISIBLESTATE.  Builds, on the GPU, every table's page table and row
+ * ranges (bit-exact integer work) plus the attention work list kept in the
+ * workspace for rk_segpaged_prefill.  Copies the layout into the workspace
+ * (stream-ordered; the host arrays may be reused once the call returns).
+ * workspace: device, >= rk_sizes.workspace_bytes, 256-byte aligned; it also
+ * holds the device error word, which this call resets.
+ * Errors (host): RK_ERR_INVALID_ARG, RK_ERR_UNALIGNED, RK_ERR_CAPACITY,
+ * RK_ERR_CUDA.  Device: RK_DEV_BAD_PAGE, RK_DEV_CAPACITY. */
+rk_status rk_select_visible(const rk_dims* dims, const rk_layout* layout, const rk_visible* out,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/* RoPE relocation of cached K pages.  For each job n, with
+ * jobs[3n..3n+2] = (src_page, dst_page, delta):
+ *   k_dst[dst_page][row][:] = bf16( R(delta) k_src[src_page][row][:] )  for row < P,
+ * R the rotate-half RoPE rotation (pairs (m, m + D/2), frequency
+ * rope_theta^(-2m/D)), computed in fp32 from angles reduced in fp64; delta = 0
+ * copies the page bit-exactly.  k_src / k_dst: device bf16 [n_pages][P][D]
+ * (may be the same pool); jobs: device int32 [n_jobs][3].  A job may read and
+ * write the same page; otherwise no page may be written by one job and read or
+ * written by another.  Jobs with a page id outside [0, n_pages) are skipped
+ * and set RK_DEV_BAD_PAGE in *device_error (device int32, may be NULL).
+ * Errors (host): RK_ERR_INVALID_ARG, RK_ERR_CUDA. */
+rk_status rk_relocate_rope(const void* k_src, void* k_dst, const int32_t* jobs, int32_t n_jobs,
+                           int64_t n_pages, int32_t page_size, int32_t head_dim,
+                           double rope_theta, int32_t* device_error, void* stream);
+
+/* EXECUTE's attention.  For every table's rows i and each q head h of its kv
+ * head:  o[layer][tok(i)][h][:] = sum_j softmax_j(softmax_scale <q_i, K'_j>) v_j
+ * over the visible keys j of the table, where K'_j is the stored key rotated
+ * by its entry's delta when fuse_rope = 1 (fuse_rope = 0: the pool already
+ * holds relocated keys and delta is ignored).  bf16 inputs, fp32 accumulation,
+ * bf16 output.  Rows outside a table's row set are not written.
+ *   q, o: device bf16 [n_layers][T][Hq][D] (token-packed varlen layout)
+ *   k_pool, v_pool: device bf16 [n_pages][P][D]; every row of every page
+ *     (including rows past n_valid) must hold finite values.
+ *   lse: device fp32 [n_layers][Hq][T] natural-log logsumexp, or NULL.
+ *   vis, workspace: as filled by rk_select_visible on the same stream.
+ * Errors (host): RK_ERR_INVALID_ARG, RK_ERR_CAPACITY, RK_ERR_CUDA.
+ * Device: RK_DEV_BAD_PAGE, RK_DEV_TIMEOUT. */
+rk_status rk_segpaged_prefill(const rk_dims* dims, const void* q, const void* k_pool,
+                              const void* v_pool, const rk_visible* vis, int32_t fuse_rope,
+                              double rope_theta, float softmax_scale, void* o, float* lse,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/* Waits for the stream, then copies the device error word of the workspace
+ * into *status (host).  Returns RK_OK when the word is 0, RK_ERR_DEVICE
+ * otherwise, RK_ERR_CUDA if the copy failed. */
+rk_status rk_get_device_status(const void* workspace, int32_t* status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RK_H_ */

@@ -384,22 +384,36 @@ int ora_attention(const ora_problem* pr, const uint16_t* q_rows, const uint16_t*
     /* relocated keys K'_j = R(delta_j) K_stored_j and values, fp64 */
     double* kr = (double*)malloc(sizeof(double) * ((size_t)L * d + 1));
     double* vr = (double*)malloc(sizeof(double) * ((size_t)L * d + 1));
-    double* x = (double*)malloc(sizeof(double) * d);
+    /* every key of a segment moves by the same delta: R(delta) is formed
+     * once per segment (cos / sin of delta * theta^(-2m/D), fp64) */
+    int h = d / 2;
+    double* cs = (double*)malloc(sizeof(double) * d);
+    int cur_seg = -1;
     for (int j = 0; j < L; ++j) {
       int s = t.seg_of[j];
       const int32_t* sg = pr->seg + 5 * s;
       int off = j - sg[1];
       int page = pr->page_base[(size_t)s * pr->n_layers * pr->hkv + lh] + off / P;
       int delta = sg[1] - sg[3];
+      if (s != cur_seg) {
+        for (int m = 0; m < h; ++m) {
+          double a = (double)delta * pow(theta, -2.0 * (double)m / (double)d);
+          cs[m] = cos(a);
+          cs[h + m] = sin(a);
+        }
+        cur_seg = s;
+      }
       const uint16_t* ks = k_pool + ((size_t)page * P + off % P) * d;
       const uint16_t* vs = v_pool + ((size_t)page * P + off % P) * d;
-      for (int c = 0; c < d; ++c) {
-        x[c] = bf16_to_double(ks[c]);
-        vr[(size_t)j * d + c] = bf16_to_double(vs[c]);
+      double* kj = kr + (size_t)j * d;
+      for (int m = 0; m < h; ++m) {
+        double x0 = bf16_to_double(ks[m]), x1 = bf16_to_double(ks[m + h]);
+        kj[m] = x0 * cs[m] - x1 * cs[h + m];
+        kj[m + h] = x0 * cs[h + m] + x1 * cs[m];
       }
-      ora_rope_rotate(x, d, theta, (double)delta, kr + (size_t)j * d);
+      for (int c = 0; c < d; ++c) vr[(size_t)j * d + c] = bf16_to_double(vs[c]);
     }
-    free(x);
+    free(cs);
     aj.tab = &t;
     aj.kr = kr;
     aj.vr = vr;

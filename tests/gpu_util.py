@@ -1,0 +1,125 @@
+"""Helpers shared by the GPU parity tests: run the CUDA path through the C ABI
+and compare it with the fp64 oracle."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from head_aware_paged_prefill_b200 import binding
+from head_aware_paged_prefill_b200.plan import relocation_plan
+
+# tolerances for bf16-in / fp32-accumulate outputs (max abs, mean relative)
+MAX_ABS = 2e-2
+MEAN_REL = 5e-3
+SENTINEL = 0x7FC0  # a bf16 NaN the kernels never write
+
+
+def u16(t: torch.Tensor) -> np.ndarray:
+    return t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def assert_close(got: np.ndarray, want: np.ndarray, what: str = ""):
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    assert np.isfinite(got).all(), f"{what}: non-finite GPU values"
+    err = np.abs(got - want)
+    mx = float(err.max()) if err.size else 0.0
+    rel = float(err.sum() / max(np.abs(want).sum(), 1e-300)) if err.size else 0.0
+    assert mx <= MAX_ABS, f"{what}: max abs err {mx:.3e} > {MAX_ABS}"
+    assert rel <= MEAN_REL, f"{what}: mean rel err {rel:.3e} > {MEAN_REL}"
+    return mx, rel
+
+
+def run_select(lay, device="cuda"):
+    hl = binding.HostLayout(lay)
+    s = hl.sizes()
+    vis = binding.Visible(s, device)
+    ws = binding.workspace(s, device)
+    binding.select_visible(hl, vis, ws)
+    return hl, vis, ws
+
+
+class PrefillRun:
+    """rk_relocate_rope over the relocation plan, then rk_select_visible and
+    rk_segpaged_prefill(fuse_rope=0) on the relocated layout, on cuda:0.
+    ``o`` starts filled with the sentinel so untouched rows can be checked."""
+
+    def __init__(self, lay, q, k_pool, v_pool, with_lse=True):
+        dev = q.device
+        jobs, rel = relocation_plan(lay)
+        self.lay, self.rel, self.jobs = lay, rel, jobs
+        extra = rel.n_pages - lay.n_pages
+        self.k_rel = torch.cat([k_pool, torch.zeros((extra,) + tuple(k_pool.shape[1:]),
+                                                    dtype=k_pool.dtype, device=dev)])
+        self.v_rel = torch.cat([v_pool, torch.zeros((extra,) + tuple(v_pool.shape[1:]),
+                                                    dtype=v_pool.dtype, device=dev)])
+        # V pages of relocated instances are delta-0 copies of their sources
+        self.dev_err = torch.zeros(1, dtype=torch.int32, device=dev)
+        if jobs.shape[0]:
+            jt = torch.from_numpy(jobs).to(dev)
+            jv = jt.clone()
+            jv[:, 2] = 0
+            binding.relocate_rope(self.k_rel, self.k_rel, jt, lay.theta, self.dev_err)
+            binding.relocate_rope(self.v_rel, self.v_rel, jv, lay.theta, self.dev_err)
+        self.hl, self.vis, self.ws = run_select(rel, dev)
+        self.o = torch.full(q.shape, SENTINEL, dtype=torch.int16, device=dev).view(torch.bfloat16)
+        self.lse = (torch.full((lay.n_layers, lay.hq, lay.total_tokens), float("nan"),
+                               device=dev) if with_lse else None)
+        binding.segpaged_prefill(self.hl, q, self.k_rel, self.v_rel, self.vis, self.ws, self.o,
+                                 self.lse)
+        torch.cuda.synchronize()
+        self.status = binding.device_status(self.ws) | int(self.dev_err.item())
+
+
+def table_rows(lay):
+    """(table -> list of row ranges) from the oracle's brute-force row sets."""
+    _, ranges = oracle.page_tables(lay)
+    return ranges
+
+
+def sample_rows(lay, per_table: int, seed: int):
+    """(layer, q_head, token) rows: for each table, its first and last rows,
+    rows around 128-row tile boundaries, and random rows; every q head."""
+    rng = np.random.default_rng(seed)
+    ranges = table_rows(lay)
+    g = lay.hq // lay.hkv
+    out = []
+    for r in range(lay.n_req):
+        t0 = int(lay.cu_seqlens[r])
+        for layer in range(lay.n_layers):
+            for kvh in range(lay.hkv):
+                rg = ranges[lay.table_index(r, layer, kvh)]
+                if rg.shape[0] == 0:
+                    continue
+                rows = np.concatenate([np.arange(a, b) for a, b in rg])
+                pick = {int(rows[0]), int(rows[-1])}
+                for a, b in rg:
+                    for x in (a + 127, a + 128, b - 129, b - 128):
+                        if a <= x < b:
+                            pick.add(int(x))
+                extra = rng.choice(rows, size=min(len(rows), per_table), replace=False)
+                pick.update(int(x) for x in extra)
+                for h in range(kvh * g, kvh * g + g):
+                    for i in sorted(pick):
+                        out.append((layer, h, t0 + i))
+    return np.asarray(out, dtype=np.int32).reshape(-1, 3)
+
+
+def oracle_rows(lay, q, k_pool, v_pool, rows):
+    qr = q[torch.from_numpy(rows[:, 0]).long(), torch.from_numpy(rows[:, 2]).long(),
+           torch.from_numpy(rows[:, 1]).long()]
+    return oracle.attention(lay, u16(qr), u16(k_pool), u16(v_pool), rows)
+
+
+def gpu_rows(run: PrefillRun, rows):
+    o = run.o[torch.from_numpy(rows[:, 0]).long().to(run.o.device),
+              torch.from_numpy(rows[:, 2]).long().to(run.o.device),
+              torch.from_numpy(rows[:, 1]).long().to(run.o.device)]
+    lse = None
+    if run.lse is not None:
+        lse = run.lse[torch.from_numpy(rows[:, 0]).long().to(run.o.device),
+                      torch.from_numpy(rows[:, 1]).long().to(run.o.device),
+                      torch.from_numpy(rows[:, 2]).long().to(run.o.device)]
+        lse = lse.double().cpu().numpy()
+    return o.double().cpu().numpy(), lse

@@ -1,0 +1,163 @@
+"""The C-ABI library loads, exports what include/rk.h declares, and rejects
+bad arguments on the host before any GPU work (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from head_aware_paged_prefill_b200 import binding, synth
+from head_aware_paged_prefill_b200.csrc import build as build_mod
+from head_aware_paged_prefill_b200.plan import relocation_plan
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return binding.lib()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "rk.h")).read()
+    return sorted(set(re.findall(r"^rk_status\s+(rk_\w+)\s*\(", src, re.M)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared()
+    assert set(names) == set(binding.EXPORTS)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def _hl(lay):
+    return binding.HostLayout(lay)
+
+
+@pytest.mark.parametrize("name", ["cfg1", "cfg2", "cfg3", "cfg4", "cfg5"])
+def test_query_sizes(lib, name):
+    lay = synth.CONFIGS[name]().layout
+    s = _hl(lay).sizes()
+    n_lh = lay.n_layers * lay.hkv
+    total_pages = sum(-(-lay.req_len(r) // lay.p) for r in range(lay.n_req))
+    assert s.n_tables == lay.n_tables
+    assert s.entry_capacity == n_lh * total_pages
+    assert s.range_capacity == n_lh * lay.segments.shape[0]
+    assert s.workspace_bytes % 256 == 0 and s.workspace_bytes > 256 + 96 * s.item_capacity
+
+
+def _status_sizes(lay, mutate):
+    hl = _hl(lay)
+    mutate(hl)
+    s = binding.RkSizes()
+    return binding.lib().rk_query_sizes(ctypes.byref(hl.dims), ctypes.byref(hl.layout),
+                                        ctypes.byref(s))
+
+
+def test_rejects_bad_dims(lib):
+    lay = synth.cfg1().layout
+    E = binding.RK_ERR_INVALID_ARG
+    assert _status_sizes(lay, lambda h: setattr(h.dims, "head_dim", 96)) == E
+    assert _status_sizes(lay, lambda h: setattr(h.dims, "page_size", 32)) == E
+    assert _status_sizes(lay, lambda h: setattr(h.dims, "num_q_heads", 3)) == E
+    assert _status_sizes(lay, lambda h: setattr(h.dims, "n_pages", 0)) == E
+    assert _status_sizes(lay, lambda h: setattr(h.dims, "total_tokens", 447)) == E
+    assert _status_sizes(lay, lambda h: setattr(h.dims, "reserved", 1)) == E
+    assert _status_sizes(lay, lambda h: setattr(h.dims, "n_req", 0)) == E
+
+
+def test_rejects_bad_layouts(lib):
+    base = synth.cfg1().layout
+
+    def with_(**kw):
+        lay = synth.Layout(**{**base.__dict__})
+        for k, v in kw.items():
+            setattr(lay, k, v)
+        return lay
+
+    E, U = binding.RK_ERR_INVALID_ARG, binding.RK_ERR_UNALIGNED
+    seg = base.segments.copy()
+    seg[0, 2] = 120
+    seg[1, 1] = 120
+    seg[1, 2] = 136
+    assert _status_sizes(with_(segments=seg), lambda h: None) == U  # 120 % 16 != 0
+    pb = base.page_base.copy()
+    pb[3, 1] = base.n_pages - 1  # tail needs 4 pages
+    assert _status_sizes(with_(page_base=pb), lambda h: None) == E
+    seg = base.segments.copy()
+    seg[2, 1] = 250  # gap
+    assert _status_sizes(with_(segments=seg), lambda h: None) == E
+    assert _status_sizes(with_(class_map=np.asarray([0, 4], np.int8)), lambda h: None) == E
+    cw = base.class_window.copy()
+    cw[1] = 0
+    assert _status_sizes(with_(class_window=cw), lambda h: None) == E
+    cu = base.cu_seqlens.copy()
+    cu[1] = 440
+    assert _status_sizes(with_(cu_seqlens=cu), lambda h: None) == E
+    # retrieval class without lists
+    lay = with_(class_map=np.asarray([0, 2], np.int8))
+    assert _status_sizes(lay, lambda h: setattr(h.layout, "retr_indptr", None)) == E
+    assert _status_sizes(base, lambda h: setattr(h.layout, "segments", None)) == E
+
+
+def test_select_rejects_on_host_without_gpu(lib):
+    lay = synth.cfg1().layout
+    hl = _hl(lay)
+    s = hl.sizes()
+    vis = binding.RkVisible()  # null pointers
+    st = lib.rk_select_visible(ctypes.byref(hl.dims), ctypes.byref(hl.layout), ctypes.byref(vis),
+                               ctypes.c_void_p(256), s.workspace_bytes, None)
+    assert st == binding.RK_ERR_INVALID_ARG
+    fake = 1 << 20  # never dereferenced: the capacity check fails first
+    vis = binding.RkVisible(fake, fake, fake, fake, fake, fake, s.entry_capacity - 1,
+                            s.range_capacity)
+    st = lib.rk_select_visible(ctypes.byref(hl.dims), ctypes.byref(hl.layout), ctypes.byref(vis),
+                               ctypes.c_void_p(fake), s.workspace_bytes, None)
+    assert st == binding.RK_ERR_CAPACITY
+    vis = binding.RkVisible(fake, fake, fake, fake, fake, fake, s.entry_capacity,
+                            s.range_capacity)
+    st = lib.rk_select_visible(ctypes.byref(hl.dims), ctypes.byref(hl.layout), ctypes.byref(vis),
+                               ctypes.c_void_p(fake), s.workspace_bytes - 256, None)
+    assert st == binding.RK_ERR_CAPACITY
+
+
+def test_relocate_and_prefill_reject_on_host(lib):
+    E = binding.RK_ERR_INVALID_ARG
+    fake = ctypes.c_void_p(1 << 20)
+    assert lib.rk_relocate_rope(fake, fake, fake, 1, 8, 64, 96, 1e4, None, None) == E
+    assert lib.rk_relocate_rope(fake, fake, fake, -1, 8, 64, 128, 1e4, None, None) == E
+    assert lib.rk_relocate_rope(fake, fake, fake, 1, 8, 64, 128, -1.0, None, None) == E
+    assert lib.rk_relocate_rope(None, fake, fake, 1, 8, 64, 128, 1e4, None, None) == E
+    assert lib.rk_relocate_rope(ctypes.c_void_p((1 << 20) + 2), fake, fake, 1, 8, 64, 128, 1e4,
+                                None, None) == E
+    lay = synth.cfg1().layout
+    hl = _hl(lay)
+    vis = binding.RkVisible(1 << 20, 1 << 20, 1 << 20, 1 << 20, 1 << 20, 1 << 20, 1, 1)
+    args = [ctypes.byref(hl.dims), fake, fake, fake, ctypes.byref(vis), 0, 1e4, 0.125, fake,
+            None, fake, 1 << 20, None]
+    bad_scale = list(args)
+    bad_scale[7] = 0.0
+    assert lib.rk_segpaged_prefill(*bad_scale) == E
+    bad_fuse = list(args)
+    bad_fuse[5] = 2
+    assert lib.rk_segpaged_prefill(*bad_fuse) == E
+    null_q = list(args)
+    null_q[1] = None
+    assert lib.rk_segpaged_prefill(*null_q) == E
+    small_ws = list(args)
+    small_ws[11] = 16
+    assert lib.rk_segpaged_prefill(*small_ws) == binding.RK_ERR_CAPACITY
+    assert lib.rk_get_device_status(None, None, None) == E
+
+
+def test_relocation_plan_covers_every_nonzero_delta():
+    lay = synth.cfg3().layout
+    jobs, rel = relocation_plan(lay)
+    n_lh = lay.n_layers * lay.hkv
+    nz = [s for s in lay.segments if s[4] and s[1] != s[3]]
+    assert jobs.shape[0] == sum(int(s[2]) // lay.p for s in nz) * n_lh
+    assert (rel.segments[:, 1] == rel.segments[:, 3]).all()
+    assert len(set(jobs[:, 1].tolist())) == jobs.shape[0]  # destinations are distinct
+    assert jobs[:, 1].min() >= lay.n_pages and rel.n_pages == lay.n_pages + jobs.shape[0]
