@@ -3,9 +3,11 @@
 
 One step = one pass of the whole hot path over the Mistral-7B-shaped 32K
 layer (Hq 32, Hkv 8, D 128, P 64; 7 cached 4096-token segments + 4096 tail;
-kv_head 0 global, 1-7 local with a 4096 window): rk_relocate_rope (K, and V
-page copies) -> rk_select_visible -> rk_segpaged_prefill, inputs resident in
-HBM, L2 flushed (256 MiB write) between timed steps.
+kv_head 0 global, 1-7 local with a 4096 window): rk_select_visible ->
+rk_segpaged_prefill with the RoPE relocation of cached keys fused into the
+K loads, inputs resident in HBM, L2 flushed (256 MiB write) between timed
+steps.  The standalone relocation kernel (rk_relocate_rope over every cached
+page of the layer) is timed after it and reported against the HBM roofline.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -163,6 +165,42 @@ def _time_oracle(lay, q, k, v, rows):
     return time.perf_counter() - t0
 
 
+def _bench_relocate(torch, lay, k_pool, dev, flush, stream, reps, peaks, peak_kind):
+    """rk_relocate_rope over every cached page with delta != 0 (one job per
+    page and (layer, kv_head)), into separate destination pages."""
+    from head_aware_paged_prefill_b200 import binding, metrics
+    from head_aware_paged_prefill_b200.plan import relocation_plan
+    jobs, _ = relocation_plan(lay)
+    if jobs.shape[0] == 0:
+        return None
+    n = jobs.shape[0]
+    # sources stay in the pool; destinations are n fresh pages appended to it
+    pool = torch.cat([k_pool, torch.empty((n, lay.p, lay.d), dtype=torch.bfloat16, device=dev)])
+    jobs = jobs.copy()
+    jobs[:, 1] = k_pool.shape[0] + np.arange(n, dtype=np.int32)
+    jt = torch.from_numpy(jobs).to(dev)
+    for _ in range(3):
+        binding.relocate_rope(pool, pool, jt, lay.theta)
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(reps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        binding.relocate_rope(pool, pool, jt, lay.theta)
+        b.record(stream)
+        ms.append((a, b))
+    torch.cuda.synchronize()
+    t = statistics.mean(x.elapsed_time(y) for x, y in ms)
+    byts = metrics.relocate_bytes(n, lay.p, lay.d)
+    gbs = byts / (t * 1e-3) / 1e9
+    peak = float(peaks["hbm_gbs"])
+    return {"bound": "hbm", "kernel": "relocate_kernel", "jobs": n, "bytes": byts,
+            "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+            "peak_kind": peak_kind, "us": t * 1e3,
+            "traffic": _recorded_traffic("relocate_kernel", "relocate_" + str(n))}
+
+
 def cpu_values(wl):
     """(q, k, v) on the host for the oracle (drawn on the GPU when the workload's
     recipe says so, then copied back)."""
@@ -216,7 +254,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="cfg2")
     ap.add_argument("--e2e-steps", type=int, default=20)
-    ap.add_argument("--cpu-sample-rows", type=int, default=2048)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--mode", default="fused", choices=["fused", "relocate"])
+    ap.add_argument("--reloc-reps", type=int, default=50)
     ap.add_argument("--ref-step-s", type=float, default=0.25)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -244,7 +284,7 @@ def main():
     wl = synth.CONFIGS[args.config]()
     lay = wl.layout
     q, k, v = wl.materialize(str(dev))
-    pre = SegPagedPrefill(lay, dev)
+    pre = SegPagedPrefill(lay, dev, mode=args.mode)
     pre.load(q, k, v)
     flops = metrics.attention_flops(lay)
     tokens = lay.total_tokens * lay.n_layers
@@ -323,15 +363,20 @@ def main():
     peak = float(peaks["bf16_tflops"])
     traffic = _recorded_traffic("segpaged_prefill_kernel", wl.name)
 
+    reloc = _bench_relocate(torch, lay, k, dev, flush, stream, args.reloc_reps, peaks, peak_kind)
+
     cpu_baseline = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
-        rows, pairs = _oracle_sample_rows(lay, args.cpu_sample_rows, seed=0)
+        rows, pairs = _oracle_sample_rows(lay, 256, seed=0)
+        dt = _time_oracle(lay, qc, kc, vc, rows)
+        n_rows = int(max(256, min(200000, 256 * args.cpu_seconds / max(dt, 1e-3))))
+        rows, pairs = _oracle_sample_rows(lay, n_rows, seed=1)
         dt = _time_oracle(lay, qc, kc, vc, rows)
         cpu_baseline = {"value": 4 * lay.d * pairs / dt / 1e12, "unit": UNIT,
                         "cores": os.cpu_count() or 1, "kind": "oracle",
-                        "sample": f"{args.cpu_sample_rows} seeded (layer, q head, row) samples "
-                                  f"of the same workload, {pairs} visible pairs, {dt:.1f} s"}
+                        "sample": f"{n_rows} seeded (layer, q head, row) samples of the same "
+                                  f"workload, {pairs} visible pairs, {dt:.1f} s"}
 
     if world > 1:
         dist.barrier()
@@ -359,6 +404,8 @@ def main():
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / E},
         "gpu_launches": K * pre.launches_per_run,
         "clocks": clocks,
+        "mode": args.mode,
+        "relocate_roofline": reloc,
     }
     print(json.dumps(line), flush=True)
     return 0

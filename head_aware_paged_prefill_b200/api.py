@@ -1,12 +1,14 @@
 """Public Python API: one SegPagedAttention prefill pass over a paged pool.
 
-``SegPagedPrefill(layout)`` plans the buffers of one layout once (relocation
-jobs, page tables, work list, workspace); ``run(q, k_pool, v_pool)`` then
-executes the three C-ABI calls on the current CUDA stream:
+``SegPagedPrefill(layout)`` plans the buffers of one layout once (page
+tables, work list, workspace); ``run(q, k_pool, v_pool)`` then executes the
+C-ABI calls on the current CUDA stream.  Two modes:
 
-  rk_relocate_rope    cached pages with a non-zero delta -> relocated pages
-  rk_select_visible   per-(request, layer, kv_head) page tables + work list
-  rk_segpaged_prefill attention over the visible pages
+  "fused"     rk_select_visible, then rk_segpaged_prefill(fuse_rope=1): cached
+              keys are rotated by their page's delta as they are loaded.
+  "relocate"  rk_relocate_rope writes relocated copies of every cached page
+              with a non-zero delta (K rotated, V copied), then
+              rk_select_visible and rk_segpaged_prefill(fuse_rope=0) read them.
 
 Inputs may live on the host (pinned tensors are copied asynchronously) or on
 the device; ``run(..., out="host")`` returns o on the host.
@@ -23,10 +25,16 @@ from .plan import relocation_plan
 
 
 class SegPagedPrefill:
-    def __init__(self, layout, device="cuda", with_lse: bool = False):
+    def __init__(self, layout, device="cuda", with_lse: bool = False, mode: str = "fused"):
+        if mode not in ("fused", "relocate"):
+            raise ValueError(mode)
         self.layout = layout
+        self.mode = mode
         self.device = torch.device(device)
-        self.jobs_np, self.rel_layout = relocation_plan(layout)
+        if mode == "relocate":
+            self.jobs_np, self.rel_layout = relocation_plan(layout)
+        else:
+            self.jobs_np, self.rel_layout = np.zeros((0, 3), np.int32), layout
         self.hl = binding.HostLayout(self.rel_layout)
         self.sizes = self.hl.sizes()
         self.vis = binding.Visible(self.sizes, self.device)
@@ -74,7 +82,8 @@ class SegPagedPrefill:
         if k3_events is not None:
             k3_events[0].record(s)
         binding.segpaged_prefill(self.hl, self.q_dev, self.k_work, self.v_work, self.vis,
-                                 self.ws, self.o, self.lse, stream=stream)
+                                 self.ws, self.o, self.lse, fuse_rope=self.mode == "fused",
+                                 stream=stream)
         if k3_events is not None:
             k3_events[1].record(s)
 

@@ -299,7 +299,8 @@ extern "C" rk_status rk_segpaged_prefill(const rk_dims* dims, const void* q, con
       !aligned(vis->entries, 16) || !aligned(workspace, 256) || !aligned(lse, 4))
     return RK_ERR_INVALID_ARG;
   if (fuse_rope != 0 && fuse_rope != 1) return RK_ERR_INVALID_ARG;
-  if (fuse_rope == 1) return RK_ERR_INVALID_ARG;  // fused relocation: not built yet
+  if (fuse_rope == 1 && (!(rope_theta > 0.0) || !std::isfinite(rope_theta)))
+    return RK_ERR_INVALID_ARG;
   if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return RK_ERR_INVALID_ARG;
   if (workspace_bytes < sizeof(WsHeader)) return RK_ERR_CAPACITY;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -322,6 +323,8 @@ extern "C" rk_status rk_segpaged_prefill(const rk_dims* dims, const void* q, con
   a.o = o;
   a.lse = lse;
   a.scale_log2 = softmax_scale * 1.4426950408889634f;
+  a.fuse_rope = fuse_rope;
+  a.rope_theta = rope_theta;
   if (dims->total_tokens == 0) return RK_OK;
   cudaError_t e = launch_prefill_args(a, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? RK_OK : RK_ERR_CUDA;

@@ -88,6 +88,8 @@ struct PrefillLaunchArgs {
   void* o;
   float* lse;
   float scale_log2;
+  int fuse_rope;
+  double rope_theta;
 };
 
 }  // namespace rk

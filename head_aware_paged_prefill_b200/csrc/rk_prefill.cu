@@ -4,22 +4,30 @@
 // pages and a fused varlen kernel attends over exactly the pages each head
 // may see, with no attn_mask; global heads recompute every row causally,
 // local heads compute the uncached rows over a window of reused KV (README
-// excerpt, "Head Classification" and "SegPagedAttention Runtime").
+// excerpt, "Head Classification" and "SegPagedAttention Runtime").  Cached
+// keys are re-rotated to their reuse position while they are loaded ("Offline
+// KV Reuse + RoPE Relocation").
 //
 // One CTA per SM, persistent over the work list of rk_select_visible.  A work
 // item is <= 128 rows of one request and up to two q heads of the same kv
 // head: both heads see identical pages, so each K/V tile loaded into shared
-// memory feeds two Q tiles.
+// memory feeds two Q tiles.  Items arrive sorted by cost; CTA b takes item
+// b, then 2G-1-b, 2G+b, ... (G = grid size), which evens out the per-SM work.
 //
 //   warp 0      TMA producer: Q tiles (3-D box out of [rows][Hq][D]) and, per
 //               KV tile, one box per page and 64-column block out of the pool.
 //   warp 1      tcgen05 issuer and TMEM owner.  S_t = Q_t K^T (M=128, N=128,
 //               K=D) into TMEM; O_t += P_t V (M=128, N=D, K=128) with P_t read
 //               from TMEM and V from shared memory (MN-major operand).
-//   warps 2-5   softmax warpgroup of Q tile 0, warps 6-9 of Q tile 1: one
+//   warps 2-3   RoPE relocation of the K tile in shared memory (fuse_rope):
+//               rows of a page with delta != 0 are rotated by R(delta) in place
+//               before the QK^T MMA may read them.
+//   warps 4-7   softmax warpgroup of Q tile 0, warps 8-11 of Q tile 1: one
 //               TMEM lane (= one query row) per thread; online softmax in the
 //               log2 domain, O rescaled in TMEM only when the running max
 //               grows by more than 2^8, P written back over S as bf16.
+// Registers are rebalanced with setmaxnreg: the first warpgroup keeps 80 per
+// thread, the two softmax warpgroups get 208.
 //
 // Invisible pages are never loaded: the item's entry range already excludes
 // them.  Element masks are evaluated only on tiles that straddle the causal
@@ -33,8 +41,11 @@
 
 namespace rk {
 
-constexpr int kPrefillThreads = 320;
+constexpr int kPrefillThreads = 384;
 constexpr float kRescaleLog2 = 8.0f;
+constexpr uint32_t kRegsAux = 80;       // warps 0-3
+constexpr uint32_t kRegsSoftmax = 208;  // warps 4-11
+static_assert(128 * kRegsAux + 256 * kRegsSoftmax <= 384 * 168, "register split over budget");
 
 template <int D, int P>
 struct PrefillCfg {
@@ -64,6 +75,8 @@ struct PrefillParams {
   int total_tokens;
   int64_t n_pages;
   float scale_log2;
+  int fuse_rope;
+  double inv_freq[64];  // theta^(-2m/D), m < D/2
 };
 
 // barrier slots
@@ -75,14 +88,60 @@ enum : int {
   kBarOFull = 6,   // [2]
   kBarOEmpty = 8,  // [2]
   kBarDrain = 10,  // MMA completion before TMEM is released
-  kBarKFull = 11,  // [kStages] x 4 groups follow
+  kBarKFull = 11,  // [kStages] x 5 groups follow (k_full, k_ready, k_empty, v_full, v_empty)
 };
+
+// Item of round r for CTA b (boustrophedon over the cost-sorted list).
+__device__ __forceinline__ int item_of_round(int r, int b, int g) {
+  return r * g + ((r & 1) ? (g - 1 - b) : b);
+}
+
+// Rotates, in place, the rows of one page of a K tile held in shared memory
+// (128-byte swizzle: 16-byte chunk c of row r lives at chunk c ^ (r & 7)).
+// Thread rt of 64 owns chunk c of rows r0, r0 + rstep, ...; pair (m, m + D/2)
+// of a row sits in chunks c and c + D/16 (D = 64) or at the same chunk of the
+// next 64-column block (D = 128).
+template <int D, int P>
+__device__ __forceinline__ void rope_rotate_rows(uint8_t* tile, int e, int rt, const float2 (&cs)[8]) {
+  constexpr int CH = D / 16;  // chunk pairs per row
+  constexpr int RSTEP = 64 / CH;
+  const int c = rt % CH, r0 = rt / CH;
+#pragma unroll 4
+  for (int r = r0; r < kKeysPerTile; r += RSTEP) {
+    if (r / P != e) continue;
+    const int sw = r & 7;
+    uint8_t* row = tile + r * 128;
+    uint4* plo;
+    uint4* phi;
+    if constexpr (D == 128) {
+      plo = reinterpret_cast<uint4*>(row + ((c ^ sw) << 4));
+      phi = reinterpret_cast<uint4*>(row + kKeysPerTile * 128 + ((c ^ sw) << 4));
+    } else {
+      plo = reinterpret_cast<uint4*>(row + ((c ^ sw) << 4));
+      phi = reinterpret_cast<uint4*>(row + (((c + 4) ^ sw) << 4));
+    }
+    uint4 a = *plo, b = *phi;
+    __nv_bfloat162* a2 = reinterpret_cast<__nv_bfloat162*>(&a);
+    __nv_bfloat162* b2 = reinterpret_cast<__nv_bfloat162*>(&b);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 x0 = __bfloat1622float2(a2[k]);
+      const float2 x1 = __bfloat1622float2(b2[k]);
+      const float2 c0 = cs[2 * k], c1 = cs[2 * k + 1];
+      a2[k] = __floats2bfloat162_rn(x0.x * c0.x - x1.x * c0.y, x0.y * c1.x - x1.y * c1.y);
+      b2[k] = __floats2bfloat162_rn(x0.x * c0.y + x1.x * c0.x, x0.y * c1.y + x1.y * c1.x);
+    }
+    *plo = a;
+    *phi = b;
+  }
+}
 
 template <int D, int P>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     segpaged_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                             const __grid_constant__ CUtensorMap tm_k,
-                            const __grid_constant__ CUtensorMap tm_v, const PrefillParams prm) {
+                            const __grid_constant__ CUtensorMap tm_v,
+                            const __grid_constant__ PrefillParams prm) {
   using C = PrefillCfg<D, P>;
   constexpr int S = C::kStages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -93,13 +152,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   uint8_t* sV = sK + S * C::kKVTileBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sV + S * C::kKVTileBytes);
   uint64_t* k_full = bars + kBarKFull;
-  uint64_t* k_empty = k_full + S;
+  uint64_t* k_ready = k_full + S;
+  uint64_t* k_empty = k_ready + S;
   uint64_t* v_full = k_empty + S;
   uint64_t* v_empty = v_full + S;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 64);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool fuse = prm.fuse_rope != 0;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars[kBarQFull], 1);
@@ -113,6 +174,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     }
     for (int s = 0; s < S; ++s) {
       mbar_init(&k_full[s], 1);
+      mbar_init(&k_ready[s], 64);
       mbar_init(&k_empty[s], 1);
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
@@ -134,15 +196,22 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int n_items = *prm.n_items;
+  const int G = gridDim.x, b = blockIdx.x;
   const WaitCtx wc{abort_flag, prm.error_word, prm.timeout_site};
 
+  if (warp < 4) {
+    // The register split happens inside each role's branch so that no control
+    // flow merges between setmaxnreg and the code it budgets for.
+    setmaxnreg_dec<kRegsAux>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       uint32_t k_issued = 0, v_issued = 0, q_uses = 0;
       bool ok = true;
       const int32_t oob_row = static_cast<int32_t>(prm.n_pages * P);
-      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+      for (int r = 0; ok; ++r) {
+        const int it = item_of_round(r, b, G);
+        if (it >= n_items) break;
         const Item w = prm.items[it];
         const int n_tiles = (w.e_end - w.e_begin + C::EPT - 1) / C::EPT;
         if (n_tiles == 0) continue;
@@ -208,6 +277,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       constexpr uint32_t idesc_s = idesc_bf16_f32(kRowsPerTile, kKeysPerTile, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(kRowsPerTile, D, true);
       const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
+      uint64_t* k_avail = fuse ? k_ready : k_full;
       uint32_t kv_iter = 0, q_uses = 0;
       uint32_t p_phase[2] = {0, 0}, o_uses[2] = {0, 0};
       bool ok = true;
@@ -217,8 +287,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::kBlockBytes + (kk & 3) * 32;
           const uint64_t a = desc_sw128(sQa + t * C::kQTileBytes + off, 16, 1024);
-          const uint64_t b = desc_sw128(sKa + st * C::kKVTileBytes + off, 16, 1024);
-          mma_bf16_ss(d, a, b, idesc_s, kk > 0 ? 1u : 0u);
+          const uint64_t bd = desc_sw128(sKa + st * C::kKVTileBytes + off, 16, 1024);
+          mma_bf16_ss(d, a, bd, idesc_s, kk > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int t, int st, bool acc) {
@@ -226,12 +296,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         const uint32_t a = tmem + C::col_s(t);
 #pragma unroll
         for (int kk = 0; kk < kKeysPerTile / 16; ++kk) {
-          const uint64_t b =
+          const uint64_t bd =
               desc_sw128(sVa + st * C::kKVTileBytes + kk * 16 * 128, C::kBlockBytes, 1024);
-          mma_bf16_ts(d, a + kk * 8, b, idesc_o, (acc || kk > 0) ? 1u : 0u);
+          mma_bf16_ts(d, a + kk * 8, bd, idesc_o, (acc || kk > 0) ? 1u : 0u);
         }
       };
-      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+      for (int r = 0; ok; ++r) {
+        const int it = item_of_round(r, b, G);
+        if (it >= n_items) break;
         const Item w = prm.items[it];
         const int n_tiles = (w.e_end - w.e_begin + C::EPT - 1) / C::EPT;
         if (n_tiles == 0) continue;
@@ -239,7 +311,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         ++q_uses;
         {
           const int st = kv_iter % S;
-          if (!(ok = mbar_wait(&k_full[st], (kv_iter / S) & 1, wc, 11))) break;
+          if (!(ok = mbar_wait(&k_avail[st], (kv_iter / S) & 1, wc, 11))) break;
           tc_fence_after();
           for (int t = 0; t < w.nh; ++t) {
             issue_s(t, st);
@@ -262,7 +334,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             tc_fence_after();
             issue_pv(t, st, j > 0);
             if (more) {
-              if (t == 0 && !(ok = mbar_wait(&k_full[stn], ((kj + 1) / S) & 1, wc, 15))) break;
+              if (t == 0 && !(ok = mbar_wait(&k_avail[stn], ((kj + 1) / S) & 1, wc, 15))) break;
               tc_fence_after();
               issue_s(t, stn);
               tc_commit(&bars[kBarSFull + t]);
@@ -284,9 +356,59 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       tc_commit(&bars[kBarDrain]);
       mbar_wait_drain(&bars[kBarDrain], 0);
     }
+  } else if (warp < 4) {
+    // ------------------------------------------------- RoPE relocation of K
+    if (fuse) {
+      const int rt = threadIdx.x - 64;
+      constexpr int CH = D / 16;
+      const int c = rt % CH;
+      int cur_delta = 0;
+      float2 cs[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) cs[q] = make_float2(1.f, 0.f);
+      uint32_t k_seen = 0;
+      bool ok = true;
+      for (int r = 0; ok; ++r) {
+        const int it = item_of_round(r, b, G);
+        if (it >= n_items) break;
+        const Item w = prm.items[it];
+        const int n_tiles = (w.e_end - w.e_begin + C::EPT - 1) / C::EPT;
+        for (int j = 0; j < n_tiles; ++j, ++k_seen) {
+          const int st = k_seen % S;
+          if (!(ok = mbar_wait(&k_full[st], (k_seen / S) & 1, wc, 30))) break;
+          uint8_t* tile = sK + st * C::kKVTileBytes;
+          for (int e = 0; e < C::EPT; ++e) {
+            const int idx = w.e_begin + j * C::EPT + e;
+            if (idx >= w.e_end) break;
+            const int delta = prm.entries[idx].delta;
+            if (delta == 0) continue;
+            if (delta != cur_delta) {
+              // angle = delta * f_m reduced modulo 2 pi in fp64 (2 pi split in
+              // a head and a tail constant), then sin / cos in fp32
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                const double a = static_cast<double>(delta) * prm.inv_freq[8 * c + q];
+                const double k = rint(a * 0.15915494309189535);
+                double red = fma(-k, 6.283185307179586, a);
+                red = fma(-k, 2.4492935982947064e-16, red);
+                float sn, cn;
+                sincosf(static_cast<float>(red), &sn, &cn);
+                cs[q] = make_float2(cn, sn);
+              }
+              cur_delta = delta;
+            }
+            rope_rotate_rows<D, P>(tile, e, rt, cs);
+          }
+          fence_proxy_async_smem();
+          mbar_arrive(&k_ready[st]);
+        }
+      }
+    }
+  }
   } else {
     // ------------------------------------------------------------ softmax
-    const int t = (warp - 2) >> 2;
+    setmaxnreg_inc<kRegsSoftmax>();
+    const int t = (warp - 4) >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
@@ -296,7 +418,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const int T = prm.total_tokens;
     uint32_t s_phase = 0, o_uses = 0;
     bool ok = true;
-    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+    for (int r = 0; ok; ++r) {
+      const int it = item_of_round(r, b, G);
+      if (it >= n_items) break;
       const Item w = prm.items[it];
       if (t >= w.nh) continue;
       const int n_tiles = (w.e_end - w.e_begin + C::EPT - 1) / C::EPT;
@@ -321,14 +445,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         s_phase ^= 1;
         tc_fence_after();
         float s[kKeysPerTile];
-#pragma unroll
-        for (int c = 0; c < kKeysPerTile / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld_x32(tS + 32 * c, r);
-          tmem_ld_wait(r);
-#pragma unroll
-          for (int k = 0; k < 32; ++k) s[32 * c + k] = __uint_as_float(r[k]);
-        }
+        tmem_ld_x128_wait(tS, s);
         // pages of this tile
         int lp[C::EPT], nv[C::EPT];
         bool full = true;
@@ -348,35 +465,40 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         full = full && lp[C::EPT - 1] + P - 1 <= i && (window < 0 || lp[0] > i - window);
         if (!full) {
 #pragma unroll
-          for (int c = 0; c < kKeysPerTile; ++c) {
-            const int e = c / P, r = c % P;
-            const int jpos = lp[e] + r;
-            const bool vis = r < nv[e] && jpos <= i && (window < 0 || jpos > i - window);
-            s[c] = vis ? s[c] : -INFINITY;
+          for (int cc = 0; cc < kKeysPerTile; ++cc) {
+            const int e = cc / P, rr = cc % P;
+            const int jpos = lp[e] + rr;
+            const bool vis = rr < nv[e] && jpos <= i && (window < 0 || jpos > i - window);
+            s[cc] = vis ? s[cc] : -INFINITY;
           }
         }
-        float mx = -INFINITY;
+        // row max: 8 independent chains, then a tree
+        float mx8[8];
 #pragma unroll
-        for (int c = 0; c < kKeysPerTile; ++c) mx = fmaxf(mx, s[c]);
+        for (int k = 0; k < 8; ++k) mx8[k] = s[k];
+#pragma unroll
+        for (int cc = 8; cc < kKeysPerTile; ++cc) mx8[cc & 7] = fmaxf(mx8[cc & 7], s[cc]);
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
         const float m_new = fmaxf(m_ref, mx * sl2);
         const bool resc = m_new > m_ref + kRescaleLog2;
         if (j > 0 && __any_sync(0xffffffffu, resc)) {
           const float alpha = resc ? ex2_approx(m_ref - m_new) : 1.f;
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t r[32];
-            tmem_ld_x32(tO + 32 * c, r);
-            tmem_ld_wait(r);
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t v[32];
+            tmem_ld_x32(tO + 32 * cc, v);
+            tmem_ld_wait(v);
 #pragma unroll
-            for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * alpha);
-            tmem_st_x32(tO + 32 * c, r);
+            for (int k = 0; k < 32; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * alpha);
+            tmem_st_x32(tO + 32 * cc, v);
           }
           tmem_st_wait();
           if (resc) l *= alpha;
         }
         if (resc) m_ref = m_new;
         const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
-        float rs = 0.f;
+        float rs4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           uint32_t pk[32];
@@ -384,12 +506,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           for (int k = 0; k < 32; ++k) {
             const float p0 = ex2_approx(fmaf(s[64 * half + 2 * k], sl2, -m_use));
             const float p1 = ex2_approx(fmaf(s[64 * half + 2 * k + 1], sl2, -m_use));
-            rs += p0 + p1;
+            rs4[k & 3] += p0 + p1;
             pk[k] = pack_bf16x2(p0, p1);
           }
           tmem_st_x32(tS + 32 * half, pk);
         }
-        l += rs;
+        l += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&bars[kBarPFull + t]);
@@ -401,16 +523,16 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld_x32(tO + 32 * c, r);
-        tmem_ld_wait(r);
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t v[32];
+        tmem_ld_x32(tO + 32 * cc, v);
+        tmem_ld_wait(v);
         if (valid) {
           uint32_t pk[16];
 #pragma unroll
           for (int k = 0; k < 16; ++k)
-            pk[k] = pack_bf16x2(__uint_as_float(r[2 * k]) * inv, __uint_as_float(r[2 * k + 1]) * inv);
-          uint4* dst = reinterpret_cast<uint4*>(prm.o + orow * D + 32 * c);
+            pk[k] = pack_bf16x2(__uint_as_float(v[2 * k]) * inv, __uint_as_float(v[2 * k + 1]) * inv);
+          uint4* dst = reinterpret_cast<uint4*>(prm.o + orow * D + 32 * cc);
 #pragma unroll
           for (int k = 0; k < 4; ++k)
             dst[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
@@ -501,6 +623,8 @@ static cudaError_t launch_typed(const PrefillLaunchArgs& a, cudaStream_t stream)
   prm.total_tokens = a.total_tokens;
   prm.n_pages = a.n_pages;
   prm.scale_log2 = a.scale_log2;
+  prm.fuse_rope = a.fuse_rope;
+  for (int m = 0; m < 64; ++m) prm.inv_freq[m] = m < D / 2 ? pow(a.rope_theta, -2.0 * m / D) : 0.0;
   segpaged_prefill_kernel<D, P><<<sms, kPrefillThreads, C::kSmemBytes, stream>>>(tq, tk, tv, prm);
   return cudaGetLastError();
 }

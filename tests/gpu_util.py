@@ -41,13 +41,20 @@ def run_select(lay, device="cuda"):
 
 
 class PrefillRun:
-    """rk_relocate_rope over the relocation plan, then rk_select_visible and
-    rk_segpaged_prefill(fuse_rope=0) on the relocated layout, on cuda:0.
+    """One pass of the CUDA path through the C ABI.
+
+    mode "relocate": rk_relocate_rope over the relocation plan, then
+    rk_select_visible and rk_segpaged_prefill(fuse_rope=0) on the relocated
+    layout.  mode "fused": rk_select_visible and
+    rk_segpaged_prefill(fuse_rope=1) on the original layout.
     ``o`` starts filled with the sentinel so untouched rows can be checked."""
 
-    def __init__(self, lay, q, k_pool, v_pool, with_lse=True):
+    def __init__(self, lay, q, k_pool, v_pool, with_lse=True, mode="relocate"):
         dev = q.device
-        jobs, rel = relocation_plan(lay)
+        if mode == "fused":
+            jobs, rel = np.zeros((0, 3), np.int32), lay
+        else:
+            jobs, rel = relocation_plan(lay)
         self.lay, self.rel, self.jobs = lay, rel, jobs
         extra = rel.n_pages - lay.n_pages
         self.k_rel = torch.cat([k_pool, torch.zeros((extra,) + tuple(k_pool.shape[1:]),
@@ -67,7 +74,7 @@ class PrefillRun:
         self.lse = (torch.full((lay.n_layers, lay.hq, lay.total_tokens), float("nan"),
                                device=dev) if with_lse else None)
         binding.segpaged_prefill(self.hl, q, self.k_rel, self.v_rel, self.vis, self.ws, self.o,
-                                 self.lse)
+                                 self.lse, fuse_rope=mode == "fused")
         torch.cuda.synchronize()
         self.status = binding.device_status(self.ws) | int(self.dev_err.item())
 

@@ -1,8 +1,9 @@
 """rk_segpaged_prefill (K3) against the fp64 oracle, element by element.
 
-The CUDA path runs K2 (relocation of every cached page with delta != 0),
-K1 on the relocated layout and K3; the oracle runs on the original layout and
-rotates the stored keys itself, so the comparison covers all three calls."""
+Two CUDA paths are checked against the same oracle rows: "fused" runs K1 and
+K3 with the RoPE relocation fused into K3's K loads; "relocate" runs K2 on
+every cached page with delta != 0, then K1 on the relocated layout and K3.
+The oracle runs on the original layout and rotates the stored keys itself."""
 import numpy as np
 import pytest
 import torch
@@ -61,25 +62,30 @@ def _untouched(lay, run):
     assert bad == 0
 
 
-def test_prefill_cfg1_all_rows():
+MODES = ("fused", "relocate")
+
+
+@pytest.mark.parametrize("mode", MODES)
+def test_prefill_cfg1_all_rows(mode):
     wl = synth.cfg1()
     lay = wl.layout
     q, k, v = wl.materialize("cpu")
-    run = PrefillRun(lay, q.cuda(), k.cuda(), v.cuda())
-    _check(lay, q, k, v, run, _all_rows(lay), "cfg1")
+    run = PrefillRun(lay, q.cuda(), k.cuda(), v.cuda(), mode=mode)
+    _check(lay, q, k, v, run, _all_rows(lay), f"cfg1 {mode}")
     _untouched(lay, run)
 
 
-def test_prefill_random_small_all_rows():
+@pytest.mark.parametrize("mode", MODES)
+def test_prefill_random_small_all_rows(mode):
     rng = np.random.default_rng(7)
     for n in range(40):
         lay = synth.random_small(rng, max_pages=12)
         wl = synth.tiny_workload(lay, seed=n)
         q, k, v = wl.materialize("cpu")
-        run = PrefillRun(lay, q.cuda(), k.cuda(), v.cuda())
+        run = PrefillRun(lay, q.cuda(), k.cuda(), v.cuda(), mode=mode)
         rows = _all_rows(lay)
         if rows.shape[0]:
-            _check(lay, q, k, v, run, rows, f"random layout {n}")
+            _check(lay, q, k, v, run, rows, f"random layout {n} {mode}")
         _untouched(lay, run)
 
 
@@ -89,16 +95,25 @@ def test_prefill_full_size_sampled(name, per_table):
     wl = synth.CONFIGS[name]()
     lay = wl.layout
     q, k, v = wl.materialize("cuda")
-    run = PrefillRun(lay, q, k, v)
     rows = sample_rows(lay, per_table, seed=11)
     # the oracle needs the sampled queries and the pools on the host
-    _check(lay, q, k.cpu(), v.cpu(), run, rows, name)
-    _untouched(lay, run)
+    o_ref, lse_ref, comp = oracle_rows(lay, q, k.cpu(), v.cpu(), rows)
+    assert comp.all()
+    for mode in MODES:
+        run = PrefillRun(lay, q, k, v, mode=mode)
+        assert run.status == 0, f"{name} {mode}: device status {run.status}"
+        o_got, lse_got = gpu_rows(run, rows)
+        assert_close(o_got, o_ref, f"{name} {mode} o")
+        assert np.abs(lse_got - lse_ref).max() <= 1e-2, f"{name} {mode} lse"
+        _untouched(lay, run)
+        del run
+        torch.cuda.empty_cache()
 
 
-def test_prefill_deterministic():
-    wl = synth.cfg1()
-    q, k, v = (t.cuda() for t in wl.materialize("cpu"))
-    a = PrefillRun(wl.layout, q, k, v)
-    b = PrefillRun(wl.layout, q, k, v)
+@pytest.mark.parametrize("mode", MODES)
+def test_prefill_deterministic(mode):
+    wl = synth.cfg3()
+    q, k, v = wl.materialize("cuda")
+    a = PrefillRun(wl.layout, q, k, v, mode=mode)
+    b = PrefillRun(wl.layout, q, k, v, mode=mode)
     assert torch.equal(a.o.view(torch.int16), b.o.view(torch.int16))
