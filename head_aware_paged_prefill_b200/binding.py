@@ -57,7 +57,7 @@ class RkSizes(ctypes.Structure):
 
 
 EXPORTS = ("rk_query_sizes", "rk_select_visible", "rk_relocate_rope", "rk_segpaged_prefill",
-           "rk_get_device_status")
+           "rk_get_device_status", "rk_select_visible_noalloc")
 
 _lib = None
 
@@ -77,6 +77,7 @@ def lib() -> ctypes.CDLL:
         L.rk_segpaged_prefill.argtypes = [vp, vp, vp, vp, vp, i32, ctypes.c_double, ctypes.c_float,
                                           vp, vp, vp, ctypes.c_size_t, vp]
         L.rk_get_device_status.argtypes = [vp, vp, vp]
+        L.rk_select_visible_noalloc.argtypes = [vp, vp, vp, vp, vp]
         for name in EXPORTS:
             getattr(L, name).restype = i32
         _lib = L
@@ -161,6 +162,15 @@ def select_visible(hl: HostLayout, vis: Visible, ws: torch.Tensor, stream=None):
     _check(lib().rk_select_visible(ctypes.byref(hl.dims), ctypes.byref(hl.layout),
                                    ctypes.byref(vis.struct), _ptr(ws), ws.numel(),
                                    _stream(stream)), "rk_select_visible")
+
+
+def select_visible_noalloc(hl: HostLayout, vis: Visible,
+                           device_error: Optional[torch.Tensor] = None, stream=None):
+    """Page tables and row ranges into ``vis`` without a caller workspace:
+    the library's own fixed-size device scratch is used (see include/rk.h)."""
+    _check(lib().rk_select_visible_noalloc(ctypes.byref(hl.dims), ctypes.byref(hl.layout),
+                                           ctypes.byref(vis.struct), _ptr(device_error),
+                                           _stream(stream)), "rk_select_visible_noalloc")
 
 
 def relocate_rope(k_src: torch.Tensor, k_dst: torch.Tensor, jobs: torch.Tensor, theta: float,

@@ -5,6 +5,7 @@
 
 #include <cmath>
 #include <cstring>
+#include <mutex>
 #include <vector>
 
 #include "rk_internal.h"
@@ -18,6 +19,8 @@ cudaError_t launch_relocate(const void* k_src, void* k_dst, const int32_t* jobs,
                             cudaStream_t stream);
 
 cudaError_t launch_prefill_args(const PrefillLaunchArgs& a, cudaStream_t stream);
+cudaError_t launch_select_tables_only(LayoutView* lv_dev, int n_tables, const rk_visible& vis,
+                                      WsHeader* hdr, cudaStream_t stream);
 
 namespace {
 
@@ -338,4 +341,79 @@ extern "C" rk_status rk_get_device_status(const void* workspace, int32_t* status
     return RK_ERR_CUDA;
   *status = v;
   return v == 0 ? RK_OK : RK_ERR_DEVICE;
+}
+
+// ----------------------------------------------------------------------------
+// rk_select_visible_noalloc: the page-table stage of rk_select_visible for
+// callers that cannot allocate device memory.  Its scratch (the device copy
+// of the layout and the device error word) lives in this file-scope array,
+// which every GPU that loads the library keeps until the process exits.
+// ----------------------------------------------------------------------------
+
+static constexpr size_t kNoAllocScratchBytes = size_t(1) << 20;  // 1 MiB
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kNoAllocMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device.  In host code
+// the array's name only stands for the symbol, so its address is looked up
+// once per device, with that device current, and cached.
+rk_status noalloc_scratch_address(uint8_t** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices)
+    return RK_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return RK_ERR_CUDA;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = static_cast<uint8_t*>(g_noalloc_addr[dev]);
+  return RK_OK;
+}
+}  // namespace
+
+extern "C" rk_status rk_select_visible_noalloc(const rk_dims* dims, const rk_layout* layout,
+                                               const rk_visible* out, int32_t* device_error,
+                                               void* stream) {
+  rk_status st = check_dims(dims);
+  if (st != RK_OK) return st;
+  Derived dv;
+  if ((st = check_layout(dims, layout, &dv)) != RK_OK) return st;
+  if (!out || !out->entries || !out->entry_start || !out->entry_count || !out->ranges ||
+      !out->range_start || !out->range_count)
+    return RK_ERR_INVALID_ARG;
+  if (!aligned(out->entries, 16) || !aligned(out->ranges, 8) || !aligned(out->entry_start, 4) ||
+      !aligned(out->entry_count, 4) || !aligned(out->range_start, 4) ||
+      !aligned(out->range_count, 4) || !aligned(device_error, 4))
+    return RK_ERR_INVALID_ARG;
+  if (out->entry_capacity < dv.entry_capacity || out->range_capacity < dv.range_capacity)
+    return RK_ERR_CAPACITY;
+  std::vector<int32_t> img;
+  build_layout_image(dims, layout, dv, &img);
+  const size_t layout_off = sizeof(WsHeader);
+  if (layout_off + 4 * img.size() > kNoAllocScratchBytes) return RK_ERR_CAPACITY;
+  uint8_t* scratch = nullptr;
+  if ((st = noalloc_scratch_address(&scratch)) != RK_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // the scratch keeps the previous call's contents: the header (with the
+  // error word) is rewritten as zeros and the layout image is rewritten whole
+  WsHeader hdr{};
+  hdr.n_tables = static_cast<int32_t>(dv.n_tables);
+  if (cudaMemcpyAsync(scratch, &hdr, sizeof hdr, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return RK_ERR_CUDA;
+  if (cudaMemcpyAsync(scratch + layout_off, img.data(), 4 * img.size(), cudaMemcpyHostToDevice,
+                      s) != cudaSuccess)
+    return RK_ERR_CUDA;
+  if (launch_select_tables_only(reinterpret_cast<LayoutView*>(scratch + layout_off),
+                                static_cast<int>(dv.n_tables), *out,
+                                reinterpret_cast<WsHeader*>(scratch), s) != cudaSuccess)
+    return RK_ERR_CUDA;
+  if (device_error && cudaMemcpyAsync(device_error, scratch, sizeof(int32_t),
+                                      cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return RK_ERR_CUDA;
+  return RK_OK;
 }

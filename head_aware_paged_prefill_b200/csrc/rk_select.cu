@@ -317,4 +317,11 @@ cudaError_t launch_select(LayoutView* lv_dev, int n_tables, const rk_visible& vi
   return cudaGetLastError();
 }
 
+// Page-table stage alone (no work list), for the no-allocation entry point.
+cudaError_t launch_select_tables_only(LayoutView* lv_dev, int n_tables, const rk_visible& vis,
+                                      WsHeader* hdr, cudaStream_t stream) {
+  if (n_tables > 0) select_tables_kernel<<<n_tables, kSelectThreads, 0, stream>>>(lv_dev, vis, hdr);
+  return cudaGetLastError();
+}
+
 }  // namespace rk

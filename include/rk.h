@@ -199,6 +199,32 @@ rk_status rk_segpaged_prefill(const rk_dims* dims, const void* q, const void* k_
  * otherwise, RK_ERR_CUDA if the copy failed. */
 rk_status rk_get_device_status(const void* workspace, int32_t* status, void* stream);
 
+/* Page tables and row ranges without any device memory from the caller
+ * beyond inputs and outputs.  The RedKnot pages have no counterpart of this
+ * call; it exists for callers that cannot allocate device memory: code whose
+ * framework owns every device allocation through its own pool, or a host
+ * thread that must not take the device-wide synchronisation a cudaMalloc can
+ * imply.  It computes exactly what rk_select_visible writes into `out`
+ * (entries, entry_start/count, ranges, range_start/count); it builds no
+ * attention work list, so it cannot feed rk_segpaged_prefill.
+ *   - Scratch: a 1 MiB array in the library's device memory (a file-scope
+ *     __device__ array, held by every GPU that loads the library until the
+ *     process exits) holds the device copy of the layout and the error word.
+ *     A layout whose copy does not fit (4 bytes per word of segments,
+ *     page_base, cu_seqlens, class map and retrieval lists, plus 256 bytes)
+ *     is rejected with RK_ERR_CAPACITY before any GPU work.
+ *   - The first call on a device looks up the scratch's device address with
+ *     that device current; make that first call before any stream capture.
+ *   - Every call shares the one scratch array and rewrites all of it that it
+ *     reads.  Calls whose GPU work overlaps (other streams, other threads)
+ *     race on it: order them on one stream.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ * device_error: device int32 (may be NULL) that receives the RK_DEV_* bits of
+ * this call.  Errors (host): RK_ERR_INVALID_ARG, RK_ERR_UNALIGNED,
+ * RK_ERR_CAPACITY, RK_ERR_CUDA. */
+rk_status rk_select_visible_noalloc(const rk_dims* dims, const rk_layout* layout,
+                                    const rk_visible* out, int32_t* device_error, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
