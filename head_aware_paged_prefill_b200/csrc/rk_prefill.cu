@@ -18,14 +18,18 @@
 //               KV tile, one box per page and 64-column block out of the pool.
 //   warp 1      tcgen05 issuer and TMEM owner.  S_t = Q_t K^T (M=128, N=128,
 //               K=D) into TMEM; O_t += P_t V (M=128, N=D, K=128) with P_t read
-//               from TMEM and V from shared memory (MN-major operand).
-//   warps 2-3   RoPE relocation of the K tile in shared memory (fuse_rope):
-//               rows of a page with delta != 0 are rotated by R(delta) in place
-//               before the QK^T MMA may read them.
+//               from TMEM and V from shared memory (MN-major operand), issued
+//               per 64-key half as soon as that half of P is stored.  Order
+//               per KV tile: PV_0, S_0(next), PV_1, S_1(next), so the two Q
+//               tiles' softmax phases alternate.
+//   warps 2-3   RoPE relocation (fuse_rope): rotate the Q tiles by -delta once
+//               per run of tiles sharing a delta, and the K pages of a tile that
+//               mixes deltas by their difference.
 //   warps 4-7   softmax warpgroup of Q tile 0, warps 8-11 of Q tile 1: one
 //               TMEM lane (= one query row) per thread; online softmax in the
 //               log2 domain, O rescaled in TMEM only when the running max
-//               grows by more than 2^8, P written back over S as bf16.
+//               grows by more than 2^8, P written back over S as bf16 in
+//               16-column quarters.
 // Registers are rebalanced with setmaxnreg: the first warpgroup keeps 80 per
 // thread, the two softmax warpgroups get 208.
 //
@@ -40,7 +44,6 @@
 #include "sm100.cuh"
 
 namespace rk {
-
 constexpr int kPrefillThreads = 384;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr uint32_t kRegsAux = 80;       // warps 0-3
@@ -84,55 +87,98 @@ enum : int {
   kBarQFull = 0,
   kBarQEmpty = 1,
   kBarSFull = 2,   // [2]
-  kBarPFull = 4,   // [2]
+  kBarPLo = 4,     // [2] P columns of keys 0-63 stored
   kBarOFull = 6,   // [2]
   kBarOEmpty = 8,  // [2]
   kBarDrain = 10,  // MMA completion before TMEM is released
-  kBarKFull = 11,  // [kStages] x 5 groups follow (k_full, k_ready, k_empty, v_full, v_empty)
+  kBarPHi = 11,    // [2] P columns of keys 64-127 stored
+  kBarQReady = 13,   // fused: the Q tiles hold the rotation the next S needs
+  kBarQFree = 14,    // fused: every S reading the current Q rotation completed
+  kBarQReload = 15,  // fused: original Q re-fetched for a new rotation
+  kBarKFull = 16,  // [kStages] x 5 groups follow (k_full, k_ready, k_empty, v_full, v_empty)
 };
+
+// kEmuNum pairs of exponentials in every kEmuDen can go through the FMA-pipe
+// polynomial instead of the MUFU (16 ex2 per clock per SM).  Measured on
+// B200 at D = 128 the softmax is latency bound rather than MUFU bound, and
+// every emulated fraction tried (1/4, 3/8, 1/2) was slower, so the default
+// keeps all exponentials on the MUFU.
+#ifndef RK_EMU_NUM
+#define RK_EMU_NUM 0
+#endif
+#ifndef RK_EMU_DEN
+#define RK_EMU_DEN 4
+#endif
+constexpr int kEmuNum = RK_EMU_NUM;
+constexpr int kEmuDen = RK_EMU_DEN;
 
 // Item of round r for CTA b (boustrophedon over the cost-sorted list).
 __device__ __forceinline__ int item_of_round(int r, int b, int g) {
   return r * g + ((r & 1) ? (g - 1 - b) : b);
 }
 
-// Rotates, in place, the rows of one page of a K tile held in shared memory
-// (128-byte swizzle: 16-byte chunk c of row r lives at chunk c ^ (r & 7)).
-// Thread rt of 64 owns chunk c of rows r0, r0 + rstep, ...; pair (m, m + D/2)
-// of a row sits in chunks c and c + D/16 (D = 64) or at the same chunk of the
-// next 64-column block (D = 128).
-template <int D, int P>
-__device__ __forceinline__ void rope_rotate_rows(uint8_t* tile, int e, int rt, const float2 (&cs)[8]) {
-  constexpr int CH = D / 16;  // chunk pairs per row
+// cos / sin of delta * f_m for the 8 frequencies m = 8c .. 8c+7 a thread
+// owns, as packed pairs (m, m+1): the angle is formed and reduced modulo 2 pi
+// in fp64 (2 pi split in a head and a tail constant), sin / cos in fp32.
+__device__ __forceinline__ void rope_table(int delta, int c, const double* inv_freq,
+                                           uint64_t (&cos2)[4], uint64_t (&sin2)[4]) {
+#pragma unroll
+  for (int q = 0; q < 8; q += 2) {
+    float cs[2], sn[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const double a = static_cast<double>(delta) * inv_freq[8 * c + q + u];
+      const double k = rint(a * 0.15915494309189535);
+      double red = fma(-k, 6.283185307179586, a);
+      red = fma(-k, 2.4492935982947064e-16, red);
+      sincosf(static_cast<float>(red), &sn[u], &cs[u]);
+    }
+    cos2[q / 2] = f2_pack(cs[0], cs[1]);
+    sin2[q / 2] = f2_pack(sn[0], sn[1]);
+  }
+}
+
+// Rotates rows [row_lo, row_hi) of a 128-row bf16 tile in shared memory (the
+// K or Q operand layout: 64-column blocks of 128-byte rows, 128-byte swizzle,
+// so 16-byte chunk c of row r sits at chunk c ^ (r & 7)).  Thread rt of 64
+// owns chunk c of rows r0, r0 + RSTEP, ...; the rotate-half partner of chunk c
+// is chunk c + D/16 of the same row (D = 64) or chunk c of the next column
+// block (D = 128).  Packed fp32 math, one bf16 rounding per element.
+template <int D>
+__device__ __forceinline__ void rope_rotate_rows(uint8_t* tile, int row_lo, int row_hi, int rt,
+                                                 const uint64_t (&cos2)[4],
+                                                 const uint64_t (&sin2)[4]) {
+  constexpr int CH = D / 16;
   constexpr int RSTEP = 64 / CH;
-  const int c = rt % CH, r0 = rt / CH;
-#pragma unroll 4
-  for (int r = r0; r < kKeysPerTile; r += RSTEP) {
-    if (r / P != e) continue;
+  const int c = rt % CH;
+  const int first = row_lo + ((rt / CH) - row_lo % RSTEP + RSTEP) % RSTEP;
+#pragma unroll 2
+  for (int r = first; r < row_hi; r += RSTEP) {
     const int sw = r & 7;
     uint8_t* row = tile + r * 128;
-    uint4* plo;
-    uint4* phi;
-    if constexpr (D == 128) {
-      plo = reinterpret_cast<uint4*>(row + ((c ^ sw) << 4));
-      phi = reinterpret_cast<uint4*>(row + kKeysPerTile * 128 + ((c ^ sw) << 4));
-    } else {
-      plo = reinterpret_cast<uint4*>(row + ((c ^ sw) << 4));
-      phi = reinterpret_cast<uint4*>(row + (((c + 4) ^ sw) << 4));
-    }
-    uint4 a = *plo, b = *phi;
-    __nv_bfloat162* a2 = reinterpret_cast<__nv_bfloat162*>(&a);
-    __nv_bfloat162* b2 = reinterpret_cast<__nv_bfloat162*>(&b);
+    uint4* plo = reinterpret_cast<uint4*>(row + ((c ^ sw) << 4));
+    uint4* phi = D == 128 ? reinterpret_cast<uint4*>(row + kKeysPerTile * 128 + ((c ^ sw) << 4))
+                          : reinterpret_cast<uint4*>(row + (((c + CH) ^ sw) << 4));
+    uint4 a = *plo, bq = *phi;
+    const uint32_t* aw = reinterpret_cast<const uint32_t*>(&a);
+    const uint32_t* bw = reinterpret_cast<const uint32_t*>(&bq);
+    uint32_t ya[4], yb[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      const float2 x0 = __bfloat1622float2(a2[k]);
-      const float2 x1 = __bfloat1622float2(b2[k]);
-      const float2 c0 = cs[2 * k], c1 = cs[2 * k + 1];
-      a2[k] = __floats2bfloat162_rn(x0.x * c0.x - x1.x * c0.y, x0.y * c1.x - x1.y * c1.y);
-      b2[k] = __floats2bfloat162_rn(x0.x * c0.y + x1.x * c0.x, x0.y * c1.y + x1.y * c1.x);
+      // x0 = (x_m, x_m+1), x1 = (x_{m+D/2}, x_{m+1+D/2})
+      const uint64_t x0 = f2_pack(__uint_as_float(aw[k] << 16), __uint_as_float(aw[k] & 0xFFFF0000u));
+      const uint64_t x1 = f2_pack(__uint_as_float(bw[k] << 16), __uint_as_float(bw[k] & 0xFFFF0000u));
+      // y0 = x0 cos - x1 sin ; y1 = x0 sin + x1 cos
+      const uint64_t y0 = f2_fma(x0, cos2[k], f2_mul_neg(x1, sin2[k]));
+      const uint64_t y1 = f2_fma(x0, sin2[k], f2_mul(x1, cos2[k]));
+      float lo, hi;
+      f2_unpack(y0, lo, hi);
+      ya[k] = pack_bf16x2(lo, hi);
+      f2_unpack(y1, lo, hi);
+      yb[k] = pack_bf16x2(lo, hi);
     }
-    *plo = a;
-    *phi = b;
+    *plo = make_uint4(ya[0], ya[1], ya[2], ya[3]);
+    *phi = make_uint4(yb[0], yb[1], yb[2], yb[3]);
   }
 }
 
@@ -166,9 +212,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     mbar_init(&bars[kBarQFull], 1);
     mbar_init(&bars[kBarQEmpty], 1);
     mbar_init(&bars[kBarDrain], 1);
+    mbar_init(&bars[kBarQReady], 64);
+    mbar_init(&bars[kBarQFree], 1);
+    mbar_init(&bars[kBarQReload], 1);
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bars[kBarSFull + t], 1);
-      mbar_init(&bars[kBarPFull + t], 128);
+      mbar_init(&bars[kBarPLo + t], 128);
+      mbar_init(&bars[kBarPHi + t], 128);
       mbar_init(&bars[kBarOFull + t], 1);
       mbar_init(&bars[kBarOEmpty + t], 128);
     }
@@ -278,7 +328,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       constexpr uint32_t idesc_o = idesc_bf16_f32(kRowsPerTile, D, true);
       const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
       uint64_t* k_avail = fuse ? k_ready : k_full;
-      uint32_t kv_iter = 0, q_uses = 0;
+      uint32_t kv_iter = 0, q_uses = 0, qrd_uses = 0;
       uint32_t p_phase[2] = {0, 0}, o_uses[2] = {0, 0};
       bool ok = true;
       auto issue_s = [&](int t, int st) {
@@ -291,11 +341,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           mma_bf16_ss(d, a, bd, idesc_s, kk > 0 ? 1u : 0u);
         }
       };
-      auto issue_pv = [&](int t, int st, bool acc) {
+      // O_t (+)= P_t V over keys [64 half, 64 half + 64)
+      auto issue_pv = [&](int t, int st, int half, bool acc) {
         const uint32_t d = tmem + C::col_o(t);
         const uint32_t a = tmem + C::col_s(t);
 #pragma unroll
-        for (int kk = 0; kk < kKeysPerTile / 16; ++kk) {
+        for (int kk = 4 * half; kk < 4 * half + 4; ++kk) {
           const uint64_t bd =
               desc_sw128(sVa + st * C::kKVTileBytes + kk * 16 * 128, C::kBlockBytes, 1024);
           mma_bf16_ts(d, a + kk * 8, bd, idesc_o, (acc || kk > 0) ? 1u : 0u);
@@ -307,8 +358,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         const Item w = prm.items[it];
         const int n_tiles = (w.e_end - w.e_begin + C::EPT - 1) / C::EPT;
         if (n_tiles == 0) continue;
-        if (!(ok = mbar_wait(&bars[kBarQFull], q_uses & 1, wc, 10))) break;
+        if (fuse) {
+          if (!(ok = mbar_wait(&bars[kBarQReady], qrd_uses & 1, wc, 10))) break;
+          ++qrd_uses;
+        } else if (!(ok = mbar_wait(&bars[kBarQFull], q_uses & 1, wc, 10))) {
+          break;
+        }
         ++q_uses;
+        int dcur = prm.entries[w.e_begin].delta;
         {
           const int st = kv_iter % S;
           if (!(ok = mbar_wait(&k_avail[st], (kv_iter / S) & 1, wc, 11))) break;
@@ -324,16 +381,25 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           const int st = kj % S;
           const int stn = (kj + 1) % S;
           const bool more = j + 1 < n_tiles;
+          // fused: a tile whose keys need another Q rotation waits for it
+          const int dnext =
+              (fuse && more) ? __ldg(&prm.entries[w.e_begin + (j + 1) * C::EPT].delta) : dcur;
+          const bool qswitch = fuse && dnext != dcur;
           for (int t = 0; t < w.nh && ok; ++t) {
-            if (!(ok = mbar_wait(&bars[kBarPFull + t], p_phase[t], wc, 12))) break;
-            p_phase[t] ^= 1;
+            if (!(ok = mbar_wait(&bars[kBarPLo + t], p_phase[t], wc, 12))) break;
             if (j == 0 && o_uses[t] > 0 &&
                 !(ok = mbar_wait(&bars[kBarOEmpty + t], (o_uses[t] - 1) & 1, wc, 13)))
               break;
             if (t == 0 && !(ok = mbar_wait(&v_full[st], (kj / S) & 1, wc, 14))) break;
             tc_fence_after();
-            issue_pv(t, st, j > 0);
-            if (more) {
+            issue_pv(t, st, 0, j > 0);
+            if (!(ok = mbar_wait(&bars[kBarPHi + t], p_phase[t], wc, 16))) break;
+            p_phase[t] ^= 1;
+            tc_fence_after();
+            issue_pv(t, st, 1, true);
+            if (qswitch) {
+              if (t == 0) tc_commit(&bars[kBarQFree]);
+            } else if (more) {
               if (t == 0 && !(ok = mbar_wait(&k_avail[stn], ((kj + 1) / S) & 1, wc, 15))) break;
               tc_fence_after();
               issue_s(t, stn);
@@ -341,6 +407,17 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             }
           }
           if (!ok) break;
+          if (qswitch) {
+            if (!(ok = mbar_wait(&bars[kBarQReady], qrd_uses & 1, wc, 17))) break;
+            ++qrd_uses;
+            if (!(ok = mbar_wait(&k_avail[stn], ((kj + 1) / S) & 1, wc, 18))) break;
+            tc_fence_after();
+            for (int t = 0; t < w.nh; ++t) {
+              issue_s(t, stn);
+              tc_commit(&bars[kBarSFull + t]);
+            }
+            dcur = dnext;
+          }
           tc_commit(&v_empty[st]);
           if (more) tc_commit(&k_empty[stn]);
         }
@@ -357,47 +434,85 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       mbar_wait_drain(&bars[kBarDrain], 0);
     }
   } else if (warp < 4) {
-    // ------------------------------------------------- RoPE relocation of K
+    // ------------------------------------------- RoPE relocation (fused)
+    // q . R(d) k = (R(-d) q) . k: the Q tiles are rotated by -d once per run
+    // of tiles whose keys share the relocation d (a cached segment), so the
+    // K tiles go to the tensor cores as loaded.  A tile whose pages carry
+    // different deltas (a segment boundary inside the tile) has those pages
+    // rotated by their delta minus the Q rotation's.  Before each new Q
+    // rotation the original Q is fetched again, so every Q element is rounded
+    // to bf16 once.
     if (fuse) {
       const int rt = threadIdx.x - 64;
-      constexpr int CH = D / 16;
-      const int c = rt % CH;
-      int cur_delta = 0;
-      float2 cs[8];
+      const int c = rt % (D / 16);
+      uint32_t k_seen = 0, q_uses = 0, qf_uses = 0, qr_uses = 0;
+      int tab_delta = 0;
+      uint64_t cos2[4], sin2[4];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) cs[q] = make_float2(1.f, 0.f);
-      uint32_t k_seen = 0;
+      for (int k = 0; k < 4; ++k) {
+        cos2[k] = f2_pack(1.f, 1.f);
+        sin2[k] = f2_pack(0.f, 0.f);
+      }
+      auto table = [&](int delta) {
+        if (delta != tab_delta) {
+          rope_table(delta, c, prm.inv_freq, cos2, sin2);
+          tab_delta = delta;
+        }
+      };
       bool ok = true;
       for (int r = 0; ok; ++r) {
         const int it = item_of_round(r, b, G);
         if (it >= n_items) break;
         const Item w = prm.items[it];
         const int n_tiles = (w.e_end - w.e_begin + C::EPT - 1) / C::EPT;
-        for (int j = 0; j < n_tiles; ++j, ++k_seen) {
+        if (n_tiles == 0) continue;
+        if (!(ok = mbar_wait(&bars[kBarQFull], q_uses & 1, wc, 31))) break;
+        ++q_uses;
+        int dq = prm.entries[w.e_begin].delta;
+        if (dq != 0) {
+          table(-dq);
+          for (int t = 0; t < w.nh; ++t)
+            rope_rotate_rows<D>(sQ + t * C::kQTileBytes, 0, kRowsPerTile, rt, cos2, sin2);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&bars[kBarQReady]);
+        for (int j = 0; j < n_tiles && ok; ++j, ++k_seen) {
+          const int dt = prm.entries[w.e_begin + j * C::EPT].delta;
+          if (j > 0 && dt != dq) {
+            if (!(ok = mbar_wait(&bars[kBarQFree], qf_uses & 1, wc, 32))) break;
+            ++qf_uses;
+            if (rt == 0) {
+              mbar_arrive_expect_tx(&bars[kBarQReload], w.nh * C::kQTileBytes);
+              for (int t = 0; t < w.nh; ++t)
+                for (int cb = 0; cb < C::KB; ++cb)
+                  tma_load_3d(sQ + t * C::kQTileBytes + cb * C::kBlockBytes, &tm_q,
+                              &bars[kBarQReload], cb * 64, w.qh0 + t, w.q_row0 + w.row_begin);
+            }
+            if (!(ok = mbar_wait(&bars[kBarQReload], qr_uses & 1, wc, 33))) {
+              // let the copy this warp started land before the CTA exits
+              if (rt == 0) mbar_wait_drain(&bars[kBarQReload], qr_uses & 1);
+              break;
+            }
+            ++qr_uses;
+            if (dt != 0) {
+              table(-dt);
+              for (int t = 0; t < w.nh; ++t)
+                rope_rotate_rows<D>(sQ + t * C::kQTileBytes, 0, kRowsPerTile, rt, cos2, sin2);
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&bars[kBarQReady]);
+            dq = dt;
+          }
           const int st = k_seen % S;
           if (!(ok = mbar_wait(&k_full[st], (k_seen / S) & 1, wc, 30))) break;
           uint8_t* tile = sK + st * C::kKVTileBytes;
-          for (int e = 0; e < C::EPT; ++e) {
+          for (int e = 1; e < C::EPT; ++e) {
             const int idx = w.e_begin + j * C::EPT + e;
             if (idx >= w.e_end) break;
-            const int delta = prm.entries[idx].delta;
-            if (delta == 0) continue;
-            if (delta != cur_delta) {
-              // angle = delta * f_m reduced modulo 2 pi in fp64 (2 pi split in
-              // a head and a tail constant), then sin / cos in fp32
-#pragma unroll
-              for (int q = 0; q < 8; ++q) {
-                const double a = static_cast<double>(delta) * prm.inv_freq[8 * c + q];
-                const double k = rint(a * 0.15915494309189535);
-                double red = fma(-k, 6.283185307179586, a);
-                red = fma(-k, 2.4492935982947064e-16, red);
-                float sn, cn;
-                sincosf(static_cast<float>(red), &sn, &cn);
-                cs[q] = make_float2(cn, sn);
-              }
-              cur_delta = delta;
-            }
-            rope_rotate_rows<D, P>(tile, e, rt, cs);
+            const int de = prm.entries[idx].delta;
+            if (de == dq) continue;
+            table(de - dq);
+            rope_rotate_rows<D>(tile, e * P, e * P + P, rt, cos2, sin2);
           }
           fence_proxy_async_smem();
           mbar_arrive(&k_ready[st]);
@@ -441,14 +556,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       const int window = w.window;
       float m_ref = -INFINITY, l = 0.f;
       for (int j = 0; j < n_tiles && ok; ++j) {
-        if (!(ok = mbar_wait(&bars[kBarSFull + t], s_phase, wc, 20))) break;
-        s_phase ^= 1;
-        tc_fence_after();
-        float s[kKeysPerTile];
-        tmem_ld_x128_wait(tS, s);
-        // pages of this tile
+        // pages of this tile (loaded before the wait, so their latency hides)
         int lp[C::EPT], nv[C::EPT];
-        bool full = true;
 #pragma unroll
         for (int e = 0; e < C::EPT; ++e) {
           const int idx = w.e_begin + j * C::EPT + e;
@@ -460,8 +569,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             lp[e] = 0;
             nv[e] = 0;
           }
-          full = full && nv[e] == P;
         }
+        if (!(ok = mbar_wait(&bars[kBarSFull + t], s_phase, wc, 20))) break;
+        s_phase ^= 1;
+        tc_fence_after();
+        float s[kKeysPerTile];
+        tmem_ld_x128_wait(tS, s);
+        bool full = true;
+#pragma unroll
+        for (int e = 0; e < C::EPT; ++e) full = full && nv[e] == P;
         full = full && lp[C::EPT - 1] + P - 1 <= i && (window < 0 || lp[0] > i - window);
         if (!full) {
 #pragma unroll
@@ -472,14 +588,16 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             s[cc] = vis ? s[cc] : -INFINITY;
           }
         }
-        // row max: 8 independent chains, then a tree
+        // row max: 3-input max over 8 independent chains, then a tree
         float mx8[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) mx8[k] = s[k];
+        for (int k = 0; k < 8; ++k) mx8[k] = fmax3(s[k], s[8 + k], s[16 + k]);
 #pragma unroll
-        for (int cc = 8; cc < kKeysPerTile; ++cc) mx8[cc & 7] = fmaxf(mx8[cc & 7], s[cc]);
-        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        for (int cc = 24; cc < kKeysPerTile; cc += 16)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mx8[k] = fmax3(mx8[k], s[cc + k], s[cc + 8 + k]);
+        const float mx = fmaxf(fmax3(mx8[0], mx8[1], mx8[2]),
+                               fmax3(fmax3(mx8[3], mx8[4], mx8[5]), mx8[6], mx8[7]));
         const float m_new = fmaxf(m_ref, mx * sl2);
         const bool resc = m_new > m_ref + kRescaleLog2;
         if (j > 0 && __any_sync(0xffffffffu, resc)) {
@@ -498,23 +616,45 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
         if (resc) m_ref = m_new;
         const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
-        float rs4[4] = {0.f, 0.f, 0.f, 0.f};
+        const uint64_t scale2 = f2_pack(sl2, sl2);
+        const uint64_t neg_m2 = f2_pack(-m_use, -m_use);
+        uint64_t acc2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-          uint32_t pk[32];
+          float* sh = s + 64 * half;
 #pragma unroll
           for (int k = 0; k < 32; ++k) {
-            const float p0 = ex2_approx(fmaf(s[64 * half + 2 * k], sl2, -m_use));
-            const float p1 = ex2_approx(fmaf(s[64 * half + 2 * k + 1], sl2, -m_use));
-            rs4[k & 3] += p0 + p1;
-            pk[k] = pack_bf16x2(p0, p1);
+            const uint64_t x2 = f2_fma(f2_pack(sh[2 * k], sh[2 * k + 1]), scale2, neg_m2);
+            f2_unpack(x2, sh[2 * k], sh[2 * k + 1]);
           }
-          tmem_st_x32(tS + 32 * half, pk);
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            if (k % kEmuDen >= kEmuDen - kEmuNum) {
+              exp2_poly_pair(sh[2 * k], sh[2 * k + 1], sh[2 * k], sh[2 * k + 1]);
+            } else {
+              sh[2 * k] = ex2_approx(sh[2 * k]);
+              sh[2 * k + 1] = ex2_approx(sh[2 * k + 1]);
+            }
+          }
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+              const int kk = 16 * q + k;
+              acc2[k & 1] = f2_add(acc2[k & 1], f2_pack(sh[2 * kk], sh[2 * kk + 1]));
+              pk[k] = pack_bf16x2(sh[2 * kk], sh[2 * kk + 1]);
+            }
+            tmem_st_x16(tS + 32 * half + 16 * q, pk);
+          }
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(&bars[(half ? kBarPHi : kBarPLo) + t]);
         }
-        l += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&bars[kBarPFull + t]);
+        float a0, a1, b0, b1;
+        f2_unpack(acc2[0], a0, a1);
+        f2_unpack(acc2[1], b0, b1);
+        l += (a0 + a1) + (b0 + b1);
       }
       if (!ok) break;
       // epilogue: O / l -> bf16
@@ -638,3 +778,4 @@ cudaError_t launch_prefill_args(const PrefillLaunchArgs& a, cudaStream_t stream)
 }
 
 }  // namespace rk
+
