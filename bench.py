@@ -126,6 +126,23 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def max_over_ranks(x: float, dist, device) -> float:
+    """The largest x over all ranks (every rank gets it); plain x without a
+    process group."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(world: int, work_per_rank: float, steps: int, max_total_ms: float) -> float:
+    """Whole-job throughput: every rank ran `steps` steps of `work_per_rank`;
+    the job took as long as the slowest rank."""
+    return world * work_per_rank * steps / (max_total_ms * 1e-3)
+
+
 def _gpu_id(torch, dev) -> str:
     try:
         return "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
@@ -320,16 +337,12 @@ def main():
     clocks = sampler.stop()
     step_ms = [a.elapsed_time(b) for a, b in ev]
     k3_ms = [a.elapsed_time(b) for a, b in ev3]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), dist if world > 1 else None, dev)
     st = pre.status()
     if st != 0:
         raise SystemExit(f"device error word {st:#x} after the timed steps")
     ms_per_step = total_ms / K
-    value = world * flops * K / (total_ms * 1e-3) / 1e12
+    value = weak_scaling_value(world, flops, K, total_ms) / 1e12
 
     # end to end through the public API: pinned host inputs in, o back to host
     q_h = q.cpu().pin_memory()
@@ -349,11 +362,8 @@ def main():
         b.record(stream)
         b.synchronize()
         e2e_ms += a.elapsed_time(b)
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * flops * E / (e2e_ms * 1e-3) / 1e12
+    e2e_ms = max_over_ranks(e2e_ms, dist if world > 1 else None, dev)
+    e2e_value = weak_scaling_value(world, flops, E, e2e_ms) / 1e12
     h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h))
     d2h = o_h.numel() * o_h.element_size()
 
@@ -365,18 +375,45 @@ def main():
 
     reloc = _bench_relocate(torch, lay, k, dev, flush, stream, args.reloc_reps, peaks, peak_kind)
 
+    # the other mode of the same path, timed the same way (context)
+    other = "relocate" if args.mode == "fused" else "fused"
+    alt = SegPagedPrefill(lay, dev, mode=other)
+    alt.load(q, k, v)
+    for _ in range(args.warmup):
+        alt.compute()
+    torch.cuda.synchronize()
+    alt_ms, alt_k3 = 0.0, 0.0
+    for s_ in range(K):
+        flush.zero_()
+        ev[s_][0].record(stream)
+        alt.compute(k3_events=ev3[s_])
+        ev[s_][1].record(stream)
+    torch.cuda.synchronize()
+    alt_ms = sum(a.elapsed_time(b) for a, b in ev) / K
+    alt_k3 = statistics.mean(a.elapsed_time(b) for a, b in ev3)
+    st = alt.status()
+    other_mode = {"mode": other, "value": flops / (alt_ms * 1e-3) / 1e12, "unit": UNIT,
+                  "ms_per_step": alt_ms, "k3_tflops": flops / (alt_k3 * 1e-3) / 1e12,
+                  "device_status": st}
+    del alt
+
     cpu_baseline = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
-        rows, pairs = _oracle_sample_rows(lay, 256, seed=0)
-        dt = _time_oracle(lay, qc, kc, vc, rows)
-        n_rows = int(max(256, min(200000, 256 * args.cpu_seconds / max(dt, 1e-3))))
-        rows, pairs = _oracle_sample_rows(lay, n_rows, seed=1)
-        dt = _time_oracle(lay, qc, kc, vc, rows)
-        cpu_baseline = {"value": 4 * lay.d * pairs / dt / 1e12, "unit": UNIT,
+        # batches of seeded rows until about args.cpu_seconds of oracle time
+        n_rows, tot_rows, tot_pairs, tot_t, seed = 1024, 0, 0, 0.0, 1
+        while tot_t < args.cpu_seconds:
+            rows, pairs = _oracle_sample_rows(lay, n_rows, seed=seed)
+            tot_t += _time_oracle(lay, qc, kc, vc, rows)
+            tot_rows += n_rows
+            tot_pairs += pairs
+            seed += 1
+            n_rows = min(2 * n_rows, 65536)
+        cpu_baseline = {"value": 4 * lay.d * tot_pairs / tot_t / 1e12, "unit": UNIT,
                         "cores": os.cpu_count() or 1, "kind": "oracle",
-                        "sample": f"{n_rows} seeded (layer, q head, row) samples of the same "
-                                  f"workload, {pairs} visible pairs, {dt:.1f} s"}
+                        "sample": f"{tot_rows} seeded (layer, q head, row) samples of the same "
+                                  f"workload in {seed - 1} batches, {tot_pairs} visible pairs, "
+                                  f"{tot_t:.1f} s"}
 
     if world > 1:
         dist.barrier()
@@ -394,7 +431,7 @@ def main():
                    "l2": "flushed between timed steps (256 MiB write)"},
         "pct_bf16_peak": 100.0 * value / world / peak,
         "pct_bf16_spec": 100.0 * value / world / SPEC_BF16_TFLOPS,
-        "tokens_per_s": world * tokens * K / (total_ms * 1e-3),
+        "tokens_per_s": weak_scaling_value(world, tokens, K, total_ms),
         "roofline": {"bound": "tensor", "kernel": "segpaged_prefill_kernel",
                      "achieved": achieved, "peak": peak, "unit": UNIT, "frac": achieved / peak,
                      "peak_kind": f"bf16 burst, {peak_kind}", "traffic": traffic,
@@ -405,6 +442,7 @@ def main():
         "gpu_launches": K * pre.launches_per_run,
         "clocks": clocks,
         "mode": args.mode,
+        "other_mode": other_mode,
         "relocate_roofline": reloc,
     }
     print(json.dumps(line), flush=True)

@@ -57,7 +57,7 @@ class RkSizes(ctypes.Structure):
 
 
 EXPORTS = ("rk_query_sizes", "rk_select_visible", "rk_relocate_rope", "rk_segpaged_prefill",
-           "rk_get_device_status", "rk_select_visible_noalloc")
+           "rk_get_device_status", "rk_select_visible_noalloc", "rk_selftest_bounded_wait")
 
 _lib = None
 
@@ -78,6 +78,7 @@ def lib() -> ctypes.CDLL:
                                           vp, vp, vp, ctypes.c_size_t, vp]
         L.rk_get_device_status.argtypes = [vp, vp, vp]
         L.rk_select_visible_noalloc.argtypes = [vp, vp, vp, vp, vp]
+        L.rk_selftest_bounded_wait.argtypes = [vp, i32, vp]
         for name in EXPORTS:
             getattr(L, name).restype = i32
         _lib = L
@@ -195,6 +196,11 @@ def segpaged_prefill(hl: HostLayout, q: torch.Tensor, k_pool: torch.Tensor,
                                      float(lay.theta), float(lay.softmax_scale), _ptr(o),
                                      _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)),
            "rk_segpaged_prefill")
+
+
+def selftest_bounded_wait(word: torch.Tensor, wait_ms: int, stream=None):
+    _check(lib().rk_selftest_bounded_wait(_ptr(word), int(wait_ms), _stream(stream)),
+           "rk_selftest_bounded_wait")
 
 
 def device_status(ws: torch.Tensor, stream=None) -> int:

@@ -19,6 +19,7 @@ cudaError_t launch_relocate(const void* k_src, void* k_dst, const int32_t* jobs,
                             cudaStream_t stream);
 
 cudaError_t launch_prefill_args(const PrefillLaunchArgs& a, cudaStream_t stream);
+cudaError_t launch_selftest_wait(int* word, int wait_ms, cudaStream_t stream);
 cudaError_t launch_select_tables_only(LayoutView* lv_dev, int n_tables, const rk_visible& vis,
                                       WsHeader* hdr, cudaStream_t stream);
 
@@ -331,6 +332,15 @@ extern "C" rk_status rk_segpaged_prefill(const rk_dims* dims, const void* q, con
   if (dims->total_tokens == 0) return RK_OK;
   cudaError_t e = launch_prefill_args(a, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? RK_OK : RK_ERR_CUDA;
+}
+
+extern "C" rk_status rk_selftest_bounded_wait(int32_t* device_word, int32_t wait_ms,
+                                              void* stream) {
+  if (!device_word || !aligned(device_word, 4) || wait_ms < 1 || wait_ms > 1000)
+    return RK_ERR_INVALID_ARG;
+  return launch_selftest_wait(device_word, wait_ms, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? RK_OK
+             : RK_ERR_CUDA;
 }
 
 extern "C" rk_status rk_get_device_status(const void* workspace, int32_t* status, void* stream) {

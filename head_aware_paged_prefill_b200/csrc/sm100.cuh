@@ -69,14 +69,14 @@ struct WaitCtx {
 // the CTA is aborting or if the wait ran past kWaitLimitNs (then it raises the
 // abort flag and RK_DEV_TIMEOUT).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtx& w,
-                                          int site) {
+                                          int site, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t n = 1;; ++n) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((n & 63u) == 0) {
       if (*w.abort_flag) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (global_timer_ns() - t0 > limit_ns) {
         *w.abort_flag = 1;
         atomicOr(w.error_word, static_cast<int>(RK_DEV_TIMEOUT));
         atomicCAS(w.timeout_site, 0, site);

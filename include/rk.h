@@ -199,6 +199,15 @@ rk_status rk_segpaged_prefill(const rk_dims* dims, const void* q, const void* k_
  * otherwise, RK_ERR_CUDA if the copy failed. */
 rk_status rk_get_device_status(const void* workspace, int32_t* status, void* stream);
 
+/* Diagnostic for the kernels' failure detection (the pages have no
+ * counterpart): launches one thread that waits, through the same bounded
+ * mbarrier wait the attention kernel uses, on a barrier that nothing
+ * completes.  After wait_ms milliseconds (1..1000) the wait gives up, ORs
+ * RK_DEV_TIMEOUT into *device_word (device int32) and the kernel returns
+ * normally; the CUDA context stays usable.  Errors (host): RK_ERR_INVALID_ARG,
+ * RK_ERR_CUDA. */
+rk_status rk_selftest_bounded_wait(int32_t* device_word, int32_t wait_ms, void* stream);
+
 /* Page tables and row ranges without any device memory from the caller
  * beyond inputs and outputs.  The RedKnot pages have no counterpart of this
  * call; it exists for callers that cannot allocate device memory: code whose

@@ -117,3 +117,37 @@ def test_prefill_deterministic(mode):
     a = PrefillRun(wl.layout, q, k, v, mode=mode)
     b = PrefillRun(wl.layout, q, k, v, mode=mode)
     assert torch.equal(a.o.view(torch.int16), b.o.view(torch.int16))
+
+
+def test_prefill_reports_bad_page_without_faulting():
+    """A page id outside the pool (corrupted after selection) is skipped by the
+    kernel (the tile loads zeros) and reported through the error word."""
+    from head_aware_paged_prefill_b200 import binding
+    from gpu_util import run_select
+    wl = synth.cfg1()
+    lay = wl.layout
+    q, k, v = (t.cuda() for t in wl.materialize("cpu"))
+    for fuse in (True, False):
+        hl, vis, ws = run_select(lay)
+        torch.cuda.synchronize()
+        vis.entries[3, 0] = lay.n_pages + 7
+        vis.entries[30, 0] = -2  # a local-head entry
+        o = torch.zeros_like(q)
+        binding.segpaged_prefill(hl, q, k, v, vis, ws, o, fuse_rope=fuse)
+        torch.cuda.synchronize()
+        assert binding.device_status(ws) & binding.RK_DEV_BAD_PAGE
+        assert torch.isfinite(o.float()).all()
+
+
+def test_bounded_wait_gives_up_and_context_survives():
+    """The kernels' bounded wait on a barrier that nothing completes raises
+    RK_DEV_TIMEOUT and returns; the context is usable afterwards."""
+    from head_aware_paged_prefill_b200 import binding
+    word = torch.zeros(1, dtype=torch.int32, device="cuda")
+    binding.selftest_bounded_wait(word, 20)
+    torch.cuda.synchronize()
+    assert int(word.item()) == binding.RK_DEV_TIMEOUT
+    wl = synth.cfg1()
+    q, k, v = (t.cuda() for t in wl.materialize("cpu"))
+    run = PrefillRun(wl.layout, q, k, v, mode="fused")
+    assert run.status == 0

@@ -1,0 +1,76 @@
+"""The oracle's pins catch plausible mistakes.
+
+Each case plants one mistake in a copy of the C oracle (on the CPU: a flipped
+sign, an off-by-one window, a dropped term, a swapped operand, ...), builds
+it, and checks that at least one pin of tests/test_oracle_pins.py fails on
+it, while the unmodified oracle passes them all."""
+import ctypes
+import os
+import subprocess
+
+import pytest
+
+import oracle
+import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "rk_oracle.c")
+
+MUTANTS = {
+    "rope_sign": ("y[m] = x0 * c - x1 * s;", "y[m] = x0 * c + x1 * s;"),
+    "rope_pair_index": ("double x0 = x[m], x1 = x[m + h];", "double x0 = x[m], x1 = x[h - 1 - m];"),
+    "window_off_by_one": ("return j > i - t->window;", "return j >= i - t->window;"),
+    "causal_excludes_diagonal": ("j >= t->L || j > i) return 0;", "j >= t->L || j >= i) return 0;"),
+    "retrieval_ignores_list": ("return t->uncached[j] || t->in_s[j / t->pr->p];", "return t->uncached[j];"),
+    "delta_sign": ("int delta = sg[1] - sg[3];", "int delta = sg[3] - sg[1];"),
+    "relocated_k_sin_sign": ("kj[m] = x0 * cs[m] - x1 * cs[h + m];", "kj[m] = x0 * cs[m] + x1 * cs[h + m];"),
+    "value_is_key": ("const double* vj = aj->vr + (size_t)j * d;", "const double* vj = aj->kr + (size_t)j * d;"),
+    "no_normalisation": ("for (int c = 0; c < d; ++c) o[c] /= sum;", ";"),
+    "lse_drops_max": ("aj->lse[idx] = mx + log(sum);", "aj->lse[idx] = log(sum);"),
+    "n_valid_always_p": ("int nv = L - k * P < P ? L - k * P : P;", "int nv = P;"),
+    "page_offset": ("int page_in_seg = (k * P - sg[1]) / P;", "int page_in_seg = (k * P - sg[1]) / P + 1;"),
+}
+
+PIN_CALLS = [
+    lambda: [pins.test_rope_matches_complex_rotation(d) for d in (4, 64)],
+    pins.test_rope_quarter_turn_by_hand,
+    pins.test_global_head_is_causal_attention,
+    pins.test_local_head_is_sliding_window,
+    pins.test_retrieval_head_is_union_mask,
+    pins.test_cfg1_page_table_by_hand,
+    pins.test_partial_last_page_by_hand,
+    lambda: [pins.test_visible_pairs_brute_force("cfg1")],
+]
+
+
+def _build(tmp_path, name, old, new):
+    src = open(SRC).read()
+    assert src.count(old) == 1, name
+    path = tmp_path / f"{name}.c"
+    path.write_text(src.replace(old, new))
+    so = tmp_path / f"{name}.so"
+    subprocess.check_call(["gcc", "-O2", "-std=c99", "-D_DEFAULT_SOURCE", "-shared", "-fPIC",
+                           "-pthread", "-o", str(so), str(path), "-lm"])
+    return str(so)
+
+
+def _fails_some_pin(so_path, monkeypatch):
+    monkeypatch.setattr(oracle, "_lib", None)
+    monkeypatch.setattr(oracle, "build", lambda force=False: so_path)
+    for call in PIN_CALLS:
+        try:
+            call()
+        except AssertionError:
+            return True
+    return False
+
+
+def test_unmodified_oracle_passes(tmp_path, monkeypatch):
+    so = _build(tmp_path, "clean", "#include <math.h>", "#include <math.h>")
+    assert not _fails_some_pin(so, monkeypatch)
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(tmp_path, monkeypatch, name):
+    old, new = MUTANTS[name]
+    so = _build(tmp_path, name, old, new)
+    assert _fails_some_pin(so, monkeypatch), f"no pin catches mutant {name}"

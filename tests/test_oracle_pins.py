@@ -370,3 +370,21 @@ def test_empty_row_set_and_empty_request():
     ent, rg = oracle.page_tables(lay)
     assert all(e.shape[0] == 0 for e in ent) and all(r.shape[0] == 0 for r in rg)
     assert oracle.visible_pairs(lay) == 0 == oracle.visible_pairs_closed_form(lay)
+
+
+def test_partial_last_page_by_hand():
+    """13 tokens over 4-token pages: a cached segment of 8 stored at 0..7
+    placed at 0 (delta 0) and a 5-token uncached tail; a global head sees all
+    four pages, the last holding one key; a local head (W=3) computes rows
+    8..12 and sees the pages holding keys 6..12."""
+    segs = [("a", 8, 0, True), ("t", 5, 0, False)]
+    lay = synth._make_layout(n_layers=1, hq=2, hkv=2, d=8, p=4, theta=1e4, requests=[segs],
+                             class_map=[synth.GLOBAL, synth.LOCAL], window=3)
+    ent, rg = oracle.page_tables(lay)
+    np.testing.assert_array_equal(ent[0][:, 1], [0, 4, 8, 12])
+    np.testing.assert_array_equal(ent[0][:, 3], [4, 4, 4, 1])
+    np.testing.assert_array_equal(ent[1][:, 1], [4, 8, 12])
+    np.testing.assert_array_equal(ent[1][:, 3], [4, 4, 1])
+    np.testing.assert_array_equal(rg[0], [[0, 13]])
+    np.testing.assert_array_equal(rg[1], [[8, 13]])
+    assert oracle.visible_pairs(lay) == 13 * 14 // 2 + 5 * 3
