@@ -16,20 +16,21 @@
 //
 //   warp 0      TMA producer: Q tiles (3-D box out of [rows][Hq][D]) and, per
 //               KV tile, one box per page and 64-column block out of the pool.
-//   warp 1      tcgen05 issuer and TMEM owner.  S_t = Q_t K^T (M=128, N=128,
-//               K=D) into TMEM; O_t += P_t V (M=128, N=D, K=128) with P_t read
-//               from TMEM and V from shared memory (MN-major operand), issued
-//               per 64-key half as soon as that half of P is stored.  Order
-//               per KV tile: PV_0, S_0(next), PV_1, S_1(next), so the two Q
-//               tiles' softmax phases alternate.
-//   warps 2-3   RoPE relocation (fuse_rope): rotate the Q tiles by -delta once
-//               per run of tiles sharing a delta, and the K pages of a tile that
-//               mixes deltas by their difference.
+//   warps 1, 3  tcgen05 issuers, one per Q tile (warp 1 also owns TMEM).
+//               S_t = Q_t K^T (M=128, N=128, K=D) into TMEM; O_t += P_t V
+//               (M=128, N=D, K=128) with P_t read from TMEM and V from shared
+//               memory (MN-major operand), issued per 64-key half as soon as
+//               that half of P is stored.
+//   warp 2      RoPE relocation (fuse_rope): rotates the Q tiles by -delta
+//               once per run of tiles sharing a delta, and the K pages of a
+//               tile that mixes deltas by their difference.
 //   warps 4-7   softmax warpgroup of Q tile 0, warps 8-11 of Q tile 1: one
 //               TMEM lane (= one query row) per thread; online softmax in the
 //               log2 domain, O rescaled in TMEM only when the running max
 //               grows by more than 2^8, P written back over S as bf16 in
-//               16-column quarters.
+//               16-column quarters.  The two warpgroups' exponential phases
+//               take turns (a pair of mbarriers), so they never compete for
+//               the MUFU while their other phases overlap.
 // Registers are rebalanced with setmaxnreg: the first warpgroup keeps 80 per
 // thread, the two softmax warpgroups get 208.
 //
@@ -90,12 +91,13 @@ enum : int {
   kBarPLo = 4,     // [2] P columns of keys 0-63 stored
   kBarOFull = 6,   // [2]
   kBarOEmpty = 8,  // [2]
-  kBarDrain = 10,  // MMA completion before TMEM is released
-  kBarPHi = 11,    // [2] P columns of keys 64-127 stored
-  kBarQReady = 13,   // fused: the Q tiles hold the rotation the next S needs
-  kBarQFree = 14,    // fused: every S reading the current Q rotation completed
-  kBarQReload = 15,  // fused: original Q re-fetched for a new rotation
-  kBarKFull = 16,  // [kStages] x 5 groups follow (k_full, k_ready, k_empty, v_full, v_empty)
+  kBarDrain = 10,  // [2] MMA completion before TMEM is released (one per issuer)
+  kBarPHi = 12,    // [2] P columns of keys 64-127 stored
+  kBarQReady = 14,   // fused: the Q tiles hold the rotation the next S needs
+  kBarQFree = 15,    // fused: every S reading the current Q rotation completed
+  kBarQReload = 16,  // fused: original Q re-fetched for a new rotation
+  kBarTurn = 17,   // [2] softmax exponential phases take turns (two-head items)
+  kBarKFull = 19,  // [kStages] x 5 groups follow (k_full, k_ready, k_empty, v_full, v_empty)
 };
 
 // kEmuNum pairs of exponentials in every kEmuDen can go through the FMA-pipe
@@ -140,7 +142,7 @@ __device__ __forceinline__ void rope_table(int delta, int c, const double* inv_f
 
 // Rotates rows [row_lo, row_hi) of a 128-row bf16 tile in shared memory (the
 // K or Q operand layout: 64-column blocks of 128-byte rows, 128-byte swizzle,
-// so 16-byte chunk c of row r sits at chunk c ^ (r & 7)).  Thread rt of 64
+// so 16-byte chunk c of row r sits at chunk c ^ (r & 7)).  Thread rt of 32
 // owns chunk c of rows r0, r0 + RSTEP, ...; the rotate-half partner of chunk c
 // is chunk c + D/16 of the same row (D = 64) or chunk c of the next column
 // block (D = 128).  Packed fp32 math, one bf16 rounding per element.
@@ -149,7 +151,7 @@ __device__ __forceinline__ void rope_rotate_rows(uint8_t* tile, int row_lo, int 
                                                  const uint64_t (&cos2)[4],
                                                  const uint64_t (&sin2)[4]) {
   constexpr int CH = D / 16;
-  constexpr int RSTEP = 64 / CH;
+  constexpr int RSTEP = 32 / CH;
   const int c = rt % CH;
   const int first = row_lo + ((rt / CH) - row_lo % RSTEP + RSTEP) % RSTEP;
 #pragma unroll 2
@@ -210,11 +212,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&bars[kBarQFull], 1);
-    mbar_init(&bars[kBarQEmpty], 1);
+    mbar_init(&bars[kBarQEmpty], 2);
     mbar_init(&bars[kBarDrain], 1);
-    mbar_init(&bars[kBarQReady], 64);
-    mbar_init(&bars[kBarQFree], 1);
+    mbar_init(&bars[kBarDrain + 1], 1);
+    mbar_init(&bars[kBarQReady], 32);
+    mbar_init(&bars[kBarQFree], 2);
     mbar_init(&bars[kBarQReload], 1);
+    mbar_init(&bars[kBarTurn], 128);
+    mbar_init(&bars[kBarTurn + 1], 128);
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bars[kBarSFull + t], 1);
       mbar_init(&bars[kBarPLo + t], 128);
@@ -224,10 +229,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     }
     for (int s = 0; s < S; ++s) {
       mbar_init(&k_full[s], 1);
-      mbar_init(&k_ready[s], 64);
-      mbar_init(&k_empty[s], 1);
+      mbar_init(&k_ready[s], 32);
+      mbar_init(&k_empty[s], 2);
       mbar_init(&v_full[s], 1);
-      mbar_init(&v_empty[s], 1);
+      mbar_init(&v_empty[s], 2);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -321,35 +326,38 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         if (q_uses > 0) mbar_wait_drain(&bars[kBarQFull], (q_uses - 1) & 1);
       }
     }
-  } else if (warp == 1) {
-    // -------------------------------------------------------- MMA issuer
+  } else if (warp == 1 || warp == 3) {
+    // ------------------------------------------------------- MMA issuers
+    // One issuing thread per Q tile (warp 1: tile 0, warp 3: tile 1), so the
+    // two tiles' S -> softmax -> PV chains never wait on each other.  K / V
+    // stages, the Q buffers and the Q-rotation handoff are released by both
+    // issuers (barrier counts of 2); an issuer whose tile is absent from an
+    // item (a single q head) still steps through the item's barriers.
     if (lane == 0) {
+      const int t = warp == 1 ? 0 : 1;
       constexpr uint32_t idesc_s = idesc_bf16_f32(kRowsPerTile, kKeysPerTile, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(kRowsPerTile, D, true);
-      const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
+      const uint32_t sQa = smem_u32(sQ) + t * C::kQTileBytes, sKa = smem_u32(sK), sVa = smem_u32(sV);
+      const uint32_t tS = tmem + C::col_s(t), tO = tmem + C::col_o(t);
       uint64_t* k_avail = fuse ? k_ready : k_full;
-      uint32_t kv_iter = 0, q_uses = 0, qrd_uses = 0;
-      uint32_t p_phase[2] = {0, 0}, o_uses[2] = {0, 0};
+      uint32_t kv_iter = 0, q_uses = 0, qrd_uses = 0, p_phase = 0, o_uses = 0;
       bool ok = true;
-      auto issue_s = [&](int t, int st) {
-        const uint32_t d = tmem + C::col_s(t);
+      auto issue_s = [&](int st) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::kBlockBytes + (kk & 3) * 32;
-          const uint64_t a = desc_sw128(sQa + t * C::kQTileBytes + off, 16, 1024);
+          const uint64_t a = desc_sw128(sQa + off, 16, 1024);
           const uint64_t bd = desc_sw128(sKa + st * C::kKVTileBytes + off, 16, 1024);
-          mma_bf16_ss(d, a, bd, idesc_s, kk > 0 ? 1u : 0u);
+          mma_bf16_ss(tS, a, bd, idesc_s, kk > 0 ? 1u : 0u);
         }
       };
       // O_t (+)= P_t V over keys [64 half, 64 half + 64)
-      auto issue_pv = [&](int t, int st, int half, bool acc) {
-        const uint32_t d = tmem + C::col_o(t);
-        const uint32_t a = tmem + C::col_s(t);
+      auto issue_pv = [&](int st, int half, bool acc) {
 #pragma unroll
         for (int kk = 4 * half; kk < 4 * half + 4; ++kk) {
           const uint64_t bd =
               desc_sw128(sVa + st * C::kKVTileBytes + kk * 16 * 128, C::kBlockBytes, 1024);
-          mma_bf16_ts(d, a + kk * 8, bd, idesc_o, (acc || kk > 0) ? 1u : 0u);
+          mma_bf16_ts(tO, tS + kk * 8, bd, idesc_o, (acc || kk > 0) ? 1u : 0u);
         }
       };
       for (int r = 0; ok; ++r) {
@@ -358,6 +366,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         const Item w = prm.items[it];
         const int n_tiles = (w.e_end - w.e_begin + C::EPT - 1) / C::EPT;
         if (n_tiles == 0) continue;
+        const bool active = t < w.nh;
         if (fuse) {
           if (!(ok = mbar_wait(&bars[kBarQReady], qrd_uses & 1, wc, 10))) break;
           ++qrd_uses;
@@ -365,13 +374,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           break;
         }
         ++q_uses;
-        int dcur = prm.entries[w.e_begin].delta;
+        int dcur = fuse ? __ldg(&prm.entries[w.e_begin].delta) : 0;
         {
           const int st = kv_iter % S;
           if (!(ok = mbar_wait(&k_avail[st], (kv_iter / S) & 1, wc, 11))) break;
-          tc_fence_after();
-          for (int t = 0; t < w.nh; ++t) {
-            issue_s(t, st);
+          if (active) {
+            tc_fence_after();
+            issue_s(st);
             tc_commit(&bars[kBarSFull + t]);
           }
           tc_commit(&k_empty[st]);
@@ -385,55 +394,51 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           const int dnext =
               (fuse && more) ? __ldg(&prm.entries[w.e_begin + (j + 1) * C::EPT].delta) : dcur;
           const bool qswitch = fuse && dnext != dcur;
-          for (int t = 0; t < w.nh && ok; ++t) {
-            if (!(ok = mbar_wait(&bars[kBarPLo + t], p_phase[t], wc, 12))) break;
-            if (j == 0 && o_uses[t] > 0 &&
-                !(ok = mbar_wait(&bars[kBarOEmpty + t], (o_uses[t] - 1) & 1, wc, 13)))
+          if (active) {
+            if (!(ok = mbar_wait(&bars[kBarPLo + t], p_phase, wc, 12))) break;
+            if (j == 0 && o_uses > 0 &&
+                !(ok = mbar_wait(&bars[kBarOEmpty + t], (o_uses - 1) & 1, wc, 13)))
               break;
-            if (t == 0 && !(ok = mbar_wait(&v_full[st], (kj / S) & 1, wc, 14))) break;
+            if (!(ok = mbar_wait(&v_full[st], (kj / S) & 1, wc, 14))) break;
             tc_fence_after();
-            issue_pv(t, st, 0, j > 0);
-            if (!(ok = mbar_wait(&bars[kBarPHi + t], p_phase[t], wc, 16))) break;
-            p_phase[t] ^= 1;
+            issue_pv(st, 0, j > 0);
+            if (!(ok = mbar_wait(&bars[kBarPHi + t], p_phase, wc, 16))) break;
+            p_phase ^= 1;
             tc_fence_after();
-            issue_pv(t, st, 1, true);
-            if (qswitch) {
-              if (t == 0) tc_commit(&bars[kBarQFree]);
-            } else if (more) {
-              if (t == 0 && !(ok = mbar_wait(&k_avail[stn], ((kj + 1) / S) & 1, wc, 15))) break;
-              tc_fence_after();
-              issue_s(t, stn);
-              tc_commit(&bars[kBarSFull + t]);
-            }
-          }
-          if (!ok) break;
-          if (qswitch) {
-            if (!(ok = mbar_wait(&bars[kBarQReady], qrd_uses & 1, wc, 17))) break;
-            ++qrd_uses;
-            if (!(ok = mbar_wait(&k_avail[stn], ((kj + 1) / S) & 1, wc, 18))) break;
-            tc_fence_after();
-            for (int t = 0; t < w.nh; ++t) {
-              issue_s(t, stn);
-              tc_commit(&bars[kBarSFull + t]);
-            }
-            dcur = dnext;
+            issue_pv(st, 1, true);
+          } else if (!(ok = mbar_wait(&v_full[st], (kj / S) & 1, wc, 14))) {
+            break;
           }
           tc_commit(&v_empty[st]);
-          if (more) tc_commit(&k_empty[stn]);
+          if (qswitch) {
+            tc_commit(&bars[kBarQFree]);
+            if (!(ok = mbar_wait(&bars[kBarQReady], qrd_uses & 1, wc, 17))) break;
+            ++qrd_uses;
+            dcur = dnext;
+          }
+          if (more) {
+            if (!(ok = mbar_wait(&k_avail[stn], ((kj + 1) / S) & 1, wc, 15))) break;
+            if (active) {
+              tc_fence_after();
+              issue_s(stn);
+              tc_commit(&bars[kBarSFull + t]);
+            }
+            tc_commit(&k_empty[stn]);
+          }
         }
         if (!ok) break;
-        for (int t = 0; t < w.nh; ++t) {
+        if (active) {
           tc_commit(&bars[kBarOFull + t]);
-          ++o_uses[t];
+          ++o_uses;
         }
         tc_commit(&bars[kBarQEmpty]);
         kv_iter += n_tiles;
       }
       // make sure no MMA still writes TMEM when it is released
-      tc_commit(&bars[kBarDrain]);
-      mbar_wait_drain(&bars[kBarDrain], 0);
+      tc_commit(&bars[kBarDrain + t]);
+      mbar_wait_drain(&bars[kBarDrain + t], 0);
     }
-  } else if (warp < 4) {
+  } else if (warp == 2) {
     // ------------------------------------------- RoPE relocation (fused)
     // q . R(d) k = (R(-d) q) . k: the Q tiles are rotated by -d once per run
     // of tiles whose keys share the relocation d (a cached segment), so the
@@ -443,7 +448,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     // rotation the original Q is fetched again, so every Q element is rounded
     // to bf16 once.
     if (fuse) {
-      const int rt = threadIdx.x - 64;
+      const int rt = lane;
       const int c = rt % (D / 16);
       uint32_t k_seen = 0, q_uses = 0, qf_uses = 0, qr_uses = 0;
       int tab_delta = 0;
@@ -531,7 +536,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const uint32_t tO = tmem + lane_base + C::col_o(t);
     const float sl2 = prm.scale_log2;
     const int T = prm.total_tokens;
-    uint32_t s_phase = 0, o_uses = 0;
+    uint32_t s_phase = 0, o_uses = 0, turn_phase = 0;
     bool ok = true;
     for (int r = 0; ok; ++r) {
       const int it = item_of_round(r, b, G);
@@ -555,6 +560,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       }
       const int window = w.window;
       float m_ref = -INFINITY, l = 0.f;
+      // tile 0's warpgroup goes first in every two-head item
+      if (w.nh == 2 && t == 1) mbar_arrive(&bars[kBarTurn]);
       for (int j = 0; j < n_tiles && ok; ++j) {
         // pages of this tile (loaded before the wait, so their latency hides)
         int lp[C::EPT], nv[C::EPT];
@@ -616,6 +623,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
         if (resc) m_ref = m_new;
         const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
+        // two-head items: the two warpgroups' exponential phases alternate
+        // (tile 0's first), so they never compete for the MUFU and issue slots
+        if (w.nh == 2 && !(ok = mbar_wait(&bars[kBarTurn + t], turn_phase, wc, 22))) break;
         const uint64_t scale2 = f2_pack(sl2, sl2);
         const uint64_t neg_m2 = f2_pack(-m_use, -m_use);
         uint64_t acc2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
@@ -650,6 +660,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           tmem_st_wait();
           tc_fence_before();
           mbar_arrive(&bars[(half ? kBarPHi : kBarPLo) + t]);
+          // the other warpgroup's turn once this one's exponentials are done
+          // (tile 1 hands back after every tile but the item's last)
+          if (half == 1 && w.nh == 2) {
+            turn_phase ^= 1;
+            if (t == 0 || j + 1 < n_tiles) mbar_arrive(&bars[kBarTurn + (1 - t)]);
+          }
         }
         float a0, a1, b0, b1;
         f2_unpack(acc2[0], a0, a1);
