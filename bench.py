@@ -3,11 +3,14 @@
 
 One step = one pass of the whole hot path over the Mistral-7B-shaped 32K
 layer (Hq 32, Hkv 8, D 128, P 64; 7 cached 4096-token segments + 4096 tail;
-kv_head 0 global, 1-7 local with a 4096 window): rk_select_visible ->
-rk_segpaged_prefill with the RoPE relocation of cached keys fused into the
-K loads, inputs resident in HBM, L2 flushed (256 MiB write) between timed
-steps.  The standalone relocation kernel (rk_relocate_rope over every cached
-page of the layer) is timed after it and reported against the HBM roofline.
+kv_head 0 global, 1-7 local with a 4096 window), inputs resident in HBM, L2
+flushed (256 MiB write) between timed steps.  Default mode "relocate":
+rk_relocate_rope (every visible page of a cached segment with a non-zero
+delta, rotated from the K store into the working K pool) ->
+rk_select_visible -> rk_segpaged_prefill.  Mode "fused":
+rk_select_visible -> rk_segpaged_prefill with the relocation done inside the
+attention kernel.  The line reports the other mode too, and the standalone
+relocation kernel against the HBM roofline.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -50,9 +53,15 @@ def _peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-def _kernel_hash() -> str:
+KERNEL_SOURCES = {"segpaged_prefill_kernel": ("rk_prefill.cu", "sm100.cuh", "rk_internal.h"),
+                  "relocate_kernel": ("rk_relocate.cu", "rk_internal.h")}
+
+
+def _kernel_hash(kernel: str = "segpaged_prefill_kernel") -> str:
+    """Hash of the sources a kernel is compiled from (ties a recorded ncu
+    figure to the code it was taken on)."""
     h = hashlib.sha256()
-    for f in ("rk_prefill.cu", "sm100.cuh", "rk_internal.h"):
+    for f in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, "head_aware_paged_prefill_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -67,7 +76,7 @@ def _recorded_traffic(kernel: str, workload: str):
     with open(p) as f:
         d = json.load(f)
     e = d.get(kernel, {})
-    if e.get("source_hash") != _kernel_hash() or e.get("workload") != workload:
+    if e.get("source_hash") != _kernel_hash(kernel) or e.get("workload") != workload:
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -183,28 +192,34 @@ def _time_oracle(lay, q, k, v, rows):
 
 
 def _bench_relocate(torch, lay, k_pool, dev, flush, stream, reps, peaks, peak_kind):
-    """rk_relocate_rope over every cached page with delta != 0 (one job per
-    page and (layer, kv_head)), into separate destination pages."""
+    """rk_relocate_rope alone over every page of every cached segment with
+    delta != 0 (all (layer, kv_head) pairs, visible or not), from the store
+    into a working pool at the same page ids: a bandwidth measurement of the
+    relocation kernel on a job list larger than the step's own."""
     from head_aware_paged_prefill_b200 import binding, metrics
-    from head_aware_paged_prefill_b200.plan import relocation_plan
-    jobs, _ = relocation_plan(lay)
-    if jobs.shape[0] == 0:
+    n_lh = lay.n_layers * lay.hkv
+    jobs = []
+    for s in range(lay.segments.shape[0]):
+        _, start, ln, stored, cached = (int(x) for x in lay.segments[s])
+        if cached and start != stored:
+            for lh in range(n_lh):
+                b0 = int(lay.page_base[s, lh])
+                jobs += [(b0 + k, b0 + k, start - stored) for k in range(-(-ln // lay.p))]
+    if not jobs:
         return None
+    jobs = np.asarray(jobs, dtype=np.int32)
     n = jobs.shape[0]
-    # sources stay in the pool; destinations are n fresh pages appended to it
-    pool = torch.cat([k_pool, torch.empty((n, lay.p, lay.d), dtype=torch.bfloat16, device=dev)])
-    jobs = jobs.copy()
-    jobs[:, 1] = k_pool.shape[0] + np.arange(n, dtype=np.int32)
+    work = torch.empty_like(k_pool)
     jt = torch.from_numpy(jobs).to(dev)
     for _ in range(3):
-        binding.relocate_rope(pool, pool, jt, lay.theta)
+        binding.relocate_rope(k_pool, work, jt, lay.theta)
     torch.cuda.synchronize()
     ms = []
     for _ in range(reps):
         flush.zero_()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        binding.relocate_rope(pool, pool, jt, lay.theta)
+        binding.relocate_rope(k_pool, work, jt, lay.theta)
         b.record(stream)
         ms.append((a, b))
     torch.cuda.synchronize()
@@ -272,7 +287,7 @@ def main():
     ap.add_argument("--config", default="cfg2")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--mode", default="fused", choices=["fused", "relocate"])
+    ap.add_argument("--mode", default="relocate", choices=["fused", "relocate"])
     ap.add_argument("--reloc-reps", type=int, default=50)
     ap.add_argument("--ref-step-s", type=float, default=0.25)
     ap.add_argument("--no-cpu-baseline", action="store_true")

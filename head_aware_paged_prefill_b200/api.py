@@ -6,9 +6,13 @@ C-ABI calls on the current CUDA stream.  Two modes:
 
   "fused"     rk_select_visible, then rk_segpaged_prefill(fuse_rope=1): cached
               keys are rotated by their page's delta as they are loaded.
-  "relocate"  rk_relocate_rope writes relocated copies of every cached page
-              with a non-zero delta (K rotated, V copied), then
-              rk_select_visible and rk_segpaged_prefill(fuse_rope=0) read them.
+  "relocate"  rk_relocate_rope rotates every visible page of a cached
+              segment with a non-zero delta from the K store into the working
+              K pool (same page id; pages reused at two offsets get an
+              appended copy, V copied alongside), then rk_select_visible and
+              rk_segpaged_prefill(fuse_rope=0) read the working pools.  The
+              jobs come from the page tables, built once on the device when
+              the object is created.
 
 Inputs may live on the host (pinned tensors are copied asynchronously) or on
 the device; ``run(..., out="host")`` returns o on the host.
@@ -21,60 +25,82 @@ import numpy as np
 import torch
 
 from . import binding
-from .plan import relocation_plan
+from .plan import RelocationPlan, relocation_plan
 
 
 class SegPagedPrefill:
-    def __init__(self, layout, device="cuda", with_lse: bool = False, mode: str = "fused"):
+    def __init__(self, layout, device="cuda", with_lse: bool = False, mode: str = "relocate"):
         if mode not in ("fused", "relocate"):
             raise ValueError(mode)
         self.layout = layout
         self.mode = mode
         self.device = torch.device(device)
+        lay = layout
         if mode == "relocate":
-            self.jobs_np, self.rel_layout = relocation_plan(layout)
+            self.plan = self._plan(layout)
         else:
-            self.jobs_np, self.rel_layout = np.zeros((0, 3), np.int32), layout
+            empty = np.zeros((0, 3), np.int32)
+            self.plan = RelocationPlan(empty, empty, layout, 0)
+        self.rel_layout = self.plan.layout
         self.hl = binding.HostLayout(self.rel_layout)
         self.sizes = self.hl.sizes()
         self.vis = binding.Visible(self.sizes, self.device)
         self.ws = binding.workspace(self.sizes, self.device)
-        lay = layout
-        self.n_extra = int(self.rel_layout.n_pages - lay.n_pages)
-        self.jobs = torch.from_numpy(self.jobs_np).to(self.device)
-        self.k_work = torch.empty((self.rel_layout.n_pages, lay.p, lay.d), dtype=torch.bfloat16,
-                                  device=self.device)
-        self.v_work = torch.empty_like(self.k_work)
+        self.n_extra = self.plan.n_extra
+        shape = (lay.n_pages + self.n_extra, lay.p, lay.d)
+        self.k_work = torch.empty(shape, dtype=torch.bfloat16, device=self.device)
+        self.v_work = torch.empty(shape, dtype=torch.bfloat16, device=self.device)
+        # the K store (pages as written) is the relocation's source
+        self.k_store = (torch.empty((lay.n_pages, lay.p, lay.d), dtype=torch.bfloat16,
+                                    device=self.device) if mode == "relocate" else None)
         self.q_dev = torch.empty((lay.n_layers, lay.total_tokens, lay.hq, lay.d),
                                  dtype=torch.bfloat16, device=self.device)
         self.o = torch.empty_like(self.q_dev)
         self.lse = (torch.empty((lay.n_layers, lay.hq, lay.total_tokens), dtype=torch.float32,
                                 device=self.device) if with_lse else None)
         self.dev_err = torch.zeros(1, dtype=torch.int32, device=self.device)
-        # V is not rotated: its relocated pages are delta-0 copies (a page gather)
-        jobs_v = self.jobs_np.copy()
-        jobs_v[:, 2] = 0
-        self.jobs_v = torch.from_numpy(jobs_v).to(self.device)
+        self.jobs_k = torch.from_numpy(self.plan.jobs_k).to(self.device)
+        self.jobs_v = torch.from_numpy(self.plan.jobs_v).to(self.device)
+
+    def _plan(self, layout) -> RelocationPlan:
+        """Page tables of the original layout (built by the library on the
+        device), read back once, turned into relocation jobs."""
+        hl = binding.HostLayout(layout)
+        sizes = hl.sizes()
+        vis = binding.Visible(sizes, self.device)
+        ws = binding.workspace(sizes, self.device)
+        binding.select_visible(hl, vis, ws)
+        torch.cuda.current_stream(self.device).synchronize()
+        st = binding.device_status(ws)
+        if st:
+            raise binding.RkError(binding.RK_ERR_DEVICE, f"rk_select_visible (device {st:#x})")
+        entries, _ = vis.tables()
+        return relocation_plan(layout, entries)
 
     # Number of library kernel launches one run() makes.
     @property
     def launches_per_run(self) -> int:
-        return 3 + (2 if self.jobs_np.shape[0] else 0)
+        return 3 + int(self.plan.jobs_k.shape[0] > 0) + int(self.plan.jobs_v.shape[0] > 0)
 
     def load(self, q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor):
         """Copies inputs (host or device) into the device working buffers."""
         n = self.layout.n_pages
         self.q_dev.copy_(q, non_blocking=True)
-        self.k_work[:n].copy_(k_pool, non_blocking=True)
+        if self.k_store is not None:
+            self.k_store.copy_(k_pool, non_blocking=True)
+            self.k_work[:n].copy_(self.k_store)
+        else:
+            self.k_work[:n].copy_(k_pool, non_blocking=True)
         self.v_work[:n].copy_(v_pool, non_blocking=True)
 
     def compute(self, stream=None, k3_events=None):
         """Runs relocation, selection and attention on the loaded inputs.
         k3_events: optional (start, end) CUDA events recorded around the
         attention kernel on the launching stream."""
-        if self.jobs_np.shape[0]:
-            binding.relocate_rope(self.k_work, self.k_work, self.jobs, self.layout.theta,
+        if self.plan.jobs_k.shape[0]:
+            binding.relocate_rope(self.k_store, self.k_work, self.jobs_k, self.layout.theta,
                                   self.dev_err, stream)
+        if self.plan.jobs_v.shape[0]:
             binding.relocate_rope(self.v_work, self.v_work, self.jobs_v, self.layout.theta,
                                   self.dev_err, stream)
         binding.select_visible(self.hl, self.vis, self.ws, stream)

@@ -73,7 +73,8 @@ def lib() -> ctypes.CDLL:
         vp, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
         L.rk_query_sizes.argtypes = [vp, vp, vp]
         L.rk_select_visible.argtypes = [vp, vp, vp, vp, ctypes.c_size_t, vp]
-        L.rk_relocate_rope.argtypes = [vp, vp, vp, i32, i64, i32, i32, ctypes.c_double, vp, vp]
+        L.rk_relocate_rope.argtypes = [vp, i64, vp, i64, vp, i32, i32, i32, ctypes.c_double, vp,
+                                       vp]
         L.rk_segpaged_prefill.argtypes = [vp, vp, vp, vp, vp, i32, ctypes.c_double, ctypes.c_float,
                                           vp, vp, vp, ctypes.c_size_t, vp]
         L.rk_get_device_status.argtypes = [vp, vp, vp]
@@ -176,11 +177,12 @@ def select_visible_noalloc(hl: HostLayout, vis: Visible,
 
 def relocate_rope(k_src: torch.Tensor, k_dst: torch.Tensor, jobs: torch.Tensor, theta: float,
                   device_error: Optional[torch.Tensor] = None, stream=None):
-    n_pages, p, d = k_src.shape
-    assert k_dst.shape == k_src.shape and k_src.dtype == torch.bfloat16
+    n_src, p, d = k_src.shape
+    assert k_dst.shape[1:] == k_src.shape[1:] and k_src.dtype == k_dst.dtype == torch.bfloat16
     assert jobs.dtype == torch.int32 and jobs.is_contiguous()
-    _check(lib().rk_relocate_rope(_ptr(k_src), _ptr(k_dst), _ptr(jobs), jobs.shape[0], n_pages,
-                                  p, d, float(theta), _ptr(device_error), _stream(stream)),
+    _check(lib().rk_relocate_rope(_ptr(k_src), n_src, _ptr(k_dst), k_dst.shape[0], _ptr(jobs),
+                                  jobs.shape[0], p, d, float(theta), _ptr(device_error),
+                                  _stream(stream)),
            "rk_relocate_rope")
 
 

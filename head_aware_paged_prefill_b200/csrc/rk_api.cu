@@ -15,8 +15,8 @@ namespace rk {
 cudaError_t launch_select(LayoutView* lv_dev, int n_tables, const rk_visible& vis, WsHeader* hdr,
                           Item* items_tmp, Item* items, cudaStream_t stream);
 cudaError_t launch_relocate(const void* k_src, void* k_dst, const int32_t* jobs, int n_jobs,
-                            int64_t n_pages, int P, int D, double theta, int* device_error,
-                            cudaStream_t stream);
+                            int64_t n_src_pages, int64_t n_dst_pages, int P, int D, double theta,
+                            int* device_error, cudaStream_t stream);
 
 cudaError_t launch_prefill_args(const PrefillLaunchArgs& a, cudaStream_t stream);
 cudaError_t launch_selftest_wait(int* word, int wait_ms, cudaStream_t stream);
@@ -274,19 +274,21 @@ extern "C" rk_status rk_select_visible(const rk_dims* dims, const rk_layout* lay
   return e == cudaSuccess ? RK_OK : RK_ERR_CUDA;
 }
 
-extern "C" rk_status rk_relocate_rope(const void* k_src, void* k_dst, const int32_t* jobs,
-                                      int32_t n_jobs, int64_t n_pages, int32_t page_size,
-                                      int32_t head_dim, double rope_theta, int32_t* device_error,
-                                      void* stream) {
-  if (n_jobs < 0 || n_pages < 1 || page_size < 1 || (head_dim != 64 && head_dim != 128))
+extern "C" rk_status rk_relocate_rope(const void* k_src, int64_t n_src_pages, void* k_dst,
+                                      int64_t n_dst_pages, const int32_t* jobs, int32_t n_jobs,
+                                      int32_t page_size, int32_t head_dim, double rope_theta,
+                                      int32_t* device_error, void* stream) {
+  if (n_jobs < 0 || n_src_pages < 1 || n_dst_pages < 1 || page_size < 1 ||
+      (head_dim != 64 && head_dim != 128))
     return RK_ERR_INVALID_ARG;
   if (!(rope_theta > 0.0) || !std::isfinite(rope_theta)) return RK_ERR_INVALID_ARG;
   if (n_jobs > 0 && (!k_src || !k_dst || !jobs)) return RK_ERR_INVALID_ARG;
   if (!aligned(k_src, 16) || !aligned(k_dst, 16) || !aligned(jobs, 4) ||
       !aligned(device_error, 4))
     return RK_ERR_INVALID_ARG;
-  cudaError_t e = launch_relocate(k_src, k_dst, jobs, n_jobs, n_pages, page_size, head_dim,
-                                  rope_theta, device_error, static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_relocate(k_src, k_dst, jobs, n_jobs, n_src_pages, n_dst_pages,
+                                  page_size, head_dim, rope_theta, device_error,
+                                  static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? RK_OK : RK_ERR_CUDA;
 }
 

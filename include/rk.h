@@ -165,16 +165,19 @@ rk_status rk_select_visible(const rk_dims* dims, const rk_layout* layout, const 
  * jobs[3n..3n+2] = (src_page, dst_page, delta):
  *   k_dst[dst_page][row][:] = bf16( R(delta) k_src[src_page][row][:] )  for row < P,
  * R the rotate-half RoPE rotation (pairs (m, m + D/2), frequency
- * rope_theta^(-2m/D)), computed in fp32 from angles reduced in fp64; delta = 0
- * copies the page bit-exactly.  k_src / k_dst: device bf16 [n_pages][P][D]
- * (may be the same pool); jobs: device int32 [n_jobs][3].  A job may read and
- * write the same page; otherwise no page may be written by one job and read or
- * written by another.  Jobs with a page id outside [0, n_pages) are skipped
- * and set RK_DEV_BAD_PAGE in *device_error (device int32, may be NULL).
- * Errors (host): RK_ERR_INVALID_ARG, RK_ERR_CUDA. */
-rk_status rk_relocate_rope(const void* k_src, void* k_dst, const int32_t* jobs, int32_t n_jobs,
-                           int64_t n_pages, int32_t page_size, int32_t head_dim,
-                           double rope_theta, int32_t* device_error, void* stream);
+ * rope_theta^(-2m/D)), computed in fp32 from angles formed in fp64; delta = 0
+ * copies the page bit-exactly.  k_src: device bf16 [n_src_pages][P][D];
+ * k_dst: device bf16 [n_dst_pages][P][D] (may be the same pool; a typical use
+ * writes R(delta) of each cached page into a working pool at the same page id,
+ * leaving the offline store untouched).  jobs: device int32 [n_jobs][3].  A job
+ * may read and write the same page; otherwise no page may be written by one
+ * job and read or written by another.  Jobs with a page id outside its pool
+ * are skipped and set RK_DEV_BAD_PAGE in *device_error (device int32, may be
+ * NULL).  Errors (host): RK_ERR_INVALID_ARG, RK_ERR_CUDA. */
+rk_status rk_relocate_rope(const void* k_src, int64_t n_src_pages, void* k_dst,
+                           int64_t n_dst_pages, const int32_t* jobs, int32_t n_jobs,
+                           int32_t page_size, int32_t head_dim, double rope_theta,
+                           int32_t* device_error, void* stream);
 
 /* EXECUTE's attention.  For every table's rows i and each q head h of its kv
  * head:  o[layer][tok(i)][h][:] = sum_j softmax_j(softmax_scale <q_i, K'_j>) v_j

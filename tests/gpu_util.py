@@ -31,6 +31,24 @@ def assert_close(got: np.ndarray, want: np.ndarray, what: str = ""):
     return mx, rel
 
 
+def assert_bf16_rounded(got: np.ndarray, want: np.ndarray, what: str = ""):
+    """A bf16 tensor computed in fp32 against its fp64 value: every element
+    within one bf16 ulp of the exact value (round-to-nearest gives half an
+    ulp; the fp32 evaluation may push a value across a rounding midpoint),
+    ulp taken at the bottom of the value's binade, 2^-7 |want|, plus an
+    absolute floor of 1e-5 for values that cancel to near zero."""
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    assert np.isfinite(got).all(), f"{what}: non-finite GPU values"
+    err = np.abs(got - want)
+    bound = np.abs(want) * 2.0 ** -7 + 1e-5
+    bad = err > bound
+    assert not bad.any(), (f"{what}: {int(bad.sum())} elements beyond one bf16 ulp, worst "
+                           f"err {float(err[bad].max()):.3e} at |want| "
+                           f"{float(np.abs(want[bad][np.argmax(err[bad])])):.3e}")
+    return float(err.max()) if err.size else 0.0
+
+
 def run_select(lay, device="cuda"):
     hl = binding.HostLayout(lay)
     s = hl.sizes()
@@ -43,32 +61,38 @@ def run_select(lay, device="cuda"):
 class PrefillRun:
     """One pass of the CUDA path through the C ABI.
 
-    mode "relocate": rk_relocate_rope over the relocation plan, then
-    rk_select_visible and rk_segpaged_prefill(fuse_rope=0) on the relocated
-    layout.  mode "fused": rk_select_visible and
+    mode "relocate": rk_select_visible on the original layout gives the
+    page tables the relocation plan is built from; rk_relocate_rope rotates
+    the visible cached K pages from the input pool (the store) into a working
+    copy, then rk_select_visible and rk_segpaged_prefill(fuse_rope=0) run on
+    the relocated layout.  mode "fused": rk_select_visible and
     rk_segpaged_prefill(fuse_rope=1) on the original layout.
     ``o`` starts filled with the sentinel so untouched rows can be checked."""
 
     def __init__(self, lay, q, k_pool, v_pool, with_lse=True, mode="relocate"):
         dev = q.device
-        if mode == "fused":
-            jobs, rel = np.zeros((0, 3), np.int32), lay
-        else:
-            jobs, rel = relocation_plan(lay)
-        self.lay, self.rel, self.jobs = lay, rel, jobs
-        extra = rel.n_pages - lay.n_pages
-        self.k_rel = torch.cat([k_pool, torch.zeros((extra,) + tuple(k_pool.shape[1:]),
-                                                    dtype=k_pool.dtype, device=dev)])
-        self.v_rel = torch.cat([v_pool, torch.zeros((extra,) + tuple(v_pool.shape[1:]),
-                                                    dtype=v_pool.dtype, device=dev)])
-        # V pages of relocated instances are delta-0 copies of their sources
         self.dev_err = torch.zeros(1, dtype=torch.int32, device=dev)
-        if jobs.shape[0]:
-            jt = torch.from_numpy(jobs).to(dev)
-            jv = jt.clone()
-            jv[:, 2] = 0
-            binding.relocate_rope(self.k_rel, self.k_rel, jt, lay.theta, self.dev_err)
-            binding.relocate_rope(self.v_rel, self.v_rel, jv, lay.theta, self.dev_err)
+        if mode == "fused":
+            rel, self.plan = lay, None
+            self.k_rel, self.v_rel = k_pool, v_pool
+        else:
+            # page tables of the original layout -> relocation jobs
+            _, vis0, _ = run_select(lay, dev)
+            torch.cuda.synchronize()
+            self.plan = relocation_plan(lay, vis0.tables()[0])
+            rel = self.plan.layout
+            extra = self.plan.n_extra
+            pad = torch.zeros((extra,) + tuple(k_pool.shape[1:]), dtype=k_pool.dtype, device=dev)
+            self.k_rel = torch.cat([k_pool, pad])
+            self.v_rel = torch.cat([v_pool, pad])
+            if self.plan.jobs_k.shape[0]:
+                binding.relocate_rope(k_pool, self.k_rel, torch.from_numpy(self.plan.jobs_k).to(dev),
+                                      lay.theta, self.dev_err)
+            if self.plan.jobs_v.shape[0]:
+                binding.relocate_rope(self.v_rel, self.v_rel,
+                                      torch.from_numpy(self.plan.jobs_v).to(dev), lay.theta,
+                                      self.dev_err)
+        self.lay, self.rel = lay, rel
         self.hl, self.vis, self.ws = run_select(rel, dev)
         self.o = torch.full(q.shape, SENTINEL, dtype=torch.int16, device=dev).view(torch.bfloat16)
         self.lse = (torch.full((lay.n_layers, lay.hq, lay.total_tokens), float("nan"),

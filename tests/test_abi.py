@@ -9,7 +9,6 @@ import pytest
 
 from head_aware_paged_prefill_b200 import binding, synth
 from head_aware_paged_prefill_b200.csrc import build as build_mod
-from head_aware_paged_prefill_b200.plan import relocation_plan
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -126,12 +125,18 @@ def test_select_rejects_on_host_without_gpu(lib):
 def test_relocate_and_prefill_reject_on_host(lib):
     E = binding.RK_ERR_INVALID_ARG
     fake = ctypes.c_void_p(1 << 20)
-    assert lib.rk_relocate_rope(fake, fake, fake, 1, 8, 64, 96, 1e4, None, None) == E
-    assert lib.rk_relocate_rope(fake, fake, fake, -1, 8, 64, 128, 1e4, None, None) == E
-    assert lib.rk_relocate_rope(fake, fake, fake, 1, 8, 64, 128, -1.0, None, None) == E
-    assert lib.rk_relocate_rope(None, fake, fake, 1, 8, 64, 128, 1e4, None, None) == E
-    assert lib.rk_relocate_rope(ctypes.c_void_p((1 << 20) + 2), fake, fake, 1, 8, 64, 128, 1e4,
-                                None, None) == E
+    # (k_src, n_src_pages, k_dst, n_dst_pages, jobs, n_jobs, P, D, theta, error, stream)
+    assert lib.rk_relocate_rope(fake, 8, fake, 8, fake, 1, 64, 96, 1e4, None, None) == E
+    assert lib.rk_relocate_rope(fake, 8, fake, 8, fake, -1, 64, 128, 1e4, None, None) == E
+    assert lib.rk_relocate_rope(fake, 8, fake, 8, fake, 1, 64, 128, -1.0, None, None) == E
+    assert lib.rk_relocate_rope(None, 8, fake, 8, fake, 1, 64, 128, 1e4, None, None) == E
+    assert lib.rk_relocate_rope(fake, 0, fake, 8, fake, 1, 64, 128, 1e4, None, None) == E
+    assert lib.rk_relocate_rope(fake, 8, fake, 0, fake, 1, 64, 128, 1e4, None, None) == E
+    assert lib.rk_relocate_rope(fake, 8, fake, 8, fake, 1, 0, 128, 1e4, None, None) == E
+    assert lib.rk_relocate_rope(ctypes.c_void_p((1 << 20) + 2), 8, fake, 8, fake, 1, 64, 128,
+                                1e4, None, None) == E
+    # no jobs: nothing to do, no pointer needed
+    assert lib.rk_relocate_rope(None, 8, None, 8, None, 0, 64, 128, 1e4, None, None) == 0
     lay = synth.cfg1().layout
     hl = _hl(lay)
     vis = binding.RkVisible(1 << 20, 1 << 20, 1 << 20, 1 << 20, 1 << 20, 1 << 20, 1, 1)
@@ -151,13 +156,3 @@ def test_relocate_and_prefill_reject_on_host(lib):
     assert lib.rk_segpaged_prefill(*small_ws) == binding.RK_ERR_CAPACITY
     assert lib.rk_get_device_status(None, None, None) == E
 
-
-def test_relocation_plan_covers_every_nonzero_delta():
-    lay = synth.cfg3().layout
-    jobs, rel = relocation_plan(lay)
-    n_lh = lay.n_layers * lay.hkv
-    nz = [s for s in lay.segments if s[4] and s[1] != s[3]]
-    assert jobs.shape[0] == sum(int(s[2]) // lay.p for s in nz) * n_lh
-    assert (rel.segments[:, 1] == rel.segments[:, 3]).all()
-    assert len(set(jobs[:, 1].tolist())) == jobs.shape[0]  # destinations are distinct
-    assert jobs[:, 1].min() >= lay.n_pages and rel.n_pages == lay.n_pages + jobs.shape[0]

@@ -1,0 +1,84 @@
+"""The relocation plan (host logic, no GPU): built from the oracle's page
+tables, its jobs must leave, in the working pools, exactly the rotated pages
+that the relocated layout's page tables point at, and nothing more."""
+import numpy as np
+import pytest
+
+import oracle
+from head_aware_paged_prefill_b200 import synth
+from head_aware_paged_prefill_b200.plan import relocation_plan, visible_pages
+
+
+def _check(lay):
+    entries, _ = oracle.page_tables(lay)
+    plan = relocation_plan(lay, entries)
+    n = int(lay.n_pages)
+    n_all = n + plan.n_extra
+    assert plan.layout.n_pages == n_all
+    # every segment of the relocated layout sits at delta 0
+    assert (plan.layout.segments[:, 1] == plan.layout.segments[:, 3]).all()
+    # symbolic working pools: K page -> (store page, rotation), V page -> pool page
+    kc = {p: (p, 0) for p in range(n)}
+    vc = {p: p for p in range(n)}
+    dst_k = plan.jobs_k[:, 1].tolist()
+    assert len(set(dst_k)) == len(dst_k), "two K jobs write one page"
+    for s, d, dl in plan.jobs_k.tolist():
+        assert 0 <= s < n and 0 <= d < n_all
+        assert d == s or d >= n, "an in-place job moved a page"
+        assert dl != 0 or d >= n, "a delta-0 job on a page that already holds it"
+        kc[d] = (s, dl)
+    dst_v = plan.jobs_v[:, 1].tolist()
+    assert len(set(dst_v)) == len(dst_v)
+    for s, d, dl in plan.jobs_v.tolist():
+        assert dl == 0 and 0 <= s < n <= d < n_all
+        vc[d] = vc[s]
+    new_entries, _ = oracle.page_tables(plan.layout)
+    read = set()
+    for t, (a, b) in enumerate(zip(entries, new_entries)):
+        assert a.shape == b.shape, f"table {t}"
+        np.testing.assert_array_equal(a[:, 1], b[:, 1])
+        np.testing.assert_array_equal(a[:, 3], b[:, 3])
+        assert (b[:, 2] == 0).all()
+        for (p0, _, dl, _), p1 in zip(a.tolist(), b[:, 0].tolist()):
+            assert kc[p1] == (p0, dl), f"table {t}: K page {p1} holds {kc[p1]}, want {(p0, dl)}"
+            assert vc[p1] == p0, f"table {t}: V page {p1}"
+            read.add(p1)
+    # no job writes a page that attention never reads
+    assert set(dst_k) <= read and set(dst_v) <= read
+    return plan
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_plan_random_tiny(seed):
+    _check(synth.random_tiny(np.random.default_rng(1000 + seed)))
+
+
+def test_plan_some_random_layout_needs_appended_pages():
+    # shared contents reused at two offsets must occur in the random family
+    extra = sum(_check(synth.random_tiny(np.random.default_rng(1000 + s))).n_extra
+                for s in range(40))
+    assert extra > 0
+
+
+def test_plan_cfg1():
+    plan = _check(synth.cfg1().layout)
+    # kv head 0 (global) sees all 3 x 8 cached pages; kv head 1 (window 128)
+    # sees the 8 pages of the last cached segment; the first segment has delta 0
+    assert plan.jobs_k.shape[0] == 16 + 8 and plan.n_extra == 0
+
+
+def test_plan_cfg3_duplicate_content():
+    lay = synth.cfg3().layout
+    plan = _check(lay)
+    # the duplicated content is seen at two offsets by the global head
+    assert plan.n_extra > 0 and plan.jobs_v.shape[0] > 0
+
+
+def test_visible_pages_cfg2_counts():
+    lay = synth.cfg2().layout
+    entries, _ = oracle.page_tables_closed_form(lay)
+    need = visible_pages(lay, entries)
+    g_pages = sum(len(v) for (s, lh), v in need.items() if lh == 0 and lay.segments[s, 4])
+    l_pages = sum(len(v) for (s, lh), v in need.items() if lh > 0 and lay.segments[s, 4])
+    assert g_pages == 7 * 64          # the global head reads every cached page
+    assert l_pages == 7 * 64          # each local head: the last cached segment (window 4096)
