@@ -57,9 +57,12 @@ struct PrefillCfg {
   static constexpr int kQTileBytes = kRowsPerTile * D * 2;
   static constexpr int kKVTileBytes = kKeysPerTile * D * 2;
   static constexpr int kBlockBytes = kKeysPerTile * 128;  // one column block of a tile
-  static constexpr int kStages = D == 128 ? 2 : 4;
+  // K gets one stage more than V at D = 128: the next S half needs its K
+  // tile a whole softmax earlier than the PV needs its V tile
+  static constexpr int kKStages = D == 128 ? 3 : 4;
+  static constexpr int kVStages = D == 128 ? 2 : 4;
   static constexpr int EPT = kKeysPerTile / P;  // pages per KV tile
-  static constexpr int kDataBytes = 2 * kQTileBytes + 2 * kStages * kKVTileBytes;
+  static constexpr int kDataBytes = 2 * kQTileBytes + (kKStages + kVStages) * kKVTileBytes;
   static constexpr int kSmemBytes = kDataBytes + 1024 + 1024;
   static constexpr uint32_t kTmemCols = 512;
   // TMEM columns: S_t (fp32, P_t as bf16 over its first 64 columns) and O_t
@@ -97,7 +100,8 @@ enum : int {
   kBarQFree = 15,    // fused: every S reading the current Q rotation completed
   kBarQReload = 16,  // fused: original Q re-fetched for a new rotation
   kBarTurn = 17,   // [2] softmax exponential phases take turns (two-head items)
-  kBarKFull = 19,  // [kStages] x 5 groups follow (k_full, k_ready, k_empty, v_full, v_empty)
+  kBarSFree = 19,  // [2] softmax has read S (keys 64-127 of TMEM S may be overwritten)
+  kBarKFull = 21,  // k_full, k_ready, k_empty [kKStages] each, then v_full, v_empty [kVStages]
 };
 
 // kEmuNum pairs of exponentials in every kEmuDen can go through the FMA-pipe
@@ -191,19 +195,20 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                             const __grid_constant__ CUtensorMap tm_v,
                             const __grid_constant__ PrefillParams prm) {
   using C = PrefillCfg<D, P>;
-  constexpr int S = C::kStages;
+  constexpr int SK = C::kKStages, SV = C::kVStages;
+  static_assert(kBarKFull + 3 * SK + 2 * SV <= 64, "barrier slots");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sQ = smem;
   uint8_t* sK = sQ + 2 * C::kQTileBytes;
-  uint8_t* sV = sK + S * C::kKVTileBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + S * C::kKVTileBytes);
+  uint8_t* sV = sK + SK * C::kKVTileBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + SV * C::kKVTileBytes);
   uint64_t* k_full = bars + kBarKFull;
-  uint64_t* k_ready = k_full + S;
-  uint64_t* k_empty = k_ready + S;
-  uint64_t* v_full = k_empty + S;
-  uint64_t* v_empty = v_full + S;
+  uint64_t* k_ready = k_full + SK;
+  uint64_t* k_empty = k_ready + SK;
+  uint64_t* v_full = k_empty + SK;
+  uint64_t* v_empty = v_full + SV;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 64);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
@@ -226,11 +231,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       mbar_init(&bars[kBarPHi + t], 128);
       mbar_init(&bars[kBarOFull + t], 1);
       mbar_init(&bars[kBarOEmpty + t], 128);
+      mbar_init(&bars[kBarSFree + t], 128);
     }
-    for (int s = 0; s < S; ++s) {
+    for (int s = 0; s < SK; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&k_ready[s], 32);
       mbar_init(&k_empty[s], 2);
+    }
+    for (int s = 0; s < SV; ++s) {
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 2);
     }
@@ -290,8 +298,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             }
           }
           {
-            const int st = k_issued % S;
-            const uint32_t u = k_issued / S;
+            const int st = k_issued % SK;
+            const uint32_t u = k_issued / SK;
             if (u > 0 && !(ok = mbar_wait(&k_empty[st], (u - 1) & 1, wc, 2))) break;
             mbar_arrive_expect_tx(&k_full[st], C::kKVTileBytes);
 #pragma unroll
@@ -303,8 +311,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             ++k_issued;
           }
           {
-            const int st = v_issued % S;
-            const uint32_t u = v_issued / S;
+            const int st = v_issued % SV;
+            const uint32_t u = v_issued / SV;
             if (u > 0 && !(ok = mbar_wait(&v_empty[st], (u - 1) & 1, wc, 3))) break;
             mbar_arrive_expect_tx(&v_full[st], C::kKVTileBytes);
 #pragma unroll
@@ -319,10 +327,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       }
       if (!ok) {
         // drain: let every copy this thread started land before the CTA exits
-        for (uint32_t k = (k_issued > S ? k_issued - S : 0); k < k_issued; ++k)
-          mbar_wait_drain(&k_full[k % S], (k / S) & 1);
-        for (uint32_t k = (v_issued > S ? v_issued - S : 0); k < v_issued; ++k)
-          mbar_wait_drain(&v_full[k % S], (k / S) & 1);
+        for (uint32_t k = (k_issued > SK ? k_issued - SK : 0); k < k_issued; ++k)
+          mbar_wait_drain(&k_full[k % SK], (k / SK) & 1);
+        for (uint32_t k = (v_issued > SV ? v_issued - SV : 0); k < v_issued; ++k)
+          mbar_wait_drain(&v_full[k % SV], (k / SV) & 1);
         if (q_uses > 0) mbar_wait_drain(&bars[kBarQFull], (q_uses - 1) & 1);
       }
     }
@@ -336,11 +344,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     if (lane == 0) {
       const int t = warp == 1 ? 0 : 1;
       constexpr uint32_t idesc_s = idesc_bf16_f32(kRowsPerTile, kKeysPerTile, false);
+      constexpr uint32_t idesc_sh = idesc_bf16_f32(kRowsPerTile, kKeysPerTile / 2, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(kRowsPerTile, D, true);
       const uint32_t sQa = smem_u32(sQ) + t * C::kQTileBytes, sKa = smem_u32(sK), sVa = smem_u32(sV);
       const uint32_t tS = tmem + C::col_s(t), tO = tmem + C::col_o(t);
       uint64_t* k_avail = fuse ? k_ready : k_full;
-      uint32_t kv_iter = 0, q_uses = 0, qrd_uses = 0, p_phase = 0, o_uses = 0;
+      uint32_t kv_iter = 0, q_uses = 0, qrd_uses = 0, p_phase = 0, o_uses = 0, sf_phase = 0;
       bool ok = true;
       auto issue_s = [&](int st) {
 #pragma unroll
@@ -349,6 +358,18 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           const uint64_t a = desc_sw128(sQa + off, 16, 1024);
           const uint64_t bd = desc_sw128(sKa + st * C::kKVTileBytes + off, 16, 1024);
           mma_bf16_ss(tS, a, bd, idesc_s, kk > 0 ? 1u : 0u);
+        }
+      };
+      // keys [64 half, 64 half + 64) of S_t = Q_t K^T into TMEM columns
+      // [64 half, 64 half + 64)
+      auto issue_s_half = [&](int st, int half) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::kBlockBytes + (kk & 3) * 32;
+          const uint64_t a = desc_sw128(sQa + off, 16, 1024);
+          const uint64_t bd =
+              desc_sw128(sKa + st * C::kKVTileBytes + half * 64 * 128 + off, 16, 1024);
+          mma_bf16_ss(tS + 64 * half, a, bd, idesc_sh, kk > 0 ? 1u : 0u);
         }
       };
       // O_t (+)= P_t V over keys [64 half, 64 half + 64)
@@ -376,8 +397,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         ++q_uses;
         int dcur = fuse ? __ldg(&prm.entries[w.e_begin].delta) : 0;
         {
-          const int st = kv_iter % S;
-          if (!(ok = mbar_wait(&k_avail[st], (kv_iter / S) & 1, wc, 11))) break;
+          const int st = kv_iter % SK;
+          if (!(ok = mbar_wait(&k_avail[st], (kv_iter / SK) & 1, wc, 11))) break;
           if (active) {
             tc_fence_after();
             issue_s(st);
@@ -387,44 +408,53 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
         for (int j = 0; j < n_tiles && ok; ++j) {
           const uint32_t kj = kv_iter + j;
-          const int st = kj % S;
-          const int stn = (kj + 1) % S;
+          const int st = kj % SV;          // V stage of tile j
+          const int stn = (kj + 1) % SK;   // K stage of tile j + 1
           const bool more = j + 1 < n_tiles;
-          // fused: a tile whose keys need another Q rotation waits for it
           const int dnext =
               (fuse && more) ? __ldg(&prm.entries[w.e_begin + (j + 1) * C::EPT].delta) : dcur;
           const bool qswitch = fuse && dnext != dcur;
+          if (more) {
+            // fused: a tile whose keys need another Q rotation waits for it
+            if (qswitch) {
+              tc_commit(&bars[kBarQFree]);
+              if (!(ok = mbar_wait(&bars[kBarQReady], qrd_uses & 1, wc, 17))) break;
+              ++qrd_uses;
+              dcur = dnext;
+            }
+            // keys 64-127 of the next S go to TMEM columns 64-127 as soon as
+            // the softmax has read S(j): P(j) lives in columns 0-63, so this
+            // half needs neither P(j) nor the PV that consumes it
+            if (!(ok = mbar_wait(&k_avail[stn], ((kj + 1) / SK) & 1, wc, 15))) break;
+            if (active) {
+              if (!(ok = mbar_wait(&bars[kBarSFree + t], sf_phase, wc, 18))) break;
+              sf_phase ^= 1;
+              tc_fence_after();
+              issue_s_half(stn, 1);
+            }
+          }
           if (active) {
             if (!(ok = mbar_wait(&bars[kBarPLo + t], p_phase, wc, 12))) break;
             if (j == 0 && o_uses > 0 &&
                 !(ok = mbar_wait(&bars[kBarOEmpty + t], (o_uses - 1) & 1, wc, 13)))
               break;
-            if (!(ok = mbar_wait(&v_full[st], (kj / S) & 1, wc, 14))) break;
+            if (!(ok = mbar_wait(&v_full[st], (kj / SV) & 1, wc, 14))) break;
             tc_fence_after();
             issue_pv(st, 0, j > 0);
             if (!(ok = mbar_wait(&bars[kBarPHi + t], p_phase, wc, 16))) break;
             p_phase ^= 1;
             tc_fence_after();
             issue_pv(st, 1, true);
-          } else if (!(ok = mbar_wait(&v_full[st], (kj / S) & 1, wc, 14))) {
+            // keys 0-63 of the next S overwrite P(j), after the PV reading it
+            if (more) {
+              issue_s_half(stn, 0);
+              tc_commit(&bars[kBarSFull + t]);
+            }
+          } else if (!(ok = mbar_wait(&v_full[st], (kj / SV) & 1, wc, 14))) {
             break;
           }
           tc_commit(&v_empty[st]);
-          if (qswitch) {
-            tc_commit(&bars[kBarQFree]);
-            if (!(ok = mbar_wait(&bars[kBarQReady], qrd_uses & 1, wc, 17))) break;
-            ++qrd_uses;
-            dcur = dnext;
-          }
-          if (more) {
-            if (!(ok = mbar_wait(&k_avail[stn], ((kj + 1) / S) & 1, wc, 15))) break;
-            if (active) {
-              tc_fence_after();
-              issue_s(stn);
-              tc_commit(&bars[kBarSFull + t]);
-            }
-            tc_commit(&k_empty[stn]);
-          }
+          if (more) tc_commit(&k_empty[stn]);
         }
         if (!ok) break;
         if (active) {
@@ -508,8 +538,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             mbar_arrive(&bars[kBarQReady]);
             dq = dt;
           }
-          const int st = k_seen % S;
-          if (!(ok = mbar_wait(&k_full[st], (k_seen / S) & 1, wc, 30))) break;
+          const int st = k_seen % SK;
+          if (!(ok = mbar_wait(&k_full[st], (k_seen / SK) & 1, wc, 30))) break;
           uint8_t* tile = sK + st * C::kKVTileBytes;
           for (int e = 1; e < C::EPT; ++e) {
             const int idx = w.e_begin + j * C::EPT + e;
@@ -582,6 +612,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         tc_fence_after();
         float s[kKeysPerTile];
         tmem_ld_x128_wait(tS, s);
+        // S is in registers: the issuer may start the next S's upper half
+        if (j + 1 < n_tiles) {
+          tc_fence_before();
+          mbar_arrive(&bars[kBarSFree + t]);
+        }
         bool full = true;
 #pragma unroll
         for (int e = 0; e < C::EPT; ++e) full = full && nv[e] == P;
