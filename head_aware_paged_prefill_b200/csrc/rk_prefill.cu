@@ -17,18 +17,21 @@
 //   warp 0      TMA producer: Q tiles (3-D box out of [rows][Hq][D]) and, per
 //               KV tile, one box per page and 64-column block out of the pool.
 //   warps 1, 3  tcgen05 issuers, one per Q tile (warp 1 also owns TMEM).
-//               S_t = Q_t K^T (M=128, N=128, K=D) into TMEM; O_t += P_t V
+//               S_t = Q_t K^T (M=128, N=128, K=D) into ONE S buffer shared by
+//               both tiles: a softmax copies S to registers as soon as it
+//               lands, so the next S (of the other tile) can follow at once,
+//               while P_t (bf16) goes to its own 64 TMEM columns.  O_t += P_t V
 //               (M=128, N=D, K=128) with P_t read from TMEM and V from shared
-//               memory (MN-major operand), issued per 64-key half as soon as
-//               that half of P is stored.
+//               memory (MN-major operand).  Per KV tile j issuer t puts
+//               S_t(j + 1) in the buffer, then issues PV_t(j).
 //   warp 2      RoPE relocation (fuse_rope): rotates the Q tiles by -delta
 //               once per run of tiles sharing a delta, and the K pages of a
 //               tile that mixes deltas by their difference.
 //   warps 4-7   softmax warpgroup of Q tile 0, warps 8-11 of Q tile 1: one
 //               TMEM lane (= one query row) per thread; online softmax in the
 //               log2 domain, O rescaled in TMEM only when the running max
-//               grows by more than 2^8, P written back over S as bf16 in
-//               16-column quarters.  The two warpgroups' exponential phases
+//               grows by more than 2^8 (after the previous PV completed), P
+//               stored as bf16 in 16-column quarters.  The two warpgroups' exponential phases
 //               take turns (a pair of mbarriers), so they never compete for
 //               the MUFU while their other phases overlap.
 // Registers are rebalanced with setmaxnreg: the first warpgroup keeps 80 per
@@ -57,17 +60,20 @@ struct PrefillCfg {
   static constexpr int kQTileBytes = kRowsPerTile * D * 2;
   static constexpr int kKVTileBytes = kKeysPerTile * D * 2;
   static constexpr int kBlockBytes = kKeysPerTile * 128;  // one column block of a tile
-  // K gets one stage more than V at D = 128: the next S half needs its K
-  // tile a whole softmax earlier than the PV needs its V tile
+  // K gets one stage more than V at D = 128: the next S needs its K tile a
+  // whole softmax phase earlier than the PV needs its V tile
   static constexpr int kKStages = D == 128 ? 3 : 4;
   static constexpr int kVStages = D == 128 ? 2 : 4;
   static constexpr int EPT = kKeysPerTile / P;  // pages per KV tile
   static constexpr int kDataBytes = 2 * kQTileBytes + (kKStages + kVStages) * kKVTileBytes;
   static constexpr int kSmemBytes = kDataBytes + 1024 + 1024;
   static constexpr uint32_t kTmemCols = 512;
-  // TMEM columns: S_t (fp32, P_t as bf16 over its first 64 columns) and O_t
-  __host__ __device__ static constexpr uint32_t col_s(int t) { return t ? 128u : 0u; }
-  __host__ __device__ static constexpr uint32_t col_o(int t) { return t ? 256u + D : 256u; }
+  // TMEM columns: O_t at 128 t, one S buffer (fp32) shared by both Q tiles
+  // at 256 (a softmax copies S to registers as soon as it lands, so the
+  // other tile's S can follow), and P_t (bf16, 128 keys) at 384 + 64 t
+  __host__ __device__ static constexpr uint32_t col_o(int t) { return 128u * t; }
+  static constexpr uint32_t kColS = 256;
+  __host__ __device__ static constexpr uint32_t col_p(int t) { return 384u + 64u * t; }
 };
 
 struct PrefillParams {
@@ -90,17 +96,17 @@ struct PrefillParams {
 enum : int {
   kBarQFull = 0,
   kBarQEmpty = 1,
-  kBarSFull = 2,   // [2]
-  kBarPLo = 4,     // [2] P columns of keys 0-63 stored
-  kBarOFull = 6,   // [2]
-  kBarOEmpty = 8,  // [2]
-  kBarDrain = 10,  // [2] MMA completion before TMEM is released (one per issuer)
-  kBarPHi = 12,    // [2] P columns of keys 64-127 stored
-  kBarQReady = 14,   // fused: the Q tiles hold the rotation the next S needs
-  kBarQFree = 15,    // fused: every S reading the current Q rotation completed
-  kBarQReload = 16,  // fused: original Q re-fetched for a new rotation
-  kBarTurn = 17,   // [2] softmax exponential phases take turns (two-head items)
-  kBarSFree = 19,  // [2] softmax has read S (keys 64-127 of TMEM S may be overwritten)
+  kBarSFull = 2,    // [2] S of Q tile t computed
+  kBarSFree = 4,    // [2] S buffer read; the next S is issuer t's (one phase per S of t)
+  kBarP = 6,        // [2] P of Q tile t stored
+  kBarPVDone = 8,   // [2] each PV of Q tile t completed (P_t and O_t reusable)
+  kBarOFull = 10,   // [2]
+  kBarOEmpty = 12,  // [2]
+  kBarDrain = 14,   // [2] MMA completion before TMEM is released (one per issuer)
+  kBarQReady = 16,   // fused: the Q tiles hold the rotation the next S needs
+  kBarQFree = 17,    // fused: every S reading the current Q rotation completed
+  kBarQReload = 18,  // fused: original Q re-fetched for a new rotation
+  kBarTurn = 19,   // [2] softmax exponential phases take turns (two-head items)
   kBarKFull = 21,  // k_full, k_ready, k_empty [kKStages] each, then v_full, v_empty [kVStages]
 };
 
@@ -216,6 +222,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   const bool fuse = prm.fuse_rope != 0;
 
   if (threadIdx.x == 0) {
+    // counts: 1 = one elected thread (or a tcgen05.commit), 2 = both
+    // issuers, 32 = the RoPE warp, 128 = a softmax warpgroup
     mbar_init(&bars[kBarQFull], 1);
     mbar_init(&bars[kBarQEmpty], 2);
     mbar_init(&bars[kBarDrain], 1);
@@ -223,15 +231,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     mbar_init(&bars[kBarQReady], 32);
     mbar_init(&bars[kBarQFree], 2);
     mbar_init(&bars[kBarQReload], 1);
-    mbar_init(&bars[kBarTurn], 128);
-    mbar_init(&bars[kBarTurn + 1], 128);
     for (int t = 0; t < 2; ++t) {
+      mbar_init(&bars[kBarSFree + t], 128);
+      mbar_init(&bars[kBarTurn + t], 128);
       mbar_init(&bars[kBarSFull + t], 1);
-      mbar_init(&bars[kBarPLo + t], 128);
-      mbar_init(&bars[kBarPHi + t], 128);
+      mbar_init(&bars[kBarP + t], 128);
+      mbar_init(&bars[kBarPVDone + t], 1);
       mbar_init(&bars[kBarOFull + t], 1);
       mbar_init(&bars[kBarOEmpty + t], 128);
-      mbar_init(&bars[kBarSFree + t], 128);
     }
     for (int s = 0; s < SK; ++s) {
       mbar_init(&k_full[s], 1);
@@ -336,50 +343,59 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     }
   } else if (warp == 1 || warp == 3) {
     // ------------------------------------------------------- MMA issuers
-    // One issuing thread per Q tile (warp 1: tile 0, warp 3: tile 1), so the
-    // two tiles' S -> softmax -> PV chains never wait on each other.  K / V
-    // stages, the Q buffers and the Q-rotation handoff are released by both
-    // issuers (barrier counts of 2); an issuer whose tile is absent from an
-    // item (a single q head) still steps through the item's barriers.
+    // One issuing thread per Q tile (warp 1: tile 0, warp 3: tile 1): a
+    // tcgen05.mma holds its issuing thread until the tensor pipe takes it,
+    // so each tile's MMAs need their own thread.  Per KV tile j, issuer t
+    // puts S_t(j + 1) into the shared S buffer, then issues PV_t(j) once P_t(j)
+    // is stored.  The S buffer is taken in a fixed global order
+    // (S_0(j), S_1(j), S_0(j + 1), ...): S number n waits until the softmax
+    // has read S number n - 1 (kBarSFree completes once per S), so the next S
+    // of one tile is computed while the other tile runs its exponentials.
+    // K / V stages, Q buffers and the Q-rotation handoff are released by both
+    // issuers (counts of 2); an issuer whose tile is absent from an item (a
+    // single q head) still steps through them.
     if (lane == 0) {
       const int t = warp == 1 ? 0 : 1;
       constexpr uint32_t idesc_s = idesc_bf16_f32(kRowsPerTile, kKeysPerTile, false);
-      constexpr uint32_t idesc_sh = idesc_bf16_f32(kRowsPerTile, kKeysPerTile / 2, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(kRowsPerTile, D, true);
       const uint32_t sQa = smem_u32(sQ) + t * C::kQTileBytes, sKa = smem_u32(sK), sVa = smem_u32(sV);
-      const uint32_t tS = tmem + C::col_s(t), tO = tmem + C::col_o(t);
+      const uint32_t tO = tmem + C::col_o(t), tP = tmem + C::col_p(t);
       uint64_t* k_avail = fuse ? k_ready : k_full;
-      uint32_t kv_iter = 0, q_uses = 0, qrd_uses = 0, p_phase = 0, o_uses = 0, sf_phase = 0;
+      uint32_t kv_iter = 0, q_uses = 0, qrd_uses = 0, p_phase = 0, o_uses = 0;
+      uint32_t sf_uses = 0;  // phases of this issuer's kBarSFree consumed
+      bool any_s = false;    // this issuer has put an S in the buffer before
       bool ok = true;
-      auto issue_s = [&](int st) {
+      // S_t = Q_t K^T (M=128, N=128, K=D) into the shared S buffer.  The
+      // softmax that reads the S before it in the global order arrives on
+      // this issuer's kBarSFree, so each issuer waits every phase of its own
+      // barrier in order (a parity wait that skipped phases could match an
+      // older completed phase of the same parity).  The kernel's very first S
+      // (tile 0's) has no predecessor.
+      auto issue_s = [&](int kst) {
+        if (t == 1 || any_s) {
+          if (!(ok = mbar_wait(&bars[kBarSFree + t], sf_uses & 1, wc, 18))) return;
+          ++sf_uses;
+        }
+        any_s = true;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::kBlockBytes + (kk & 3) * 32;
           const uint64_t a = desc_sw128(sQa + off, 16, 1024);
-          const uint64_t bd = desc_sw128(sKa + st * C::kKVTileBytes + off, 16, 1024);
-          mma_bf16_ss(tS, a, bd, idesc_s, kk > 0 ? 1u : 0u);
+          const uint64_t bd = desc_sw128(sKa + kst * C::kKVTileBytes + off, 16, 1024);
+          mma_bf16_ss(tmem + C::kColS, a, bd, idesc_s, kk > 0 ? 1u : 0u);
         }
+        tc_commit(&bars[kBarSFull + t]);
       };
-      // keys [64 half, 64 half + 64) of S_t = Q_t K^T into TMEM columns
-      // [64 half, 64 half + 64)
-      auto issue_s_half = [&](int st, int half) {
+      // O_t (+)= P_t V (M=128, N=D, K=128), P_t read from TMEM
+      auto issue_pv = [&](int vst, bool acc) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::kBlockBytes + (kk & 3) * 32;
-          const uint64_t a = desc_sw128(sQa + off, 16, 1024);
+        for (int kk = 0; kk < kKeysPerTile / 16; ++kk) {
           const uint64_t bd =
-              desc_sw128(sKa + st * C::kKVTileBytes + half * 64 * 128 + off, 16, 1024);
-          mma_bf16_ss(tS + 64 * half, a, bd, idesc_sh, kk > 0 ? 1u : 0u);
+              desc_sw128(sVa + vst * C::kKVTileBytes + kk * 16 * 128, C::kBlockBytes, 1024);
+          mma_bf16_ts(tO, tP + kk * 8, bd, idesc_o, (acc || kk > 0) ? 1u : 0u);
         }
-      };
-      // O_t (+)= P_t V over keys [64 half, 64 half + 64)
-      auto issue_pv = [&](int st, int half, bool acc) {
-#pragma unroll
-        for (int kk = 4 * half; kk < 4 * half + 4; ++kk) {
-          const uint64_t bd =
-              desc_sw128(sVa + st * C::kKVTileBytes + kk * 16 * 128, C::kBlockBytes, 1024);
-          mma_bf16_ts(tO, tS + kk * 8, bd, idesc_o, (acc || kk > 0) ? 1u : 0u);
-        }
+        tc_commit(&bars[kBarPVDone + t]);
       };
       for (int r = 0; ok; ++r) {
         const int it = item_of_round(r, b, G);
@@ -387,7 +403,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         const Item w = prm.items[it];
         const int n_tiles = (w.e_end - w.e_begin + C::EPT - 1) / C::EPT;
         if (n_tiles == 0) continue;
-        const bool active = t < w.nh;
+        const int nh = w.nh;
+        const bool active = t < nh;
         if (fuse) {
           if (!(ok = mbar_wait(&bars[kBarQReady], qrd_uses & 1, wc, 10))) break;
           ++qrd_uses;
@@ -396,65 +413,53 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
         ++q_uses;
         int dcur = fuse ? __ldg(&prm.entries[w.e_begin].delta) : 0;
-        {
-          const int st = kv_iter % SK;
-          if (!(ok = mbar_wait(&k_avail[st], (kv_iter / SK) & 1, wc, 11))) break;
-          if (active) {
-            tc_fence_after();
-            issue_s(st);
-            tc_commit(&bars[kBarSFull + t]);
+        // K stage of KV tile jn, resident (and, fused, Q rotated for it)
+        auto k_tile = [&](int jn) -> int {
+          if (fuse && jn > 0) {
+            const int dn = __ldg(&prm.entries[w.e_begin + jn * C::EPT].delta);
+            if (dn != dcur) {
+              // every S that read the old rotation precedes this commit
+              tc_commit(&bars[kBarQFree]);
+              if (!(ok = mbar_wait(&bars[kBarQReady], qrd_uses & 1, wc, 17))) return 0;
+              ++qrd_uses;
+              dcur = dn;
+            }
           }
-          tc_commit(&k_empty[st]);
+          const uint32_t kj = kv_iter + jn;
+          const int kst = kj % SK;
+          ok = mbar_wait(&k_avail[kst], (kj / SK) & 1, wc, 11);
+          return kst;
+        };
+        {
+          const int kst = k_tile(0);
+          if (ok && active) issue_s(kst);
+          if (ok) tc_commit(&k_empty[kst]);
         }
         for (int j = 0; j < n_tiles && ok; ++j) {
           const uint32_t kj = kv_iter + j;
-          const int st = kj % SV;          // V stage of tile j
-          const int stn = (kj + 1) % SK;   // K stage of tile j + 1
+          const int vst = kj % SV;
           const bool more = j + 1 < n_tiles;
-          const int dnext =
-              (fuse && more) ? __ldg(&prm.entries[w.e_begin + (j + 1) * C::EPT].delta) : dcur;
-          const bool qswitch = fuse && dnext != dcur;
+          int kstn = 0;
           if (more) {
-            // fused: a tile whose keys need another Q rotation waits for it
-            if (qswitch) {
-              tc_commit(&bars[kBarQFree]);
-              if (!(ok = mbar_wait(&bars[kBarQReady], qrd_uses & 1, wc, 17))) break;
-              ++qrd_uses;
-              dcur = dnext;
-            }
-            // keys 64-127 of the next S go to TMEM columns 64-127 as soon as
-            // the softmax has read S(j): P(j) lives in columns 0-63, so this
-            // half needs neither P(j) nor the PV that consumes it
-            if (!(ok = mbar_wait(&k_avail[stn], ((kj + 1) / SK) & 1, wc, 15))) break;
+            kstn = k_tile(j + 1);
+            if (!ok) break;
             if (active) {
-              if (!(ok = mbar_wait(&bars[kBarSFree + t], sf_phase, wc, 18))) break;
-              sf_phase ^= 1;
-              tc_fence_after();
-              issue_s_half(stn, 1);
+              issue_s(kstn);
+              if (!ok) break;
             }
           }
+          if (!(ok = mbar_wait(&v_full[vst], (kj / SV) & 1, wc, 14))) break;
           if (active) {
-            if (!(ok = mbar_wait(&bars[kBarPLo + t], p_phase, wc, 12))) break;
+            if (!(ok = mbar_wait(&bars[kBarP + t], p_phase, wc, 12))) break;
+            p_phase ^= 1;
             if (j == 0 && o_uses > 0 &&
                 !(ok = mbar_wait(&bars[kBarOEmpty + t], (o_uses - 1) & 1, wc, 13)))
               break;
-            if (!(ok = mbar_wait(&v_full[st], (kj / SV) & 1, wc, 14))) break;
             tc_fence_after();
-            issue_pv(st, 0, j > 0);
-            if (!(ok = mbar_wait(&bars[kBarPHi + t], p_phase, wc, 16))) break;
-            p_phase ^= 1;
-            tc_fence_after();
-            issue_pv(st, 1, true);
-            // keys 0-63 of the next S overwrite P(j), after the PV reading it
-            if (more) {
-              issue_s_half(stn, 0);
-              tc_commit(&bars[kBarSFull + t]);
-            }
-          } else if (!(ok = mbar_wait(&v_full[st], (kj / SV) & 1, wc, 14))) {
-            break;
+            issue_pv(vst, j > 0);
           }
-          tc_commit(&v_empty[st]);
-          if (more) tc_commit(&k_empty[stn]);
+          if (more) tc_commit(&k_empty[kstn]);
+          tc_commit(&v_empty[vst]);
         }
         if (!ok) break;
         if (active) {
@@ -562,11 +567,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t tS = tmem + lane_base + C::col_s(t);
+    const uint32_t tS = tmem + lane_base + C::kColS;
+    const uint32_t tP = tmem + lane_base + C::col_p(t);
     const uint32_t tO = tmem + lane_base + C::col_o(t);
     const float sl2 = prm.scale_log2;
     const int T = prm.total_tokens;
     uint32_t s_phase = 0, o_uses = 0, turn_phase = 0;
+    uint32_t n_pv = 0;  // PVs of this Q tile issued before the current tile
     bool ok = true;
     for (int r = 0; ok; ++r) {
       const int it = item_of_round(r, b, G);
@@ -612,11 +619,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         tc_fence_after();
         float s[kKeysPerTile];
         tmem_ld_x128_wait(tS, s);
-        // S is in registers: the issuer may start the next S's upper half
-        if (j + 1 < n_tiles) {
-          tc_fence_before();
-          mbar_arrive(&bars[kBarSFree + t]);
-        }
+        // S is in registers: the issuer of the next S in the global order
+        // (S_1 of this tile after S_0 of a two-head item, else an S_0) may
+        // put it in the buffer
+        tc_fence_before();
+        mbar_arrive(&bars[kBarSFree + ((t == 0 && w.nh == 2) ? 1 : 0)]);
         bool full = true;
 #pragma unroll
         for (int e = 0; e < C::EPT; ++e) full = full && nv[e] == P;
@@ -643,6 +650,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         const float m_new = fmaxf(m_ref, mx * sl2);
         const bool resc = m_new > m_ref + kRescaleLog2;
         if (j > 0 && __any_sync(0xffffffffu, resc)) {
+          // O holds the sum through the previous tile's PV: let it finish
+          if (!(ok = mbar_wait(&bars[kBarPVDone + t], (n_pv - 1) & 1, wc, 23))) break;
+          tc_fence_after();
           const float alpha = resc ? ex2_approx(m_ref - m_new) : 1.f;
 #pragma unroll
           for (int cc = 0; cc < D / 32; ++cc) {
@@ -681,6 +691,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
               sh[2 * k + 1] = ex2_approx(sh[2 * k + 1]);
             }
           }
+          // P_t still feeds the previous PV until that completes (its phase
+          // is waited even across items, so no phase of the barrier is skipped)
+          if (half == 0 && n_pv > 0) {
+            if (!(ok = mbar_wait(&bars[kBarPVDone + t], (n_pv - 1) & 1, wc, 24))) break;
+            tc_fence_after();
+          }
 #pragma unroll
           for (int q = 0; q < 2; ++q) {
             uint32_t pk[16];
@@ -690,17 +706,19 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
               acc2[k & 1] = f2_add(acc2[k & 1], f2_pack(sh[2 * kk], sh[2 * kk + 1]));
               pk[k] = pack_bf16x2(sh[2 * kk], sh[2 * kk + 1]);
             }
-            tmem_st_x16(tS + 32 * half + 16 * q, pk);
+            tmem_st_x16(tP + 32 * half + 16 * q, pk);
           }
-          tmem_st_wait();
-          tc_fence_before();
-          mbar_arrive(&bars[(half ? kBarPHi : kBarPLo) + t]);
-          // the other warpgroup's turn once this one's exponentials are done
-          // (tile 1 hands back after every tile but the item's last)
-          if (half == 1 && w.nh == 2) {
-            turn_phase ^= 1;
-            if (t == 0 || j + 1 < n_tiles) mbar_arrive(&bars[kBarTurn + (1 - t)]);
-          }
+        }
+        if (!ok) break;
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bars[kBarP + t]);
+        ++n_pv;
+        // the other warpgroup's turn once this one's exponentials are done
+        // (tile 1 hands back after every tile but the item's last)
+        if (w.nh == 2) {
+          turn_phase ^= 1;
+          if (t == 0 || j + 1 < n_tiles) mbar_arrive(&bars[kBarTurn + (1 - t)]);
         }
         float a0, a1, b0, b1;
         f2_unpack(acc2[0], a0, a1);
