@@ -668,6 +668,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
         if (resc) m_ref = m_new;
         const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
+        // P_t still feeds the previous PV until that completes; waited here,
+        // while the other warpgroup has the turn (every phase of the barrier
+        // is waited, across items too, so none is skipped)
+        if (n_pv > 0) {
+          if (!(ok = mbar_wait(&bars[kBarPVDone + t], (n_pv - 1) & 1, wc, 24))) break;
+          tc_fence_after();
+        }
         // two-head items: the two warpgroups' exponential phases alternate
         // (tile 0's first), so they never compete for the MUFU and issue slots
         if (w.nh == 2 && !(ok = mbar_wait(&bars[kBarTurn + t], turn_phase, wc, 22))) break;
@@ -691,11 +698,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
               sh[2 * k + 1] = ex2_approx(sh[2 * k + 1]);
             }
           }
-          // P_t still feeds the previous PV until that completes (its phase
-          // is waited even across items, so no phase of the barrier is skipped)
-          if (half == 0 && n_pv > 0) {
-            if (!(ok = mbar_wait(&bars[kBarPVDone + t], (n_pv - 1) & 1, wc, 24))) break;
-            tc_fence_after();
+          // the other warpgroup's turn as soon as the last exponential is
+          // issued: its wake-up overlaps this one's packing and P stores
+          // (tile 1 hands back after every tile but the item's last)
+          if (half == 1 && w.nh == 2) {
+            turn_phase ^= 1;
+            if (t == 0 || j + 1 < n_tiles) mbar_arrive(&bars[kBarTurn + (1 - t)]);
           }
 #pragma unroll
           for (int q = 0; q < 2; ++q) {
@@ -709,17 +717,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             tmem_st_x16(tP + 32 * half + 16 * q, pk);
           }
         }
-        if (!ok) break;
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&bars[kBarP + t]);
         ++n_pv;
-        // the other warpgroup's turn once this one's exponentials are done
-        // (tile 1 hands back after every tile but the item's last)
-        if (w.nh == 2) {
-          turn_phase ^= 1;
-          if (t == 0 || j + 1 < n_tiles) mbar_arrive(&bars[kBarTurn + (1 - t)]);
-        }
         float a0, a1, b0, b1;
         f2_unpack(acc2[0], a0, a1);
         f2_unpack(acc2[1], b0, b1);
