@@ -122,6 +122,10 @@ enum : int {
 #define RK_EMU_DEN 4
 #endif
 constexpr int kEmuNum = RK_EMU_NUM;
+#ifndef RK_TURN_AT
+#define RK_TURN_AT 16
+#endif
+constexpr int kTurnAt = RK_TURN_AT;  // exponential pairs of the last half before the turn passes
 constexpr int kEmuDen = RK_EMU_DEN;
 
 // Item of round r for CTA b (boustrophedon over the cost-sorted list).
@@ -691,6 +695,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           }
 #pragma unroll
           for (int k = 0; k < 32; ++k) {
+            // the other warpgroup's turn once kTurnAt pairs of the last half
+            // are issued: its wake-up overlaps this one's remaining
+            // exponentials, packing and P stores (tile 1 hands back after
+            // every tile but the item's last)
+            if (half == 1 && k == kTurnAt && w.nh == 2) {
+              turn_phase ^= 1;
+              if (t == 0 || j + 1 < n_tiles) mbar_arrive(&bars[kBarTurn + (1 - t)]);
+            }
             if (k % kEmuDen >= kEmuDen - kEmuNum) {
               exp2_poly_pair(sh[2 * k], sh[2 * k + 1], sh[2 * k], sh[2 * k + 1]);
             } else {
@@ -698,10 +710,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
               sh[2 * k + 1] = ex2_approx(sh[2 * k + 1]);
             }
           }
-          // the other warpgroup's turn as soon as the last exponential is
-          // issued: its wake-up overlaps this one's packing and P stores
-          // (tile 1 hands back after every tile but the item's last)
-          if (half == 1 && w.nh == 2) {
+          if (half == 1 && kTurnAt >= 32 && w.nh == 2) {
             turn_phase ^= 1;
             if (t == 0 || j + 1 < n_tiles) mbar_arrive(&bars[kBarTurn + (1 - t)]);
           }
