@@ -80,7 +80,8 @@ class SegPagedPrefill:
     # Number of library kernel launches one run() makes.
     @property
     def launches_per_run(self) -> int:
-        return 3 + int(self.plan.jobs_k.shape[0] > 0) + int(self.plan.jobs_v.shape[0] > 0)
+        # select (one kernel) + attention, plus the relocation launches
+        return 2 + int(self.plan.jobs_k.shape[0] > 0) + int(self.plan.jobs_v.shape[0] > 0)
 
     def load(self, q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor):
         """Copies inputs (host or device) into the device working buffers."""

@@ -3,6 +3,7 @@
 // host is done here, synchronously, before any GPU work is enqueued.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -177,6 +178,10 @@ void build_layout_image(const rk_dims* d, const rk_layout* lay, const Derived& d
   v.total_pages = static_cast<int32_t>(dv.total_pages);
   v.window = lay->class_window[RK_LOCAL];
   v.item_capacity = static_cast<int32_t>(dv.item_capacity);
+  int32_t max_pages = 0;
+  for (int r = 0; r < d->n_req; ++r)
+    max_pages = std::max(max_pages, dv.page_prefix[r + 1] - dv.page_prefix[r]);
+  v.max_table_pages = max_pages;
   int32_t off = static_cast<int32_t>((sizeof(LayoutView) + 3) / 4);
   int32_t* w = img->data();
   v.off_seg = off;
@@ -211,7 +216,46 @@ void build_layout_image(const rk_dims* d, const rk_layout* lay, const Derived& d
   v.off_retr_pages = off;
   if (dv.n_retr > 0) std::memcpy(w + off, lay->retr_pages, 4 * static_cast<size_t>(dv.n_retr));
   off += static_cast<int32_t>(dv.n_retr);
+  // work items per table (the attention work list's shape, known from the
+  // layout): <= 128-row tiles of the table's row set x pairs of q heads; the
+  // row set follows the class rule that the select kernel also applies
+  // (global / dense: the whole request; local / retrieval: the uncached
+  // segments, adjacent ones merged)
   v.off_tile_prefix = off;
+  {
+    const int G = d->num_q_heads / d->num_kv_heads;
+    const int npairs = (G + 1) / 2;
+    int64_t acc = 0;
+    for (int r = 0; r < d->n_req; ++r) {
+      const int L = lay->cu_seqlens[r + 1] - lay->cu_seqlens[r];
+      int all_tiles = (L + kRowsPerTile - 1) / kRowsPerTile;
+      int unc_tiles = 0;
+      for (int sg = dv.seg_indptr[r], cur_b = -1, cur_e = -1; sg <= dv.seg_indptr[r + 1]; ++sg) {
+        const bool end = sg == dv.seg_indptr[r + 1];
+        const bool unc = !end && !lay->segments[sg].cached;
+        const int a = end ? 0 : lay->segments[sg].logical_start;
+        if (unc && cur_e == a) {
+          cur_e = a + lay->segments[sg].len;
+          continue;
+        }
+        if (cur_e > cur_b) unc_tiles += (cur_e - cur_b + kRowsPerTile - 1) / kRowsPerTile;
+        cur_b = cur_e = -1;
+        if (unc) {
+          cur_b = a;
+          cur_e = a + lay->segments[sg].len;
+        }
+      }
+      for (int layer = 0; layer < d->n_layers; ++layer)
+        for (int h = 0; h < d->num_kv_heads; ++h) {
+          const int t = (r * d->n_layers + layer) * d->num_kv_heads + h;
+          const int cls = lay->class_map[layer * d->num_kv_heads + h];
+          w[off + t] = static_cast<int32_t>(acc);
+          acc += static_cast<int64_t>(npairs) *
+                 ((cls == RK_GLOBAL || cls == RK_DENSE) ? all_tiles : unc_tiles);
+        }
+    }
+    w[off + dv.n_tables] = static_cast<int32_t>(acc);
+  }
   off += static_cast<int32_t>(dv.n_tables + 1);
   v.layout_words = off;
   std::memcpy(w, &v, sizeof(LayoutView));
@@ -253,16 +297,12 @@ extern "C" rk_status rk_select_visible(const rk_dims* dims, const rk_layout* lay
   if (out->entry_capacity < dv.entry_capacity || out->range_capacity < dv.range_capacity ||
       workspace_bytes < dv.map.total)
     return RK_ERR_CAPACITY;
-  // header + layout image, one host-to-device copy each
-  WsHeader hdr{};
-  hdr.n_tables = static_cast<int32_t>(dv.n_tables);
-  hdr.item_capacity = static_cast<int32_t>(dv.item_capacity);
+  // one host-to-device copy: the layout image (its error word and completion
+  // counter zeroed); the select kernel's last CTA rewrites the header
   std::vector<int32_t> img;
   build_layout_image(dims, layout, dv, &img);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  if (cudaMemcpyAsync(ws, &hdr, sizeof hdr, cudaMemcpyHostToDevice, s) != cudaSuccess)
-    return RK_ERR_CUDA;
   if (cudaMemcpyAsync(ws + dv.map.layout, img.data(), 4 * img.size(), cudaMemcpyHostToDevice, s) !=
       cudaSuccess)
     return RK_ERR_CUDA;

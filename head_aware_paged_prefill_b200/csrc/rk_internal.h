@@ -48,6 +48,10 @@ struct LayoutView {
   int32_t total_tokens, total_pages;  // total_pages = sum_r ceil(L_r / P)
   int32_t window;                     // class_window[RK_LOCAL]
   int32_t item_capacity;
+  int32_t max_table_pages;            // max_r ceil(L_r / P)
+  // written by the select kernel (the host uploads them as zero each call)
+  int32_t error;       // RK_DEV_* bits raised while selecting
+  int32_t done_count;  // CTAs of the select kernel that finished their table
   // offsets (in int32 elements from the start of the layout block)
   int32_t off_seg;          // [n_seg][5]
   int32_t off_seg_indptr;   // [n_req + 1]
@@ -57,7 +61,7 @@ struct LayoutView {
   int32_t off_class;        // [n_layers * hkv]
   int32_t off_retr_indptr;  // [n_tables + 1]
   int32_t off_retr_pages;   // [n_retr]
-  int32_t off_tile_prefix;  // [n_tables + 1] scratch: items per table, scanned
+  int32_t off_tile_prefix;  // [n_tables + 1] exclusive prefix of the work items per table
   int32_t layout_words;
 };
 

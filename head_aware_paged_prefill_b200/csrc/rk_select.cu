@@ -2,11 +2,15 @@
 // per request, choose which reused KV each head sees; README excerpt
 // "SegPagedAttention Runtime": per-head page table over a segmented store).
 //
-// select_tables_kernel : one CTA per table (request, layer, kv_head) derives
-//   the ordered page table and the merged row ranges from the class rules.
-// build_worklist_kernel: one CTA turns the tables into attention work items
-//   (<= 128 rows x up to two q heads of one kv head) with the entry range each
-//   item needs, sorted by cost (KV tiles), longest first.
+// One launch, one CTA per table (request, layer, kv_head):
+//   1. the ordered page table and the merged row ranges, from the class rule;
+//   2. the table's attention work items (<= 128 rows x up to two q heads of
+//      one kv head) with the entry range each needs, found by binary search
+//      over the table's page positions kept in shared memory; the host gives
+//      every table's first item (the item counts follow from the layout);
+//   3. the last CTA to finish (a counter in the uploaded layout block) sorts
+//      all items by cost (KV tiles), longest first, and publishes the item
+//      count and the selection's error bits in the workspace header.
 #include <cuda_runtime.h>
 
 #include "rk_internal.h"
@@ -46,11 +50,28 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int* t
 }
 
 constexpr int kSelectThreads = 256;
+constexpr int kCostBuckets = 4096;
+constexpr int kPosCap = 3072;  // page positions of one table kept in shared memory
+
+// index of the first of n entries whose key exceeds v (keys ascending)
+template <typename Key>
+__device__ __forceinline__ int upper_bound(int n, int v, Key key) {
+  int a = 0, b = n;
+  while (a < b) {
+    const int mid = (a + b) >> 1;
+    if (key(mid) <= v) a = mid + 1; else b = mid;
+  }
+  return a;
+}
 
 __global__ void __launch_bounds__(kSelectThreads)
-    select_tables_kernel(const LayoutView* __restrict__ lv, rk_visible vis, WsHeader* hdr) {
+    select_kernel(LayoutView* __restrict__ lv, rk_visible vis, WsHeader* hdr, Item* items_tmp,
+                  Item* items) {
   __shared__ int warp_tot[kSelectThreads / 32];
   __shared__ int s_total;
+  __shared__ int s_last;
+  __shared__ int hist[kCostBuckets];
+  __shared__ int2 s_pos[kPosCap];  // (logical_pos, n_valid) of the table's entries
   const int t = blockIdx.x;
   const int hkv = lv->hkv, n_layers = lv->n_layers, P = lv->p;
   const int kvh = t % hkv, layer = (t / hkv) % n_layers, r = t / (hkv * n_layers);
@@ -64,6 +85,7 @@ __global__ void __launch_bounds__(kSelectThreads)
   const int32_t* cls_arr = lv_arr(lv, lv->off_class);
   const int32_t* retr_indptr = lv_arr(lv, lv->off_retr_indptr);
   const int32_t* retr_pages = lv_arr(lv, lv->off_retr_pages);
+  const int32_t* tile_prefix = lv_arr(lv, lv->off_tile_prefix);
 
   const int L = cu[r + 1] - cu[r];
   const int npg = (L + P - 1) / P;
@@ -79,6 +101,7 @@ __global__ void __launch_bounds__(kSelectThreads)
   for (int s = s0; s < s1; ++s)
     if (!seg[5 * s + 4]) last_unc = max(last_unc, seg[5 * s + 1] + seg[5 * s + 2] - 1);
 
+  // ---- 1. page table
   int count = 0;
   for (int base = 0; base < npg; base += kSelectThreads) {
     const int k = base + threadIdx.x;
@@ -115,9 +138,7 @@ __global__ void __launch_bounds__(kSelectThreads)
       if (flag) {
         const int pis = (pos - start) / P;
         int64_t phys = static_cast<int64_t>(page_base[static_cast<int64_t>(s) * n_lh + lh]) + pis;
-        if (phys < 0 || phys >= lv->n_pages) {
-          atomicOr(&hdr->error, static_cast<int>(RK_DEV_BAD_PAGE));
-        }
+        if (phys < 0 || phys >= lv->n_pages) atomicOr(&lv->error, static_cast<int>(RK_DEV_BAD_PAGE));
         e.phys_page = static_cast<int32_t>(phys);
         e.logical_pos = pos;
         e.delta = start - seg[5 * s + 3];
@@ -125,7 +146,10 @@ __global__ void __launch_bounds__(kSelectThreads)
       }
     }
     const int off = block_exclusive_scan<kSelectThreads>(flag, warp_tot, &s_total);
-    if (flag) vis.entries[estart + count + off] = e;
+    if (flag) {
+      vis.entries[estart + count + off] = e;
+      if (count + off < kPosCap) s_pos[count + off] = make_int2(e.logical_pos, e.n_valid);
+    }
     count += s_total;
     __syncthreads();
   }
@@ -156,171 +180,119 @@ __global__ void __launch_bounds__(kSelectThreads)
     }
     vis.range_start[t] = rstart;
     vis.range_count[t] = n;
-  }
-}
-
-constexpr int kWorklistThreads = 1024;
-constexpr int kCostBuckets = 4096;
-
-__global__ void __launch_bounds__(kWorklistThreads)
-    build_worklist_kernel(LayoutView* lv, rk_visible vis, WsHeader* hdr, Item* items_tmp,
-                          Item* items) {
-  __shared__ int warp_tot[kWorklistThreads / 32];
-  __shared__ int s_total;
-  __shared__ int hist[kCostBuckets];
-  const int hkv = lv->hkv, n_layers = lv->n_layers, P = lv->p;
-  const int n_tables = lv->n_req * n_layers * hkv;
-  const int G = lv->hq / hkv;
-  const int npairs = (G + 1) / 2;
-  const int ept = kKeysPerTile / P;
-  const int W = lv->window;
-  const int T = lv->total_tokens;
-  int32_t* tile_prefix = reinterpret_cast<int32_t*>(lv) + lv->off_tile_prefix;
-  const int32_t* cu = lv_arr(lv, lv->off_cu);
-  const int32_t* cls_arr = lv_arr(lv, lv->off_class);
-
-  // items per table
-  for (int t = threadIdx.x; t < n_tables; t += kWorklistThreads) {
-    const int rs = vis.range_start[t], rn = vis.range_count[t];
-    int tiles = 0;
-    for (int x = 0; x < rn; ++x) {
-      const rk_range rg = vis.ranges[rs + x];
-      tiles += (rg.end - rg.begin + kRowsPerTile - 1) / kRowsPerTile;
-    }
-    tile_prefix[t + 1] = tiles * npairs;
+    s_total = n;
   }
   __syncthreads();
-  // exclusive prefix over tables
-  int carry = 0;
-  for (int base = 0; base < n_tables; base += kWorklistThreads) {
-    const int t = base + threadIdx.x;
-    const int v = t < n_tables ? tile_prefix[t + 1] : 0;
-    const int ex = block_exclusive_scan<kWorklistThreads>(v, warp_tot, &s_total);
-    if (t < n_tables) tile_prefix[t] = carry + ex;
-    carry += s_total;
+
+  // ---- 2. this table's work items
+  if (items_tmp) {
+    const int n_rng = s_total;
+    const int G = lv->hq / hkv;
+    const int npairs = (G + 1) / 2;
+    const int ept = kKeysPerTile / P;
+    const int T = lv->total_tokens;
+    const int first = tile_prefix[t], n_it = tile_prefix[t + 1] - first;
+    const rk_entry* E = vis.entries + estart;
+    const bool in_smem = count <= kPosCap;
+    auto lp = [&](int m) { return in_smem ? s_pos[m].x : E[m].logical_pos; };
+    auto last_key = [&](int m) {
+      return in_smem ? s_pos[m].x + s_pos[m].y - 1 : E[m].logical_pos + E[m].n_valid - 1;
+    };
+    for (int x = threadIdx.x; x < n_it; x += kSelectThreads) {
+      const int pair = x % npairs;
+      int tile = x / npairs;
+      int rbeg = 0, rend = 0;
+      for (int k = 0; k < n_rng; ++k) {
+        const rk_range rg = vis.ranges[rstart + k];
+        const int nt = (rg.end - rg.begin + kRowsPerTile - 1) / kRowsPerTile;
+        if (tile < nt) {
+          rbeg = rg.begin + tile * kRowsPerTile;
+          rend = min(rbeg + kRowsPerTile, rg.end);
+          break;
+        }
+        tile -= nt;
+      }
+      // entries whose first key is at most the tile's last row
+      const int e_hi = upper_bound(count, rend - 1, lp);
+      int e_lo = 0, window = -1;
+      if (cls == RK_LOCAL) {
+        // first entry whose last key reaches the first row's window start
+        window = W;
+        e_lo = upper_bound(e_hi, rbeg - W, last_key);
+      }
+      Item it;
+      it.q_row0 = layer * T + cu[r];
+      it.row_begin = rbeg;
+      it.row_end = rend;
+      it.e_begin = estart + e_lo;
+      it.e_end = estart + e_hi;
+      it.qh0 = kvh * G + 2 * pair;
+      it.nh = min(2, G - 2 * pair);
+      it.window = window;
+      it.layer = layer;
+      it.req = r;
+      it.table = t;
+      it.cost = (e_hi - e_lo + ept - 1) / ept;
+      items_tmp[first + x] = it;
+    }
+  }
+
+  // ---- 3. the last CTA sorts the work list and publishes the header
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = atomicAdd(&lv->done_count, 1) == static_cast<int>(gridDim.x) - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  const int total = items_tmp ? tile_prefix[gridDim.x] : 0;
+  if (items_tmp) {
+    for (int k = threadIdx.x; k < kCostBuckets; k += kSelectThreads) hist[k] = 0;
     __syncthreads();
-  }
-  if (threadIdx.x == 0) tile_prefix[n_tables] = carry;
-  __syncthreads();
-  const int total = carry;
-  if (total > lv->item_capacity) {
-    if (threadIdx.x == 0) {
-      atomicOr(&hdr->error, static_cast<int>(RK_DEV_CAPACITY));
-      hdr->n_items = 0;
-    }
-    return;
-  }
-
-  for (int b = threadIdx.x; b < kCostBuckets; b += kWorklistThreads) hist[b] = 0;
-  __syncthreads();
-
-  for (int x = threadIdx.x; x < total; x += kWorklistThreads) {
-    // table of item x: last t with tile_prefix[t] <= x
-    int lo = 0, hi = n_tables - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (tile_prefix[mid] <= x) lo = mid; else hi = mid - 1;
-    }
-    const int t = lo;
-    const int kvh = t % hkv, layer = (t / hkv) % n_layers, r = t / (hkv * n_layers);
-    const int local = x - tile_prefix[t];
-    const int pair = local % npairs;
-    int tile = local / npairs;
-    const int rs = vis.range_start[t], rn = vis.range_count[t];
-    int rbeg = 0, rend = 0;
-    for (int k = 0; k < rn; ++k) {
-      const rk_range rg = vis.ranges[rs + k];
-      const int nt = (rg.end - rg.begin + kRowsPerTile - 1) / kRowsPerTile;
-      if (tile < nt) {
-        rbeg = rg.begin + tile * kRowsPerTile;
-        rend = min(rbeg + kRowsPerTile, rg.end);
-        break;
-      }
-      tile -= nt;
-    }
-    const int es = vis.entry_start[t], en = vis.entry_count[t];
-    const rk_entry* E = vis.entries + es;
-    // e_hi: first entry whose page starts after the tile's last row
-    int a = 0, b = en;
-    while (a < b) {
-      const int mid = (a + b) >> 1;
-      if (E[mid].logical_pos <= rend - 1) a = mid + 1; else b = mid;
-    }
-    const int e_hi = a;
-    const int cls = cls_arr[layer * hkv + kvh];
-    int e_lo = 0;
-    int window = -1;
-    if (cls == RK_LOCAL) {
-      window = W;
-      // first entry whose last key reaches the first row's window start
-      const int first_key = rbeg - W + 1;
-      a = 0;
-      b = e_hi;
-      while (a < b) {
-        const int mid = (a + b) >> 1;
-        if (E[mid].logical_pos + E[mid].n_valid - 1 < first_key) a = mid + 1; else b = mid;
-      }
-      e_lo = a;
-    }
-    Item it;
-    it.q_row0 = layer * T + cu[r];
-    it.row_begin = rbeg;
-    it.row_end = rend;
-    it.e_begin = es + e_lo;
-    it.e_end = es + e_hi;
-    it.qh0 = kvh * G + 2 * pair;
-    it.nh = min(2, G - 2 * pair);
-    it.window = window;
-    it.layer = layer;
-    it.req = r;
-    it.table = t;
-    it.cost = (e_hi - e_lo + ept - 1) / ept;
-    items_tmp[x] = it;
-    atomicAdd(&hist[kCostBuckets - 1 - min(it.cost, kCostBuckets - 1)], 1);
-  }
-  __syncthreads();
-  // bucket offsets (descending cost order), 4 buckets per thread
-  {
-    constexpr int per = kCostBuckets / kWorklistThreads;
-    int loc[per];
-    int sum = 0;
+    for (int x = threadIdx.x; x < total; x += kSelectThreads)
+      atomicAdd(&hist[kCostBuckets - 1 - min(items_tmp[x].cost, kCostBuckets - 1)], 1);
+    __syncthreads();
+    // bucket offsets in descending cost order, kCostBuckets / kSelectThreads per thread
+    {
+      constexpr int per = kCostBuckets / kSelectThreads;
+      int loc[per];
+      int sum = 0;
 #pragma unroll
-    for (int k = 0; k < per; ++k) {
-      loc[k] = hist[threadIdx.x * per + k];
-      sum += loc[k];
-    }
-    const int ex = block_exclusive_scan<kWorklistThreads>(sum, warp_tot, &s_total);
-    int run = ex;
+      for (int k = 0; k < per; ++k) {
+        loc[k] = hist[threadIdx.x * per + k];
+        sum += loc[k];
+      }
+      const int ex = block_exclusive_scan<kSelectThreads>(sum, warp_tot, &s_total);
+      int run = ex;
 #pragma unroll
-    for (int k = 0; k < per; ++k) {
-      hist[threadIdx.x * per + k] = run;
-      run += loc[k];
+      for (int k = 0; k < per; ++k) {
+        hist[threadIdx.x * per + k] = run;
+        run += loc[k];
+      }
+    }
+    __syncthreads();
+    for (int x = threadIdx.x; x < total; x += kSelectThreads) {
+      const Item it = items_tmp[x];
+      items[atomicAdd(&hist[kCostBuckets - 1 - min(it.cost, kCostBuckets - 1)], 1)] = it;
     }
   }
-  __syncthreads();
-  for (int x = threadIdx.x; x < total; x += kWorklistThreads) {
-    const Item it = items_tmp[x];
-    const int pos = atomicAdd(&hist[kCostBuckets - 1 - min(it.cost, kCostBuckets - 1)], 1);
-    items[pos] = it;
+  if (threadIdx.x == 0) {
+    hdr->n_items = total;
+    hdr->timeout_site = 0;
+    hdr->error = *reinterpret_cast<volatile int*>(&lv->error);
   }
-  if (threadIdx.x == 0) hdr->n_items = total;
 }
 
 cudaError_t launch_select(LayoutView* lv_dev, int n_tables, const rk_visible& vis, WsHeader* hdr,
                           Item* items_tmp, Item* items, cudaStream_t stream) {
-  if (n_tables > 0) {
-    select_tables_kernel<<<n_tables, kSelectThreads, 0, stream>>>(lv_dev, vis, hdr);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
-  build_worklist_kernel<<<1, kWorklistThreads, 0, stream>>>(lv_dev, vis, hdr, items_tmp, items);
+  if (n_tables > 0) select_kernel<<<n_tables, kSelectThreads, 0, stream>>>(lv_dev, vis, hdr, items_tmp, items);
   return cudaGetLastError();
 }
 
 // Page-table stage alone (no work list), for the no-allocation entry point.
 cudaError_t launch_select_tables_only(LayoutView* lv_dev, int n_tables, const rk_visible& vis,
                                       WsHeader* hdr, cudaStream_t stream) {
-  if (n_tables > 0) select_tables_kernel<<<n_tables, kSelectThreads, 0, stream>>>(lv_dev, vis, hdr);
+  if (n_tables > 0)
+    select_kernel<<<n_tables, kSelectThreads, 0, stream>>>(lv_dev, vis, hdr, nullptr, nullptr);
   return cudaGetLastError();
 }
 
