@@ -110,6 +110,34 @@ def test_prefill_full_size_sampled(name, per_table):
         torch.cuda.empty_cache()
 
 
+def _many_items_odd_group():
+    """GQA group of 3 (work items alternate between two q heads and one) and
+    enough rows that every CTA runs several items of both kinds in a row: the
+    four global / dense kv heads alone give 4 x 108 row tiles x 2 head pairs."""
+    segs = [(f"c{i}", 2048, 0, True) for i in range(6)] + [("tail", 1536, 0, False)]
+    lay = synth._make_layout(n_layers=1, hq=24, hkv=8, d=128, p=64, theta=1e6,
+                             requests=[segs], class_map=[0, 1, 0, 1, 3, 1, 0, 1], window=1024)
+    return synth.Workload("odd_group_L13824", 21, lay, "cuda")
+
+
+def test_prefill_many_items_odd_group():
+    wl = _many_items_odd_group()
+    lay = wl.layout
+    q, k, v = wl.materialize("cuda")
+    rows = sample_rows(lay, 12, seed=5)
+    o_ref, lse_ref, comp = oracle_rows(lay, q, k.cpu(), v.cpu(), rows)
+    assert comp.all()
+    for mode in MODES:
+        run = PrefillRun(lay, q, k, v, mode=mode)
+        assert run.status == 0, f"{mode}: device status {run.status}"
+        o_got, lse_got = gpu_rows(run, rows)
+        assert_close(o_got, o_ref, f"odd group {mode} o")
+        assert np.abs(lse_got - lse_ref).max() <= 1e-2, f"odd group {mode} lse"
+        _untouched(lay, run)
+        del run
+        torch.cuda.empty_cache()
+
+
 @pytest.mark.parametrize("mode", MODES)
 def test_prefill_deterministic(mode):
     wl = synth.cfg3()
