@@ -61,6 +61,9 @@ class SegPagedPrefill:
         self.dev_err = torch.zeros(1, dtype=torch.int32, device=self.device)
         self.jobs_k = torch.from_numpy(self.plan.jobs_k).to(self.device)
         self.jobs_v = torch.from_numpy(self.plan.jobs_v).to(self.device)
+        # relocation and selection are independent: the relocation runs on a
+        # side stream that the attention launch waits for
+        self.side = torch.cuda.Stream(self.device) if mode == "relocate" else None
 
     def _plan(self, layout) -> RelocationPlan:
         """Page tables of the original layout (built by the library on the
@@ -98,19 +101,24 @@ class SegPagedPrefill:
         """Runs relocation, selection and attention on the loaded inputs.
         k3_events: optional (start, end) CUDA events recorded around the
         attention kernel on the launching stream."""
-        if self.plan.jobs_k.shape[0]:
-            binding.relocate_rope(self.k_store, self.k_work, self.jobs_k, self.layout.theta,
-                                  self.dev_err, stream)
-        if self.plan.jobs_v.shape[0]:
-            binding.relocate_rope(self.v_work, self.v_work, self.jobs_v, self.layout.theta,
-                                  self.dev_err, stream)
-        binding.select_visible(self.hl, self.vis, self.ws, stream)
         s = stream if stream is not None else torch.cuda.current_stream()
+        relocating = self.plan.jobs_k.shape[0] > 0 or self.plan.jobs_v.shape[0] > 0
+        if relocating:
+            self.side.wait_stream(s)
+            if self.plan.jobs_k.shape[0]:
+                binding.relocate_rope(self.k_store, self.k_work, self.jobs_k, self.layout.theta,
+                                      self.dev_err, self.side)
+            if self.plan.jobs_v.shape[0]:
+                binding.relocate_rope(self.v_work, self.v_work, self.jobs_v, self.layout.theta,
+                                      self.dev_err, self.side)
+        binding.select_visible(self.hl, self.vis, self.ws, s)
+        if relocating:
+            s.wait_stream(self.side)
         if k3_events is not None:
             k3_events[0].record(s)
         binding.segpaged_prefill(self.hl, self.q_dev, self.k_work, self.v_work, self.vis,
                                  self.ws, self.o, self.lse, fuse_rope=self.mode == "fused",
-                                 stream=stream)
+                                 stream=s)
         if k3_events is not None:
             k3_events[1].record(s)
 
