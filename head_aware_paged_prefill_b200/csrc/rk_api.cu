@@ -363,6 +363,8 @@ extern "C" rk_status rk_segpaged_prefill(const rk_dims* dims, const void* q, con
   a.total_tokens = dims->total_tokens;
   a.items = reinterpret_cast<const Item*>(ws + sizeof(WsHeader));
   a.n_items = &hdr->n_items;
+  a.work_next = &hdr->work_next;
+  a.work_done = &hdr->work_done;
   a.error_word = &hdr->error;
   a.timeout_site = &hdr->timeout_site;
   a.entries = vis->entries;

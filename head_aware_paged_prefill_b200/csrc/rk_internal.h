@@ -19,7 +19,9 @@ struct WsHeader {
   int32_t n_tables;
   int32_t item_capacity;
   int32_t timeout_site;   // first bounded wait that gave up (diagnostics)
-  int32_t pad[59];
+  int32_t work_next;      // attention: next work item to hand out (dynamic schedule)
+  int32_t work_done;      // attention: CTAs finished (the last one resets both)
+  int32_t pad[57];
 };
 static_assert(sizeof(WsHeader) == 256, "header size");
 
@@ -86,6 +88,8 @@ struct PrefillLaunchArgs {
   int total_tokens;
   const Item* items;
   const int32_t* n_items;
+  int* work_next;
+  int* work_done;
   int* error_word;
   int* timeout_site;
   const rk_entry* entries;

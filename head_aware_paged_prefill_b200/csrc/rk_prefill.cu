@@ -79,6 +79,8 @@ struct PrefillCfg {
 struct PrefillParams {
   const Item* items;
   const int32_t* n_items;
+  int* work_next;  // next item of the cost-sorted list to hand out
+  int* work_done;  // CTAs finished
   int* error_word;
   int* timeout_site;
   const rk_entry* entries;
@@ -107,7 +109,9 @@ enum : int {
   kBarQFree = 17,    // fused: every S reading the current Q rotation completed
   kBarQReload = 18,  // fused: original Q re-fetched for a new rotation
   kBarTurn = 19,   // [2] softmax exponential phases take turns (two-head items)
-  kBarKFull = 21,  // k_full, k_ready, k_empty [kKStages] each, then v_full, v_empty [kVStages]
+  kBarItemFull = 21,   // [2] ring of work-item indices: slot written by the producer
+  kBarItemEmpty = 23,  // [2] slot read by every other role
+  kBarKFull = 25,  // k_full, k_ready, k_empty [kKStages] each, then v_full, v_empty [kVStages]
 };
 
 // kEmuNum pairs of exponentials in every kEmuDen can go through the FMA-pipe
@@ -128,9 +132,16 @@ constexpr int kEmuNum = RK_EMU_NUM;
 constexpr int kTurnAt = RK_TURN_AT;  // exponential pairs of the last half before the turn passes
 constexpr int kEmuDen = RK_EMU_DEN;
 
-// Item of round r for CTA b (boustrophedon over the cost-sorted list).
-__device__ __forceinline__ int item_of_round(int r, int b, int g) {
-  return r * g + ((r & 1) ? (g - 1 - b) : b);
+// Index of the r-th work item of this CTA, from the producer's two-slot ring
+// (-1 once the list is exhausted).  Every thread of a consuming role reads
+// the slot and arrives on its empty barrier.
+__device__ __forceinline__ int next_item(uint64_t* bars, const volatile int* s_item, uint32_t r,
+                                         const WaitCtx& wc, int site, bool& ok) {
+  const int slot = r & 1;
+  if (!(ok = mbar_wait(&bars[kBarItemFull + slot], (r >> 1) & 1, wc, site))) return -1;
+  const int it = s_item[slot];
+  mbar_arrive(&bars[kBarItemEmpty + slot]);
+  return it;
 }
 
 // cos / sin of delta * f_m for the 8 frequencies m = 8c .. 8c+7 a thread
@@ -221,6 +232,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   uint64_t* v_empty = v_full + SV;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 64);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  volatile int* s_item = reinterpret_cast<volatile int*>(tmem_slot + 2);  // [2]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool fuse = prm.fuse_rope != 0;
@@ -236,6 +248,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     mbar_init(&bars[kBarQFree], 2);
     mbar_init(&bars[kBarQReload], 1);
     for (int t = 0; t < 2; ++t) {
+      mbar_init(&bars[kBarItemFull + t], 1);
+      // readers of a slot: both issuers, the RoPE warp when it runs, both
+      // softmax warpgroups
+      mbar_init(&bars[kBarItemEmpty + t], 2 + (fuse ? 32 : 0) + 256);
       mbar_init(&bars[kBarSFree + t], 128);
       mbar_init(&bars[kBarTurn + t], 128);
       mbar_init(&bars[kBarSFull + t], 1);
@@ -270,7 +286,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int n_items = *prm.n_items;
-  const int G = gridDim.x, b = blockIdx.x;
   const WaitCtx wc{abort_flag, prm.error_word, prm.timeout_site};
 
   if (warp < 4) {
@@ -283,9 +298,18 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       uint32_t k_issued = 0, v_issued = 0, q_uses = 0;
       bool ok = true;
       const int32_t oob_row = static_cast<int32_t>(prm.n_pages * P);
-      for (int r = 0; ok; ++r) {
-        const int it = item_of_round(r, b, G);
-        if (it >= n_items) break;
+      // items are handed out dynamically, longest first: every CTA takes the
+      // next item of the cost-sorted list when it is ready for one (greedy
+      // longest-processing-time scheduling)
+      for (uint32_t r = 0; ok; ++r) {
+        const int slot = r & 1;
+        if (r >= 2 && !(ok = mbar_wait(&bars[kBarItemEmpty + slot], ((r >> 1) - 1) & 1, wc, 4)))
+          break;
+        const int got = atomicAdd(prm.work_next, 1);
+        const int it = got < n_items ? got : -1;
+        s_item[slot] = it;
+        mbar_arrive(&bars[kBarItemFull + slot]);
+        if (it < 0) break;
         const Item w = prm.items[it];
         const int n_tiles = (w.e_end - w.e_begin + C::EPT - 1) / C::EPT;
         if (n_tiles == 0) continue;
@@ -401,9 +425,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
         tc_commit(&bars[kBarPVDone + t]);
       };
-      for (int r = 0; ok; ++r) {
-        const int it = item_of_round(r, b, G);
-        if (it >= n_items) break;
+      for (uint32_t r = 0; ok; ++r) {
+        const int it = next_item(bars, s_item, r, wc, 5, ok);
+        if (it < 0) break;
         const Item w = prm.items[it];
         const int n_tiles = (w.e_end - w.e_begin + C::EPT - 1) / C::EPT;
         if (n_tiles == 0) continue;
@@ -504,9 +528,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
       };
       bool ok = true;
-      for (int r = 0; ok; ++r) {
-        const int it = item_of_round(r, b, G);
-        if (it >= n_items) break;
+      for (uint32_t r = 0; ok; ++r) {
+        const int it = next_item(bars, s_item, r, wc, 5, ok);
+        if (it < 0) break;
         const Item w = prm.items[it];
         const int n_tiles = (w.e_end - w.e_begin + C::EPT - 1) / C::EPT;
         if (n_tiles == 0) continue;
@@ -579,9 +603,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     uint32_t s_phase = 0, o_uses = 0, turn_phase = 0;
     uint32_t n_pv = 0;  // PVs of this Q tile issued before the current tile
     bool ok = true;
-    for (int r = 0; ok; ++r) {
-      const int it = item_of_round(r, b, G);
-      if (it >= n_items) break;
+    for (uint32_t r = 0; ok; ++r) {
+      const int it = next_item(bars, s_item, r, wc, 6, ok);
+      if (it < 0) break;
       const Item w = prm.items[it];
       if (t >= w.nh) continue;
       const int n_tiles = (w.e_end - w.e_begin + C::EPT - 1) / C::EPT;
@@ -766,6 +790,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  // the last CTA to finish leaves the work counter at 0 for the next launch
+  if (threadIdx.x == 0 && atomicAdd(prm.work_done, 1) == static_cast<int>(gridDim.x) - 1) {
+    *prm.work_next = 0;
+    *prm.work_done = 0;
+  }
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
@@ -833,6 +862,8 @@ static cudaError_t launch_typed(const PrefillLaunchArgs& a, cudaStream_t stream)
   PrefillParams prm;
   prm.items = a.items;
   prm.n_items = a.n_items;
+  prm.work_next = a.work_next;
+  prm.work_done = a.work_done;
   prm.error_word = a.error_word;
   prm.timeout_site = a.timeout_site;
   prm.entries = a.entries;

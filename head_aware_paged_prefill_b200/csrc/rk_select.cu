@@ -278,6 +278,8 @@ __global__ void __launch_bounds__(kSelectThreads)
   if (threadIdx.x == 0) {
     hdr->n_items = total;
     hdr->timeout_site = 0;
+    hdr->work_next = 0;
+    hdr->work_done = 0;
     hdr->error = *reinterpret_cast<volatile int*>(&lv->error);
   }
 }
