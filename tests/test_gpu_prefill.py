@@ -147,6 +147,24 @@ def test_prefill_deterministic(mode):
     assert torch.equal(a.o.view(torch.int16), b.o.view(torch.int16))
 
 
+def test_prefill_repeated_on_one_selection():
+    """Work items are handed out from a counter in the workspace: three
+    attention launches on one selection must each cover every item (the
+    last CTA of a launch resets the counter for the next), bit-identically."""
+    from head_aware_paged_prefill_b200 import binding
+    wl = synth.cfg2()
+    q, k, v = wl.materialize("cuda")
+    run = PrefillRun(wl.layout, q, k, v, mode="relocate")
+    assert run.status == 0
+    first = run.o.clone()
+    for _ in range(2):
+        run.o.view(torch.int16).fill_(SENTINEL)
+        binding.segpaged_prefill(run.hl, q, run.k_rel, run.v_rel, run.vis, run.ws, run.o, run.lse)
+        torch.cuda.synchronize()
+        assert binding.device_status(run.ws) == 0
+        assert torch.equal(run.o.view(torch.int16), first.view(torch.int16))
+
+
 def test_prefill_reports_bad_page_without_faulting():
     """A page id outside the pool (corrupted after selection) is skipped by the
     kernel (the tile loads zeros) and reported through the error word."""
