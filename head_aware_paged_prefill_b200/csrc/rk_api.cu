@@ -14,7 +14,7 @@
 namespace rk {
 
 cudaError_t launch_select(LayoutView* lv_dev, int n_tables, const rk_visible& vis, WsHeader* hdr,
-                          Item* items_tmp, Item* items, cudaStream_t stream);
+                          Item* items_tmp, Item* items, int32_t* cursor, cudaStream_t stream);
 cudaError_t launch_relocate(const void* k_src, void* k_dst, const int32_t* jobs, int n_jobs,
                             int64_t n_src_pages, int64_t n_dst_pages, int P, int D, double theta,
                             int* device_error, cudaStream_t stream);
@@ -148,14 +148,15 @@ rk_status check_layout(const rk_dims* d, const rk_layout* lay, Derived* out) {
   const int64_t words_fixed = (sizeof(LayoutView) + 3) / 4;
   const int64_t words = words_fixed + 5 * static_cast<int64_t>(lay->n_segments) + (n_req + 1) +
                         lay->n_segments * n_lh + (n_req + 1) + (n_req + 1) + n_lh +
-                        (out->n_tables + 1) + out->n_retr + (out->n_tables + 1) + 8;
+                        (out->n_tables + 1) + out->n_retr + (out->n_tables + 1) + kCostBuckets + 8;
   if (words >= kMaxI32) return RK_ERR_INVALID_ARG;
   out->layout_words = static_cast<int32_t>(words);
   WsMap& m = out->map;
   m.header = 0;
   m.items = sizeof(WsHeader);
   m.items_tmp = align_up(m.items + sizeof(Item) * out->item_capacity, 256);
-  m.layout = align_up(m.items_tmp + sizeof(Item) * out->item_capacity, 256);
+  m.cursor = align_up(m.items_tmp + sizeof(Item) * out->item_capacity, 256);
+  m.layout = align_up(m.cursor + 4 * static_cast<size_t>(kCostBuckets), 256);
   m.total = align_up(m.layout + 4 * static_cast<size_t>(words), 256);
   return RK_OK;
 }
@@ -257,6 +258,8 @@ void build_layout_image(const rk_dims* d, const rk_layout* lay, const Derived& d
     w[off + dv.n_tables] = static_cast<int32_t>(acc);
   }
   off += static_cast<int32_t>(dv.n_tables + 1);
+  v.off_cost_hist = off;  // zero: the select kernel's CTAs add their items' costs
+  off += kCostBuckets;
   v.layout_words = off;
   std::memcpy(w, &v, sizeof(LayoutView));
 }
@@ -310,7 +313,8 @@ extern "C" rk_status rk_select_visible(const rk_dims* dims, const rk_layout* lay
                                 static_cast<int>(dv.n_tables), *out,
                                 reinterpret_cast<WsHeader*>(ws),
                                 reinterpret_cast<Item*>(ws + dv.map.items_tmp),
-                                reinterpret_cast<Item*>(ws + dv.map.items), s);
+                                reinterpret_cast<Item*>(ws + dv.map.items),
+                                reinterpret_cast<int32_t*>(ws + dv.map.cursor), s);
   return e == cudaSuccess ? RK_OK : RK_ERR_CUDA;
 }
 

@@ -11,6 +11,9 @@ namespace rk {
 
 constexpr int kRowsPerTile = 128;  // query rows per Q tile (one TMEM lane per row)
 constexpr int kKeysPerTile = 128;  // keys per KV tile (N of the QK^T MMA)
+// Work items are ordered by cost (KV tiles) in this many buckets, longest
+// first; costs past the last bucket (over 256K keys) share it.
+constexpr int kCostBuckets = 2048;
 
 // Workspace header (first 256 bytes of the workspace).
 struct WsHeader {
@@ -64,6 +67,7 @@ struct LayoutView {
   int32_t off_retr_indptr;  // [n_tables + 1]
   int32_t off_retr_pages;   // [n_retr]
   int32_t off_tile_prefix;  // [n_tables + 1] exclusive prefix of the work items per table
+  int32_t off_cost_hist;    // [kCostBuckets] items per cost bucket (uploaded as zero)
   int32_t layout_words;
 };
 
@@ -72,6 +76,7 @@ struct WsMap {
   size_t header = 0;
   size_t items = 0;      // Item[item_capacity], sorted by cost (longest first)
   size_t items_tmp = 0;  // Item[item_capacity], unsorted
+  size_t cursor = 0;     // int32[kCostBuckets]: next sorted slot of each cost bucket
   size_t layout = 0;     // LayoutView followed by the int32 arrays
   size_t total = 0;
 };

@@ -223,8 +223,9 @@ rk_status rk_selftest_bounded_wait(int32_t* device_word, int32_t wait_ms, void* 
  *     __device__ array, held by every GPU that loads the library until the
  *     process exits) holds the device copy of the layout and the error word.
  *     A layout whose copy does not fit (4 bytes per word of segments,
- *     page_base, cu_seqlens, class map and retrieval lists, plus 256 bytes)
- *     is rejected with RK_ERR_CAPACITY before any GPU work.
+ *     page_base, cu_seqlens, class map, retrieval lists and per-table work
+ *     item offsets, plus about 8.5 KB of fixed fields) is rejected with
+ *     RK_ERR_CAPACITY before any GPU work.
  *   - The first call on a device looks up the scratch's device address with
  *     that device current; make that first call before any stream capture.
  *   - Every call shares the one scratch array and rewrites all of it that it
