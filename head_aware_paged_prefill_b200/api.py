@@ -16,6 +16,9 @@ C-ABI calls on the current CUDA stream.  Two modes:
 
 Inputs may live on the host (pinned tensors are copied asynchronously) or on
 the device; ``run(..., out="host")`` returns o on the host.
+``run_host_pipelined`` runs a sequence of host-resident steps with the copies
+of one step overlapping the computation of its neighbours (two device buffer
+sets, a copy-in, a compute and a copy-out stream).
 """
 from __future__ import annotations
 
@@ -47,15 +50,9 @@ class SegPagedPrefill:
         self.vis = binding.Visible(self.sizes, self.device)
         self.ws = binding.workspace(self.sizes, self.device)
         self.n_extra = self.plan.n_extra
-        shape = (lay.n_pages + self.n_extra, lay.p, lay.d)
-        self.k_work = torch.empty(shape, dtype=torch.bfloat16, device=self.device)
-        self.v_work = torch.empty(shape, dtype=torch.bfloat16, device=self.device)
-        # the K store (pages as written) is the relocation's source
-        self.k_store = (torch.empty((lay.n_pages, lay.p, lay.d), dtype=torch.bfloat16,
-                                    device=self.device) if mode == "relocate" else None)
-        self.q_dev = torch.empty((lay.n_layers, lay.total_tokens, lay.hq, lay.d),
-                                 dtype=torch.bfloat16, device=self.device)
-        self.o = torch.empty_like(self.q_dev)
+        self._sets = [self._buffers()]
+        self.k_work, self.v_work = self._sets[0]["k_work"], self._sets[0]["v_work"]
+        self.k_store, self.q_dev, self.o = (self._sets[0][n] for n in ("k_store", "q", "o"))
         self.lse = (torch.empty((lay.n_layers, lay.hq, lay.total_tokens), dtype=torch.float32,
                                 device=self.device) if with_lse else None)
         self.dev_err = torch.zeros(1, dtype=torch.int32, device=self.device)
@@ -64,6 +61,21 @@ class SegPagedPrefill:
         # relocation and selection are independent: the relocation runs on a
         # side stream that the attention launch waits for
         self.side = torch.cuda.Stream(self.device) if mode == "relocate" else None
+
+    def _buffers(self) -> dict:
+        """One set of device buffers a step reads and writes."""
+        lay, dev, bf = self.layout, self.device, torch.bfloat16
+        shape = (lay.n_pages + self.n_extra, lay.p, lay.d)
+        q = torch.empty((lay.n_layers, lay.total_tokens, lay.hq, lay.d), dtype=bf, device=dev)
+        return {
+            "q": q,
+            "o": torch.empty_like(q),
+            "k_work": torch.empty(shape, dtype=bf, device=dev),
+            "v_work": torch.empty(shape, dtype=bf, device=dev),
+            # the K store (pages as written) is the relocation's source
+            "k_store": (torch.empty((lay.n_pages, lay.p, lay.d), dtype=bf, device=dev)
+                        if self.mode == "relocate" else None),
+        }
 
     def _plan(self, layout) -> RelocationPlan:
         """Page tables of the original layout (built by the library on the
@@ -86,38 +98,49 @@ class SegPagedPrefill:
         # select (one kernel) + attention, plus the relocation launches
         return 2 + int(self.plan.jobs_k.shape[0] > 0) + int(self.plan.jobs_v.shape[0] > 0)
 
+    def _copy_in(self, b: dict, q, k_pool, v_pool):
+        """Copies a step's inputs (host or device) into buffer set b on the
+        current stream; the K store copy into the working K pool is left to
+        the step's computation."""
+        n = self.layout.n_pages
+        b["q"].copy_(q, non_blocking=True)
+        if b["k_store"] is not None:
+            b["k_store"].copy_(k_pool, non_blocking=True)
+        else:
+            b["k_work"][:n].copy_(k_pool, non_blocking=True)
+        b["v_work"][:n].copy_(v_pool, non_blocking=True)
+
     def load(self, q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor):
         """Copies inputs (host or device) into the device working buffers."""
-        n = self.layout.n_pages
-        self.q_dev.copy_(q, non_blocking=True)
-        if self.k_store is not None:
-            self.k_store.copy_(k_pool, non_blocking=True)
-            self.k_work[:n].copy_(self.k_store)
-        else:
-            self.k_work[:n].copy_(k_pool, non_blocking=True)
-        self.v_work[:n].copy_(v_pool, non_blocking=True)
+        b = self._sets[0]
+        self._copy_in(b, q, k_pool, v_pool)
+        if b["k_store"] is not None:
+            b["k_work"][:self.layout.n_pages].copy_(b["k_store"])
 
     def compute(self, stream=None, k3_events=None):
         """Runs relocation, selection and attention on the loaded inputs.
         k3_events: optional (start, end) CUDA events recorded around the
         attention kernel on the launching stream."""
+        self._compute(self._sets[0], stream, k3_events)
+
+    def _compute(self, b: dict, stream=None, k3_events=None):
         s = stream if stream is not None else torch.cuda.current_stream()
         relocating = self.plan.jobs_k.shape[0] > 0 or self.plan.jobs_v.shape[0] > 0
         if relocating:
             self.side.wait_stream(s)
             if self.plan.jobs_k.shape[0]:
-                binding.relocate_rope(self.k_store, self.k_work, self.jobs_k, self.layout.theta,
+                binding.relocate_rope(b["k_store"], b["k_work"], self.jobs_k, self.layout.theta,
                                       self.dev_err, self.side)
             if self.plan.jobs_v.shape[0]:
-                binding.relocate_rope(self.v_work, self.v_work, self.jobs_v, self.layout.theta,
+                binding.relocate_rope(b["v_work"], b["v_work"], self.jobs_v, self.layout.theta,
                                       self.dev_err, self.side)
         binding.select_visible(self.hl, self.vis, self.ws, s)
         if relocating:
             s.wait_stream(self.side)
         if k3_events is not None:
             k3_events[0].record(s)
-        binding.segpaged_prefill(self.hl, self.q_dev, self.k_work, self.v_work, self.vis,
-                                 self.ws, self.o, self.lse, fuse_rope=self.mode == "fused",
+        binding.segpaged_prefill(self.hl, b["q"], b["k_work"], b["v_work"], self.vis,
+                                 self.ws, b["o"], self.lse, fuse_rope=self.mode == "fused",
                                  stream=s)
         if k3_events is not None:
             k3_events[1].record(s)
@@ -131,6 +154,60 @@ class SegPagedPrefill:
             dst.copy_(self.o, non_blocking=True)
             return dst
         return self.o
+
+    def run_host_pipelined(self, inputs, outs, stream=None):
+        """Runs one step per entry of ``inputs`` ((q, k_pool, v_pool), pinned
+        host tensors) and copies each step's o into the pinned host tensor at
+        the same index of ``outs``.
+
+        Step n's inputs cross to the device on a copy-in stream and its o
+        comes back on a copy-out stream, each step in one of two device buffer
+        sets, so the copies of steps n + 1 and n - 1 overlap step n's
+        relocation, selection and attention on ``stream`` (default: the
+        current stream).  Every step waits for its own inputs; a buffer set is
+        refilled only after the step that last read it, and its o rewritten
+        only after that o reached the host.  Returns once all work is queued;
+        ``stream`` is ordered after the last copy out."""
+        if len(inputs) != len(outs):
+            raise ValueError("one output per step")
+        s = stream if stream is not None else torch.cuda.current_stream()
+        while len(self._sets) < 2:
+            self._sets.append(self._buffers())
+        if not hasattr(self, "_cp_in"):
+            self._cp_in = torch.cuda.Stream(self.device)
+            self._cp_out = torch.cuda.Stream(self.device)
+        n = self.layout.n_pages
+        consumed = [None, None]  # compute of the step that last read set i
+        drained = [None, None]   # copy out of the o last written in set i
+        self._cp_in.wait_stream(s)
+        self._cp_out.wait_stream(s)
+        for step, ((q, k_pool, v_pool), dst) in enumerate(zip(inputs, outs)):
+            i = step % 2
+            b = self._sets[i]
+            with torch.cuda.stream(self._cp_in):
+                if consumed[i] is not None:
+                    self._cp_in.wait_event(consumed[i])
+                self._copy_in(b, q, k_pool, v_pool)
+                loaded = torch.cuda.Event()
+                loaded.record(self._cp_in)
+            s.wait_event(loaded)
+            if drained[i] is not None:
+                s.wait_event(drained[i])
+            with torch.cuda.stream(s):
+                if b["k_store"] is not None:
+                    b["k_work"][:n].copy_(b["k_store"])
+            self._compute(b, s)
+            done = torch.cuda.Event()
+            done.record(s)
+            consumed[i] = done
+            with torch.cuda.stream(self._cp_out):
+                self._cp_out.wait_event(done)
+                dst.copy_(b["o"], non_blocking=True)
+                out_done = torch.cuda.Event()
+                out_done.record(self._cp_out)
+            drained[i] = out_done
+        s.wait_stream(self._cp_out)
+        s.wait_stream(self._cp_in)
 
     def status(self) -> int:
         """Device error bits of the last run (synchronises the stream)."""
