@@ -31,9 +31,9 @@
 //               TMEM lane (= one query row) per thread; online softmax in the
 //               log2 domain, O rescaled in TMEM only when the running max
 //               grows by more than 2^8 (after the previous PV completed), P
-//               stored as bf16 in 16-column quarters.  The two warpgroups' exponential phases
-//               take turns (a pair of mbarriers), so they never compete for
-//               the MUFU while their other phases overlap.
+//               stored as bf16 in 16-column quarters.  The two warpgroups
+//               run free: their exponential phases overlap wherever their
+//               dependencies allow (taking turns on the MUFU was slower).
 // Registers are rebalanced with setmaxnreg: the first warpgroup keeps 80 per
 // thread, the two softmax warpgroups get 208.
 //
@@ -108,7 +108,7 @@ enum : int {
   kBarQReady = 16,   // fused: the Q tiles hold the rotation the next S needs
   kBarQFree = 17,    // fused: every S reading the current Q rotation completed
   kBarQReload = 18,  // fused: original Q re-fetched for a new rotation
-  kBarTurn = 19,   // [2] softmax exponential phases take turns (two-head items)
+  // 19, 20 unused
   kBarItemFull = 21,   // [2] ring of work-item indices: slot written by the producer
   kBarItemEmpty = 23,  // [2] slot read by every other role
   kBarKFull = 25,  // k_full, k_ready, k_empty [kKStages] each, then v_full, v_empty [kVStages]
@@ -116,9 +116,9 @@ enum : int {
 
 // kEmuNum pairs of exponentials in every kEmuDen can go through the FMA-pipe
 // polynomial instead of the MUFU (16 ex2 per clock per SM).  Measured on
-// B200 at D = 128 the softmax is latency bound rather than MUFU bound, and
-// every emulated fraction tried (1/4, 3/8, 1/2) was slower, so the default
-// keeps all exponentials on the MUFU.
+// B200 at D = 128, FP32 work on a sub-partition slows that sub-partition's
+// MUFU, and every emulated fraction tried (1/8 to 5/8) was slower, so the
+// default keeps all exponentials on the MUFU.
 #ifndef RK_EMU_NUM
 #define RK_EMU_NUM 0
 #endif
@@ -126,10 +126,6 @@ enum : int {
 #define RK_EMU_DEN 4
 #endif
 constexpr int kEmuNum = RK_EMU_NUM;
-#ifndef RK_TURN_AT
-#define RK_TURN_AT 16
-#endif
-constexpr int kTurnAt = RK_TURN_AT;  // exponential pairs of the last half before the turn passes
 constexpr int kEmuDen = RK_EMU_DEN;
 
 // Index of the r-th work item of this CTA, from the producer's two-slot ring
@@ -253,7 +249,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       // softmax warpgroups
       mbar_init(&bars[kBarItemEmpty + t], 2 + (fuse ? 32 : 0) + 256);
       mbar_init(&bars[kBarSFree + t], 128);
-      mbar_init(&bars[kBarTurn + t], 128);
       mbar_init(&bars[kBarSFull + t], 1);
       mbar_init(&bars[kBarP + t], 128);
       mbar_init(&bars[kBarPVDone + t], 1);
@@ -600,7 +595,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const uint32_t tO = tmem + lane_base + C::col_o(t);
     const float sl2 = prm.scale_log2;
     const int T = prm.total_tokens;
-    uint32_t s_phase = 0, o_uses = 0, turn_phase = 0;
+    uint32_t s_phase = 0, o_uses = 0;
     uint32_t n_pv = 0;  // PVs of this Q tile issued before the current tile
     bool ok = true;
     for (uint32_t r = 0; ok; ++r) {
@@ -625,8 +620,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       }
       const int window = w.window;
       float m_ref = -INFINITY, l = 0.f;
-      // tile 0's warpgroup goes first in every two-head item
-      if (w.nh == 2 && t == 1) mbar_arrive(&bars[kBarTurn]);
       for (int j = 0; j < n_tiles && ok; ++j) {
         // pages of this tile (loaded before the wait, so their latency hides)
         int lp[C::EPT], nv[C::EPT];
@@ -696,16 +689,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
         if (resc) m_ref = m_new;
         const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
-        // P_t still feeds the previous PV until that completes; waited here,
-        // while the other warpgroup has the turn (every phase of the barrier
-        // is waited, across items too, so none is skipped)
+        // P_t still feeds the previous PV until that completes (every phase
+        // of the barrier is waited, across items too, so none is skipped)
         if (n_pv > 0) {
           if (!(ok = mbar_wait(&bars[kBarPVDone + t], (n_pv - 1) & 1, wc, 24))) break;
           tc_fence_after();
         }
-        // two-head items: the two warpgroups' exponential phases alternate
-        // (tile 0's first), so they never compete for the MUFU and issue slots
-        if (w.nh == 2 && !(ok = mbar_wait(&bars[kBarTurn + t], turn_phase, wc, 22))) break;
         const uint64_t scale2 = f2_pack(sl2, sl2);
         const uint64_t neg_m2 = f2_pack(-m_use, -m_use);
         uint64_t acc2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
@@ -719,24 +708,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           }
 #pragma unroll
           for (int k = 0; k < 32; ++k) {
-            // the other warpgroup's turn once kTurnAt pairs of the last half
-            // are issued: its wake-up overlaps this one's remaining
-            // exponentials, packing and P stores (tile 1 hands back after
-            // every tile but the item's last)
-            if (half == 1 && k == kTurnAt && w.nh == 2) {
-              turn_phase ^= 1;
-              if (t == 0 || j + 1 < n_tiles) mbar_arrive(&bars[kBarTurn + (1 - t)]);
-            }
             if (k % kEmuDen >= kEmuDen - kEmuNum) {
               exp2_poly_pair(sh[2 * k], sh[2 * k + 1], sh[2 * k], sh[2 * k + 1]);
             } else {
               sh[2 * k] = ex2_approx(sh[2 * k]);
               sh[2 * k + 1] = ex2_approx(sh[2 * k + 1]);
             }
-          }
-          if (half == 1 && kTurnAt >= 32 && w.nh == 2) {
-            turn_phase ^= 1;
-            if (t == 0 || j + 1 < n_tiles) mbar_arrive(&bars[kBarTurn + (1 - t)]);
           }
 #pragma unroll
           for (int q = 0; q < 2; ++q) {
