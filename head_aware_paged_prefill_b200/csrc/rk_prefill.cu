@@ -689,12 +689,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
         if (resc) m_ref = m_new;
         const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
-        // P_t still feeds the previous PV until that completes (every phase
-        // of the barrier is waited, across items too, so none is skipped)
-        if (n_pv > 0) {
-          if (!(ok = mbar_wait(&bars[kBarPVDone + t], (n_pv - 1) & 1, wc, 24))) break;
-          tc_fence_after();
-        }
         const uint64_t scale2 = f2_pack(sl2, sl2);
         const uint64_t neg_m2 = f2_pack(-m_use, -m_use);
         uint64_t acc2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
@@ -716,12 +710,25 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             }
           }
 #pragma unroll
+          for (int k = 0; k < 32; ++k)
+            acc2[k & 1] = f2_add(acc2[k & 1], f2_pack(sh[2 * k], sh[2 * k + 1]));
+        }
+        // P_t still feeds the previous PV until that completes: waited only
+        // now, so the exponentials overlap that PV (every phase of the
+        // barrier is waited, across items too, so none is skipped)
+        if (n_pv > 0) {
+          if (!(ok = mbar_wait(&bars[kBarPVDone + t], (n_pv - 1) & 1, wc, 24))) break;
+          tc_fence_after();
+        }
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const float* sh = s + 64 * half;
+#pragma unroll
           for (int q = 0; q < 2; ++q) {
             uint32_t pk[16];
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
               const int kk = 16 * q + k;
-              acc2[k & 1] = f2_add(acc2[k & 1], f2_pack(sh[2 * kk], sh[2 * kk + 1]));
               pk[k] = pack_bf16x2(sh[2 * kk], sh[2 * kk + 1]);
             }
             tmem_st_x16(tP + 32 * half + 16 * q, pk);
