@@ -315,11 +315,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             tma_load_3d(sQ + t * C::kQTileBytes + cb * C::kBlockBytes, &tm_q, &bars[kBarQFull],
                         cb * 64, w.qh0 + t, w.q_row0 + w.row_begin);
         ++q_uses;
-        for (int j = 0; j < n_tiles; ++j) {
-          int32_t rows[C::EPT];
+        auto tile_rows = [&](int jt, int32_t (&rows)[C::EPT]) {
 #pragma unroll
           for (int e = 0; e < C::EPT; ++e) {
-            const int idx = w.e_begin + j * C::EPT + e;
+            const int idx = w.e_begin + jt * C::EPT + e;
             rows[e] = oob_row;
             if (idx < w.e_end) {
               const int32_t pg = prm.entries[idx].phys_page;
@@ -327,7 +326,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
               else atomicOr(prm.error_word, static_cast<int>(RK_DEV_BAD_PAGE));
             }
           }
-          {
+        };
+        // K runs one tile ahead of V: with two V stages a V load waits for
+        // an older PV to finish, and K loads queued behind it arrived late
+        for (int j = -1; j < n_tiles; ++j) {
+          int32_t rows[C::EPT];
+          if (j + 1 < n_tiles) {
+            tile_rows(j + 1, rows);
             const int st = k_issued % SK;
             const uint32_t u = k_issued / SK;
             if (u > 0 && !(ok = mbar_wait(&k_empty[st], (u - 1) & 1, wc, 2))) break;
@@ -340,7 +345,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                             &k_full[st], cb * 64, rows[e]);
             ++k_issued;
           }
-          {
+          if (j >= 0) {
+            tile_rows(j, rows);
             const int st = v_issued % SV;
             const uint32_t u = v_issued / SV;
             if (u > 0 && !(ok = mbar_wait(&v_empty[st], (u - 1) & 1, wc, 3))) break;
