@@ -54,7 +54,7 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int* t
   return excl;
 }
 
-constexpr int kSelectThreads = 256;
+constexpr int kSelectThreads = 512;
 static_assert(kCostBuckets % kSelectThreads == 0, "buckets per thread");
 constexpr int kPosCap = 3072;  // page positions of one table kept in shared memory
 
