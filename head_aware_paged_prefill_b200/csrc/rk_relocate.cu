@@ -24,9 +24,9 @@ struct RopeFreqs {
   double f[64];  // theta^(-2m/D), m < D/2
 };
 
-constexpr int kRelocThreads = 256;
+constexpr int kRelocThreads = 128;
 constexpr int kRelocMaxStages = 16;
-constexpr int kRelocRingBytes = 64 * 1024;
+constexpr int kRelocRingBytes = 48 * 1024;
 
 // Stages for a page size: about kRelocRingBytes of ring, 2 .. kRelocMaxStages.
 __host__ __device__ inline int reloc_stages(int page_bytes) {
