@@ -14,7 +14,8 @@
 namespace rk {
 
 cudaError_t launch_select(LayoutView* lv_dev, int n_tables, const rk_visible& vis, WsHeader* hdr,
-                          Item* items_tmp, Item* items, int32_t* cursor, cudaStream_t stream);
+                          Item* items_tmp, Item* items, int32_t* cursor, int64_t n_items,
+                          cudaStream_t stream);
 cudaError_t launch_relocate(const void* k_src, void* k_dst, const int32_t* jobs, int n_jobs,
                             int64_t n_src_pages, int64_t n_dst_pages, int P, int D, double theta,
                             int* device_error, cudaStream_t stream);
@@ -314,7 +315,10 @@ extern "C" rk_status rk_select_visible(const rk_dims* dims, const rk_layout* lay
                                 reinterpret_cast<WsHeader*>(ws),
                                 reinterpret_cast<Item*>(ws + dv.map.items_tmp),
                                 reinterpret_cast<Item*>(ws + dv.map.items),
-                                reinterpret_cast<int32_t*>(ws + dv.map.cursor), s);
+                                reinterpret_cast<int32_t*>(ws + dv.map.cursor),
+                                img[reinterpret_cast<const LayoutView*>(img.data())->off_tile_prefix +
+                                    dv.n_tables],
+                                s);
   return e == cudaSuccess ? RK_OK : RK_ERR_CUDA;
 }
 

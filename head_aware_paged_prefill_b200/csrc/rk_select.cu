@@ -13,8 +13,9 @@
 //      into the first sorted slot of each cost bucket, longest first, and
 //      publishes the item count and the selection's error bits in the
 //      workspace header.
-// A second launch, again one CTA per table, moves each table's items to
-// their sorted slots (a counting sort spread over all tables: one CTA alone
+// Up to kLastCtaSortItems items, the last CTA also moves every item to its
+// sorted slot; beyond that a second launch, again one CTA per table, moves
+// each table's items (a counting sort spread over all tables: one CTA alone
 // took ~0.4 ms for 250K items).
 #include <cuda_runtime.h>
 
@@ -56,6 +57,8 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int* t
 
 constexpr int kSelectThreads = 512;
 static_assert(kCostBuckets % kSelectThreads == 0, "buckets per thread");
+constexpr int kLastCtaSortItems = 16384;
+constexpr int kScatterBatch = 4;  // items a thread loads before claiming their slots
 constexpr int kPosCap = 3072;  // page positions of one table kept in shared memory
 
 // Claims one slot of counter hist[b] per lane; lanes of the warp with the
@@ -92,7 +95,7 @@ __device__ __forceinline__ int upper_bound(int n, int v, Key key) {
 
 __global__ void __launch_bounds__(kSelectThreads)
     select_kernel(LayoutView* __restrict__ lv, rk_visible vis, WsHeader* hdr, Item* items_tmp,
-                  int32_t* cursor) {
+                  int32_t* cursor, Item* items) {
   __shared__ int warp_tot[kSelectThreads / 32];
   __shared__ int s_total;
   __shared__ int s_last;
@@ -298,10 +301,31 @@ __global__ void __launch_bounds__(kSelectThreads)
     }
     const int ex = block_exclusive_scan<kSelectThreads>(sum, warp_tot, &s_total);
     int run = ex;
+    // items given: this CTA sorts them, with the cursors in shared memory
+    int* cur = items ? hist : cursor;
 #pragma unroll
     for (int k = 0; k < per; ++k) {
-      cursor[threadIdx.x * per + k] = run;
+      cur[threadIdx.x * per + k] = run;
       run += loc[k];
+    }
+    if (items) {
+      __syncthreads();
+      constexpr int kChunk = kSelectThreads * kScatterBatch;
+      for (int base = 0; base < total; base += kChunk) {
+        Item it[kScatterBatch];
+#pragma unroll
+        for (int b = 0; b < kScatterBatch; ++b) {
+          const int x = base + b * kSelectThreads + threadIdx.x;
+          if (x < total) it[b] = items_tmp[x];
+        }
+#pragma unroll
+        for (int b = 0; b < kScatterBatch; ++b) {
+          const int x = base + b * kSelectThreads + threadIdx.x;
+          const bool v = x < total;
+          const int pos = warp_claim(hist, v ? cost_bucket(it[b].cost) : 0, v);
+          if (v) items[pos] = it[b];
+        }
+      }
     }
   }
   if (threadIdx.x == 0) {
@@ -346,10 +370,17 @@ __global__ void __launch_bounds__(kSelectThreads)
 }
 
 cudaError_t launch_select(LayoutView* lv_dev, int n_tables, const rk_visible& vis, WsHeader* hdr,
-                          Item* items_tmp, Item* items, int32_t* cursor, cudaStream_t stream) {
+                          Item* items_tmp, Item* items, int32_t* cursor, int64_t n_items,
+                          cudaStream_t stream) {
   if (n_tables <= 0) return cudaSuccess;
-  select_kernel<<<n_tables, kSelectThreads, 0, stream>>>(lv_dev, vis, hdr, items_tmp, cursor);
-  scatter_kernel<<<n_tables, kSelectThreads, 0, stream>>>(lv_dev, items_tmp, items, cursor);
+  if (n_items <= kLastCtaSortItems) {
+    select_kernel<<<n_tables, kSelectThreads, 0, stream>>>(lv_dev, vis, hdr, items_tmp, cursor,
+                                                           items);
+  } else {
+    select_kernel<<<n_tables, kSelectThreads, 0, stream>>>(lv_dev, vis, hdr, items_tmp, cursor,
+                                                           nullptr);
+    scatter_kernel<<<n_tables, kSelectThreads, 0, stream>>>(lv_dev, items_tmp, items, cursor);
+  }
   return cudaGetLastError();
 }
 
@@ -357,7 +388,8 @@ cudaError_t launch_select(LayoutView* lv_dev, int n_tables, const rk_visible& vi
 cudaError_t launch_select_tables_only(LayoutView* lv_dev, int n_tables, const rk_visible& vis,
                                       WsHeader* hdr, cudaStream_t stream) {
   if (n_tables > 0)
-    select_kernel<<<n_tables, kSelectThreads, 0, stream>>>(lv_dev, vis, hdr, nullptr, nullptr);
+    select_kernel<<<n_tables, kSelectThreads, 0, stream>>>(lv_dev, vis, hdr, nullptr, nullptr,
+                                                           nullptr);
   return cudaGetLastError();
 }
 

@@ -1,0 +1,66 @@
+"""The attention work list the selection builds in the workspace: a
+permutation of the per-table items, longest first.  Small lists are sorted by
+the selection kernel's last CTA, large ones by the per-table scatter launch;
+both are checked.  White-box: reads the workspace through its internal map
+(a 256-byte header, then the sorted list, then the unsorted list)."""
+import numpy as np
+import pytest
+import torch
+
+from head_aware_paged_prefill_b200 import binding, synth
+
+pytestmark = pytest.mark.gpu
+
+HEADER = 256
+ITEM_WORDS = 12  # q_row0, row_begin, row_end, e_begin, e_end, qh0, nh, window, layer, req, table, cost
+COST_BUCKETS = 2048
+
+
+def _align(x, a):
+    return (x + a - 1) // a * a
+
+
+def _work_lists(lay):
+    hl = binding.HostLayout(lay)
+    sz = hl.sizes()
+    vis = binding.Visible(sz, "cuda")
+    ws = binding.workspace(sz, "cuda")
+    binding.select_visible(hl, vis, ws)
+    torch.cuda.synchronize()
+    assert binding.device_status(ws) == 0
+    raw = ws.cpu().numpy().view(np.uint8)
+    n_items = int(raw[4:8].view(np.int32)[0])
+    cap = int(sz.item_capacity)
+    sorted_off = HEADER
+    tmp_off = _align(HEADER + 48 * cap, 256)
+    items = raw[sorted_off:sorted_off + 48 * n_items].view(np.int32).reshape(-1, ITEM_WORDS)
+    tmp = raw[tmp_off:tmp_off + 48 * n_items].view(np.int32).reshape(-1, ITEM_WORDS)
+    return n_items, items, tmp, cap
+
+
+def _check(lay, expect_large=None):
+    n, items, tmp, cap = _work_lists(lay)
+    assert 0 <= n <= cap
+    if expect_large is not None:
+        assert (n > 16384) == expect_large
+    # a permutation of the per-table items
+    key = lambda a: np.lexsort(a.T[::-1])
+    assert np.array_equal(items[key(items)], tmp[key(tmp)])
+    # longest first (costs past the last bucket share it)
+    c = np.minimum(items[:, 11], COST_BUCKETS - 1)
+    assert np.all(c[:-1] >= c[1:])
+    # every item of a table lies in that table and has a cost of its entries
+    assert np.all(items[:, 4] >= items[:, 3])
+    assert np.all(items[:, 6] >= 1) and np.all(items[:, 6] <= 2)
+
+
+@pytest.mark.parametrize("name,large", [("cfg1", False), ("cfg2", False), ("cfg4", False),
+                                        ("cfg5", True)])
+def test_work_list_sorted_permutation(name, large):
+    _check(synth.CONFIGS[name]().layout, expect_large=large)
+
+
+def test_work_list_random_small():
+    rng = np.random.default_rng(77)
+    for _ in range(20):
+        _check(synth.random_small(rng))
