@@ -39,8 +39,13 @@ class SegPagedPrefill:
         self.mode = mode
         self.device = torch.device(device)
         lay = layout
+        entries, ranges = self._tables(layout)
+        # attention work items: 128-row tiles of each table's row ranges x
+        # pairs of q heads (the library's own rule)
+        npairs = (layout.hq // layout.hkv + 1) // 2
+        self.n_items = npairs * sum(-(-(int(b) - int(a)) // 128) for rr in ranges for a, b in rr)
         if mode == "relocate":
-            self.plan = self._plan(layout)
+            self.plan = relocation_plan(layout, entries)
         else:
             empty = np.zeros((0, 3), np.int32)
             self.plan = RelocationPlan(empty, empty, layout, 0)
@@ -77,9 +82,10 @@ class SegPagedPrefill:
                         if self.mode == "relocate" else None),
         }
 
-    def _plan(self, layout) -> RelocationPlan:
-        """Page tables of the original layout (built by the library on the
-        device), read back once, turned into relocation jobs."""
+    def _tables(self, layout):
+        """Page tables and row ranges of the original layout, built once by
+        the library on the device and read back (relocation jobs, item
+        count)."""
         hl = binding.HostLayout(layout)
         sizes = hl.sizes()
         vis = binding.Visible(sizes, self.device)
@@ -89,14 +95,16 @@ class SegPagedPrefill:
         st = binding.device_status(ws)
         if st:
             raise binding.RkError(binding.RK_ERR_DEVICE, f"rk_select_visible (device {st:#x})")
-        entries, _ = vis.tables()
-        return relocation_plan(layout, entries)
+        return vis.tables()
 
     # Number of library kernel launches one run() makes.
     @property
     def launches_per_run(self) -> int:
-        # select (one kernel) + attention, plus the relocation launches
-        return 2 + int(self.plan.jobs_k.shape[0] > 0) + int(self.plan.jobs_v.shape[0] > 0)
+        # selection (one kernel; a second one moves the work list into cost
+        # order above 16384 items), attention, and the relocation launches
+        select = 1 if self.n_items <= 16384 else 2
+        return (select + 1 + int(self.plan.jobs_k.shape[0] > 0) +
+                int(self.plan.jobs_v.shape[0] > 0))
 
     def _copy_in(self, b: dict, q, k_pool, v_pool):
         """Copies a step's inputs (host or device) into buffer set b on the

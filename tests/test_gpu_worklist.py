@@ -64,3 +64,12 @@ def test_work_list_random_small():
     rng = np.random.default_rng(77)
     for _ in range(20):
         _check(synth.random_small(rng))
+
+
+@pytest.mark.parametrize("name", ["cfg1", "cfg3", "cfg5"])
+def test_api_item_count_matches_library(name):
+    """The API's launch accounting counts work items by the library's rule."""
+    from head_aware_paged_prefill_b200.api import SegPagedPrefill
+    lay = synth.CONFIGS[name]().layout
+    n, _, _, _ = _work_lists(lay)
+    assert SegPagedPrefill(lay, "cuda", mode="fused").n_items == n
