@@ -89,6 +89,27 @@ def test_prefill_random_small_all_rows(mode):
         _untouched(lay, run)
 
 
+@pytest.mark.parametrize("mode", MODES)
+@pytest.mark.parametrize("cmap", [(0, 1, 2), (3, 2, 1)])
+def test_prefill_edge_layout_all_rows(mode, cmap):
+    """An empty request between others, a request whose rows are all cached
+    (no local / retrieval rows), a one-token request, window 1, retrieval
+    lists that name pages before and after the rows, D 64 with 16-token
+    pages and a partial last page."""
+    reqs = [[("a", 64, 0, True), ("t0", 37, 0, False)], [],
+            [("b", 64, 5, True), ("c", 128, 9, True)], [("t3", 1, 0, False)]]
+    lay = synth._make_layout(n_layers=1, hq=3, hkv=3, d=64, p=16, theta=1e4, requests=reqs,
+                             class_map=list(cmap), window=1,
+                             retrieval={0: [0, 3], 1: [1], 2: [2, 5], 7: [0, 1]})
+    wl = synth.tiny_workload(lay, seed=11)
+    q, k, v = wl.materialize("cpu")
+    run = PrefillRun(lay, q.cuda(), k.cuda(), v.cuda(), mode=mode)
+    rows = _all_rows(lay)
+    assert rows.shape[0] > 0
+    _check(lay, q, k, v, run, rows, f"edge layout {cmap} {mode}")
+    _untouched(lay, run)
+
+
 @pytest.mark.parametrize("name,per_table", [("cfg2", 24), ("cfg3", 16), ("cfg4", 16),
                                             ("cfg5", 3)])
 def test_prefill_full_size_sampled(name, per_table):
