@@ -269,10 +269,20 @@ def run_reference(args, rank, world):
     lay = wl.layout
     q, k, v = cpu_values(wl)
     cores = os.cpu_count() or 1
-    # size the per-step sample so one step takes about args.ref_step_s seconds
-    rows, pairs = _oracle_sample_rows(lay, 64, seed=0)
-    dt = _time_oracle(lay, q, k, v, rows)
-    n_rows = int(max(16, min(4096, 64 * args.ref_step_s / max(dt, 1e-3))))
+    # size the per-step sample: one oracle call has a fixed cost (layout
+    # setup, key relocation) besides its cost per row, so two calls of
+    # different sizes give both; a step then takes about 4x the fixed cost
+    # (at least --ref-step-s), within a budget that ends the whole run in
+    # about four minutes
+    rows, _ = _oracle_sample_rows(lay, 64, seed=0)
+    t_a = _time_oracle(lay, q, k, v, rows)
+    rows, _ = _oracle_sample_rows(lay, 512, seed=0)
+    t_b = _time_oracle(lay, q, k, v, rows)
+    per_row = max((t_b - t_a) / (512 - 64), 1e-7)
+    fixed = max(t_a - 64 * per_row, 0.0)
+    budget = max(240.0 / (args.warmup + args.steps), args.ref_step_s)
+    step_s = min(max(args.ref_step_s, 4 * fixed), budget)
+    n_rows = int(max(64, min(65536, (step_s - fixed) / per_row)))
     tot_t, tot_pairs = 0.0, 0
     for s in range(args.warmup + args.steps):
         rows, pairs = _oracle_sample_rows(lay, n_rows, seed=1 + s)
