@@ -59,6 +59,10 @@ def _load():
                                       ctypes.c_void_p, ctypes.c_double, ctypes.c_double,
                                       ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p,
                                       ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+        lib.ora_score_pages.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                        ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                        ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
+        lib.ora_score_pages.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -153,6 +157,37 @@ def page_tables(lay, threads=None) -> Tuple[List[np.ndarray], List[np.ndarray]]:
     with ThreadPoolExecutor(_threads(threads)) as ex:
         list(ex.map(one, list(_tables(lay))))
     return entries, ranges
+
+
+# ------------------------------------------------- retrieval page scoring
+
+def score_pages(lay, q_u16: np.ndarray, k_pool_u16: np.ndarray, top_k: int = 16,
+                threads=None) -> Tuple[List[np.ndarray], List[np.ndarray]]:
+    """Per table: the retrieval page picks (ascending page indices within the
+    request) and the fp64 score of every page of the request (NaN for pages
+    that are not candidates).  The reading is stated in ``ora_score_pages``.
+    q: bf16 bits [n_layers][T][Hq][D]; k_pool: bf16 bits [n_pages][P][D]."""
+    lib = _load()
+    pref = _ProblemRef(lay)
+    q = np.ascontiguousarray(q_u16.view(np.uint16))
+    k = np.ascontiguousarray(k_pool_u16.view(np.uint16))
+    n_t = lay.n_tables
+    picks: List[np.ndarray] = [None] * n_t
+    scores: List[np.ndarray] = [None] * n_t
+
+    def one(args):
+        t, r, layer, h = args
+        npg = -(-lay.req_len(r) // lay.p)
+        pg = np.zeros(max(npg, 1), dtype=np.int32)
+        sc = np.zeros(max(npg, 1), dtype=np.float64)
+        n = lib.ora_score_pages(pref.ptr, q.ctypes.data, k.ctypes.data, float(lay.theta),
+                                int(top_k), r, layer, h, pg.ctypes.data, sc.ctypes.data)
+        picks[t] = pg[:n].copy()
+        scores[t] = sc[:npg].copy()
+
+    with ThreadPoolExecutor(_threads(threads)) as ex:
+        list(ex.map(one, list(_tables(lay))))
+    return picks, scores
 
 
 def _uncached_ranges(lay, r) -> List[Tuple[int, int]]:

@@ -28,6 +28,8 @@
  *     (phys_page, logical_pos, delta, n_valid); row set as merged half-open
  *     ranges.  Both are derived by brute force over (row, key) pairs.
  *
+ *   - Retrieval page scoring (ora_score_pages, a reading stated there).
+ *
  * parity pins: see tests/test_oracle_pins.py (RoPE closed form and
  * composition, causal and windowed SDPA special cases, perturbation
  * invariance, sharing, brute-force vs closed-form page tables, pair counts).
@@ -434,4 +436,110 @@ int ora_attention(const ora_problem* pr, const uint16_t* q_rows, const uint16_t*
   free(key);
   free(order);
   return 0;
+}
+
+/* ------------------------------------------------ retrieval page scoring */
+
+/* Retrieval heads attend the uncached tail plus a list of cached pages that
+ * the RedKnot pages say is chosen "by query semantics" (paooo page, "how to
+ * use" section, SELECTVISIBLESTATE) without giving a rule.  The reading
+ * implemented here, for one retrieval table (r, layer, kvh):
+ *   rows     = the table's computed rows (the uncached positions of r);
+ *   u        = sum over the G q heads h of kvh of the mean over the rows i of
+ *              q[layer][cu[r] + i][h] (queries are given post-RoPE);
+ *   cand     = pages pg of r whose keys are cached and whose first position
+ *              is at most the last row;
+ *   kbar_pg  = mean over the page's n_valid keys of the relocated key
+ *              R(delta) K_stored;
+ *   score_pg = <u, kbar_pg>;
+ *   pick     = the top_k candidates by score (ties to the lower page index),
+ *              all candidates when there are at most top_k, in ascending
+ *              page order.
+ * q: bf16 [n_layers][T][hq][d]; k_pool: bf16 [n_pages][p][d].  pages_out
+ * gets the picks; scores_out[pg] (length = pages of the request) gets each
+ * candidate's score and NaN elsewhere.  Returns the number of picks (0 for a
+ * table of another class or without rows). */
+int ora_score_pages(const ora_problem* pr, const uint16_t* q, const uint16_t* k_pool,
+                    double theta, int top_k, int r, int layer, int kvh, int32_t* pages_out,
+                    double* scores_out) {
+  ora_table t;
+  table_open(&t, pr, r, layer, kvh);
+  int L = t.L, P = pr->p, d = pr->d, h = d / 2;
+  int npg = (L + P - 1) / P;
+  int T = pr->cu_seqlens[pr->n_req];
+  for (int pg = 0; pg < npg; ++pg) scores_out[pg] = NAN;
+  int n_out = 0;
+  int last_row = -1, n_rows = 0;
+  for (int i = 0; i < L; ++i)
+    if (is_row(&t, i)) {
+      last_row = i;
+      ++n_rows;
+    }
+  if (t.cls != ORA_RETRIEVAL || n_rows == 0) {
+    table_close(&t);
+    return 0;
+  }
+  int g = pr->hq / pr->hkv;
+  double* u = (double*)calloc((size_t)d, sizeof(double));
+  for (int hh = kvh * g; hh < kvh * g + g; ++hh) {
+    for (int c = 0; c < d; ++c) {
+      double acc = 0.0;
+      for (int i = 0; i < L; ++i) {
+        if (!is_row(&t, i)) continue;
+        size_t off = (((size_t)layer * T + pr->cu_seqlens[r] + i) * pr->hq + hh) * d + c;
+        acc += bf16_to_double(q[off]);
+      }
+      u[c] += acc / n_rows;
+    }
+  }
+  int lh = layer * pr->hkv + kvh;
+  double* kbar = (double*)malloc(sizeof(double) * d);
+  double* kr = (double*)malloc(sizeof(double) * d);
+  double* x = (double*)malloc(sizeof(double) * d);
+  int* cand = (int*)malloc(sizeof(int) * ((size_t)npg + 1));
+  int n_cand = 0;
+  for (int pg = 0; pg < npg; ++pg) {
+    int j0 = pg * P;
+    if (t.uncached[j0] || j0 > last_row) continue;
+    int s = t.seg_of[j0];
+    const int32_t* sg = pr->seg + 5 * s;
+    const int shift = sg[1] - sg[3]; /* the page's relocation delta */
+    int nv = L - j0 < P ? L - j0 : P;
+    for (int c = 0; c < d; ++c) kbar[c] = 0.0;
+    for (int rr = 0; rr < nv; ++rr) {
+      int off = j0 + rr - sg[1];
+      int page = pr->page_base[(size_t)s * pr->n_layers * pr->hkv + lh] + off / P;
+      const uint16_t* ks = k_pool + ((size_t)page * P + off % P) * d;
+      for (int c = 0; c < d; ++c) x[c] = bf16_to_double(ks[c]);
+      ora_rope_rotate(x, d, theta, (double)shift, kr);
+      for (int c = 0; c < d; ++c) kbar[c] += kr[c];
+    }
+    double sc = 0.0;
+    for (int c = 0; c < d; ++c) sc += u[c] * (kbar[c] / nv);
+    scores_out[pg] = sc;
+    cand[n_cand++] = pg;
+  }
+  (void)h;
+  /* top_k by repeated selection of the best remaining candidate */
+  int8_t* taken = (int8_t*)calloc((size_t)npg + 1, 1);
+  int n_pick = n_cand < top_k ? n_cand : top_k;
+  for (int k = 0; k < n_pick; ++k) {
+    int best = -1;
+    for (int a = 0; a < n_cand; ++a) {
+      int pg = cand[a];
+      if (taken[pg]) continue;
+      if (best < 0 || scores_out[pg] > scores_out[best]) best = pg;
+    }
+    taken[best] = 1;
+  }
+  for (int pg = 0; pg < npg; ++pg)
+    if (taken[pg]) pages_out[n_out++] = pg;
+  free(taken);
+  free(cand);
+  free(x);
+  free(kr);
+  free(kbar);
+  free(u);
+  table_close(&t);
+  return n_out;
 }

@@ -12,6 +12,7 @@ import pytest
 
 import oracle
 import test_oracle_pins as pins
+import test_oracle_scoring as scoring
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "rk_oracle.c")
 
@@ -28,6 +29,18 @@ MUTANTS = {
     "lse_drops_max": ("aj->lse[idx] = mx + log(sum);", "aj->lse[idx] = log(sum);"),
     "n_valid_always_p": ("int nv = L - k * P < P ? L - k * P : P;", "int nv = P;"),
     "page_offset": ("int page_in_seg = (k * P - sg[1]) / P;", "int page_in_seg = (k * P - sg[1]) / P + 1;"),
+    # retrieval page scoring
+    "score_no_relocation": ("ora_rope_rotate(x, d, theta, (double)shift, kr);",
+                            "ora_rope_rotate(x, d, theta, 0.0, kr);"),
+    "score_shift_sign": ("ora_rope_rotate(x, d, theta, (double)shift, kr);",
+                         "ora_rope_rotate(x, d, theta, -(double)shift, kr);"),
+    "score_rows_summed": ("u[c] += acc / n_rows;", "u[c] += acc;"),
+    "score_one_head": ("for (int hh = kvh * g; hh < kvh * g + g; ++hh) {",
+                       "for (int hh = kvh * g; hh < kvh * g + 1; ++hh) {"),
+    "score_ties_upper": ("if (best < 0 || scores_out[pg] > scores_out[best]) best = pg;",
+                         "if (best < 0 || scores_out[pg] >= scores_out[best]) best = pg;"),
+    "score_uncached_candidates": ("if (t.uncached[j0] || j0 > last_row) continue;",
+                                  "if (j0 > last_row) continue;"),
 }
 
 PIN_CALLS = [
@@ -39,6 +52,10 @@ PIN_CALLS = [
     pins.test_cfg1_page_table_by_hand,
     pins.test_partial_last_page_by_hand,
     lambda: [pins.test_visible_pairs_brute_force("cfg1")],
+    scoring.test_scores_equal_bilinear_expansion,
+    scoring.test_planted_pages_win,
+    scoring.test_few_candidates_all_picked_and_other_tables_empty,
+    scoring.test_ties_go_to_the_lower_page,
 ]
 
 
