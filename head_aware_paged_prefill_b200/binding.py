@@ -57,7 +57,8 @@ class RkSizes(ctypes.Structure):
 
 
 EXPORTS = ("rk_query_sizes", "rk_select_visible", "rk_relocate_rope", "rk_segpaged_prefill",
-           "rk_get_device_status", "rk_select_visible_noalloc", "rk_selftest_bounded_wait")
+           "rk_get_device_status", "rk_select_visible_noalloc", "rk_selftest_bounded_wait",
+           "rk_score_query_sizes", "rk_score_retrieval_pages")
 
 _lib = None
 
@@ -80,6 +81,9 @@ def lib() -> ctypes.CDLL:
         L.rk_get_device_status.argtypes = [vp, vp, vp]
         L.rk_select_visible_noalloc.argtypes = [vp, vp, vp, vp, vp]
         L.rk_selftest_bounded_wait.argtypes = [vp, i32, vp]
+        L.rk_score_query_sizes.argtypes = [vp, vp, i32, vp]
+        L.rk_score_retrieval_pages.argtypes = [vp, vp, vp, vp, ctypes.c_double, i32, vp, vp, vp,
+                                               i64, vp, ctypes.c_size_t, vp]
         for name in EXPORTS:
             getattr(L, name).restype = i32
         _lib = L
@@ -99,6 +103,11 @@ def _stream(stream) -> ctypes.c_void_p:
     if stream is None:
         stream = torch.cuda.current_stream()
     return ctypes.c_void_p(stream.cuda_stream)
+
+
+class RkScoreSizes(ctypes.Structure):
+    _fields_ = [("n_tables", ctypes.c_int64), ("max_pages", ctypes.c_int64),
+                ("workspace_bytes", ctypes.c_int64)]
 
 
 class HostLayout:
@@ -211,3 +220,46 @@ def device_status(ws: torch.Tensor, stream=None) -> int:
     if st not in (RK_OK, RK_ERR_DEVICE):
         raise RkError(st, "rk_get_device_status")
     return int(v.value)
+
+
+# ------------------------------------------------------ retrieval page scoring
+
+def score_sizes(hl: HostLayout, top_k: int = 16) -> RkScoreSizes:
+    s = RkScoreSizes()
+    _check(lib().rk_score_query_sizes(ctypes.byref(hl.dims), ctypes.byref(hl.layout), int(top_k),
+                                      ctypes.byref(s)), "rk_score_query_sizes")
+    return s
+
+
+class ScoreOutputs:
+    """Device outputs of rk_score_retrieval_pages for one layout."""
+
+    def __init__(self, sizes: RkScoreSizes, top_k: int, device, with_scores: bool = True):
+        dev = torch.device(device)
+        n = int(sizes.n_tables)
+        self.top_k = int(top_k)
+        self.pages = torch.zeros((n, self.top_k), dtype=torch.int32, device=dev)
+        self.count = torch.zeros(n, dtype=torch.int32, device=dev)
+        self.stride = max(int(sizes.max_pages), 1)
+        self.scores = (torch.empty((n, self.stride), dtype=torch.float32, device=dev)
+                       if with_scores else None)
+        self.ws = torch.zeros(max(int(sizes.workspace_bytes), 256), dtype=torch.uint8, device=dev)
+
+    def lists(self):
+        """The picks as a host CSR (retr_indptr, retr_pages) over tables."""
+        count = self.count.cpu().numpy()
+        pages = self.pages.cpu().numpy()
+        indptr = np.zeros(count.shape[0] + 1, dtype=np.int32)
+        indptr[1:] = np.cumsum(count)
+        flat = np.concatenate([pages[t, :count[t]] for t in range(count.shape[0])] +
+                              [np.zeros(0, np.int32)]).astype(np.int32)
+        return indptr, flat
+
+
+def score_retrieval_pages(hl: HostLayout, q: torch.Tensor, k_store: torch.Tensor, theta: float,
+                          out: ScoreOutputs, stream=None):
+    _check(lib().rk_score_retrieval_pages(
+        ctypes.byref(hl.dims), ctypes.byref(hl.layout), _ptr(q), _ptr(k_store), float(theta),
+        out.top_k, _ptr(out.pages), _ptr(out.count), _ptr(out.scores),
+        out.stride if out.scores is not None else 0, _ptr(out.ws), out.ws.numel(),
+        _stream(stream)), "rk_score_retrieval_pages")

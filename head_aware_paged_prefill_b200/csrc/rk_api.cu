@@ -265,6 +265,132 @@ void build_layout_image(const rk_dims* d, const rk_layout* lay, const Derived& d
   std::memcpy(w, &v, sizeof(LayoutView));
 }
 
+// ---- retrieval page scoring: the host image the scoring kernels read
+
+struct ScorePlan {
+  std::vector<int32_t> img;  // ScoreView followed by its arrays
+  ScoreView sv{};
+  int64_t max_pages = 0;     // pages of the longest request (scores row length)
+  size_t off_partials = 0, off_cand_scores = 0, total = 0;  // workspace byte offsets
+};
+
+// A copy of the layout whose retrieval lists are empty when it has none:
+// scoring produces the lists, so it must accept a layout without them.
+struct ScoreLayout {
+  rk_layout lay;
+  std::vector<int32_t> empty_indptr;
+};
+
+void score_layout(const rk_dims* d, const rk_layout* in, ScoreLayout* out) {
+  out->lay = *in;
+  if (!in->retr_indptr) {
+    const int64_t n_tables = static_cast<int64_t>(d->n_req) * d->n_layers * d->num_kv_heads;
+    out->empty_indptr.assign(static_cast<size_t>(n_tables + 1), 0);
+    out->lay.retr_indptr = out->empty_indptr.data();
+    out->lay.retr_pages = nullptr;
+  }
+}
+
+rk_status build_score_plan(const rk_dims* d, const rk_layout* lay, const Derived& dv,
+                           int top_k, ScorePlan* out) {
+  const int P = d->page_size, D = d->head_dim, n_req = d->n_req;
+  const int hkv = d->num_kv_heads, g = d->num_q_heads / hkv;
+  std::vector<ScoreTable> tables;
+  std::vector<ScoreChunk> chunks;
+  std::vector<ScoreCand> cands;
+  std::vector<int32_t> blocks;  // (st, first candidate) pairs
+  std::vector<int32_t> table_map(static_cast<size_t>(dv.n_tables), -1);
+  int64_t max_pages = 0;
+  for (int r = 0; r < n_req; ++r) {
+    const int L = lay->cu_seqlens[r + 1] - lay->cu_seqlens[r];
+    max_pages = std::max<int64_t>(max_pages, (L + P - 1) / P);
+    // the request's rows for retrieval heads: its uncached positions, merged
+    std::vector<std::pair<int, int>> rows;
+    int last_row = -1, n_rows = 0;
+    for (int s = dv.seg_indptr[r]; s < dv.seg_indptr[r + 1]; ++s) {
+      const rk_segment& sg = lay->segments[s];
+      if (sg.cached || sg.len == 0) continue;
+      const int a = sg.logical_start, b = a + sg.len;
+      if (!rows.empty() && rows.back().second == a) rows.back().second = b;
+      else rows.emplace_back(a, b);
+      last_row = b - 1;
+      n_rows += sg.len;
+    }
+    for (int layer = 0; layer < d->n_layers; ++layer)
+      for (int kvh = 0; kvh < hkv; ++kvh) {
+        const int lh = layer * hkv + kvh;
+        if (lay->class_map[lh] != RK_RETRIEVAL || n_rows == 0) continue;
+        const int t = (r * d->n_layers + layer) * hkv + kvh;
+        ScoreTable st{};
+        st.table = t;
+        st.q_row0 = layer * d->total_tokens + lay->cu_seqlens[r];
+        st.head0 = kvh * g;
+        st.n_rows = n_rows;
+        st.chunk_begin = static_cast<int32_t>(chunks.size());
+        const int st_idx = static_cast<int>(tables.size());
+        for (const auto& rg : rows)
+          for (int a = rg.first; a < rg.second; a += kScoreChunkRows)
+            chunks.push_back(ScoreChunk{st_idx, a, std::min(kScoreChunkRows, rg.second - a), 0});
+        st.chunk_end = static_cast<int32_t>(chunks.size());
+        st.cand_begin = static_cast<int32_t>(cands.size());
+        for (int s = dv.seg_indptr[r]; s < dv.seg_indptr[r + 1]; ++s) {
+          const rk_segment& sg = lay->segments[s];
+          if (!sg.cached) continue;
+          const int32_t base = lay->page_base[static_cast<int64_t>(s) * dv.n_lh + lh];
+          for (int pos = sg.logical_start; pos < sg.logical_start + sg.len && pos <= last_row;
+               pos += P)
+            cands.push_back(ScoreCand{pos / P, base + (pos - sg.logical_start) / P,
+                                      sg.logical_start - sg.stored_pos_base, std::min(P, L - pos)});
+        }
+        st.cand_end = static_cast<int32_t>(cands.size());
+        if (st.cand_end - st.cand_begin > kScoreMaxCand) return RK_ERR_CAPACITY;
+        for (int c = st.cand_begin; c < st.cand_end; c += kScorePagesPerCta) {
+          blocks.push_back(st_idx);
+          blocks.push_back(c);
+        }
+        table_map[static_cast<size_t>(t)] = st_idx;
+        tables.push_back(st);
+      }
+  }
+  if (cands.size() >= static_cast<size_t>(kMaxI32 / 8) ||
+      chunks.size() >= static_cast<size_t>(kMaxI32 / 8))
+    return RK_ERR_INVALID_ARG;
+  ScoreView& v = out->sv;
+  v.n_st = static_cast<int32_t>(tables.size());
+  v.n_chunks = static_cast<int32_t>(chunks.size());
+  v.n_cand = static_cast<int32_t>(cands.size());
+  v.n_blocks = static_cast<int32_t>(blocks.size() / 2);
+  v.n_tables = static_cast<int32_t>(dv.n_tables);
+  v.top_k = top_k;
+  v.hq = d->num_q_heads;
+  v.g = g;
+  int32_t off = static_cast<int32_t>((sizeof(ScoreView) + 3) / 4);
+  v.off_tables = off;
+  off += static_cast<int32_t>(tables.size() * sizeof(ScoreTable) / 4);
+  v.off_chunks = off;
+  off += static_cast<int32_t>(chunks.size() * sizeof(ScoreChunk) / 4);
+  v.off_cand = off;
+  off += static_cast<int32_t>(cands.size() * sizeof(ScoreCand) / 4);
+  v.off_blocks = off;
+  off += static_cast<int32_t>(blocks.size());
+  v.off_table_map = off;
+  off += static_cast<int32_t>(table_map.size());
+  v.words = off;
+  out->img.assign(static_cast<size_t>(off), 0);
+  int32_t* w = out->img.data();
+  std::memcpy(w, &v, sizeof v);
+  if (!tables.empty()) std::memcpy(w + v.off_tables, tables.data(), tables.size() * sizeof(ScoreTable));
+  if (!chunks.empty()) std::memcpy(w + v.off_chunks, chunks.data(), chunks.size() * sizeof(ScoreChunk));
+  if (!cands.empty()) std::memcpy(w + v.off_cand, cands.data(), cands.size() * sizeof(ScoreCand));
+  if (!blocks.empty()) std::memcpy(w + v.off_blocks, blocks.data(), blocks.size() * 4);
+  if (!table_map.empty()) std::memcpy(w + v.off_table_map, table_map.data(), table_map.size() * 4);
+  out->max_pages = max_pages;
+  out->off_partials = align_up(4 * static_cast<size_t>(off), 256);
+  out->off_cand_scores = align_up(out->off_partials + 4 * chunks.size() * D, 256);
+  out->total = align_up(out->off_cand_scores + 4 * cands.size(), 256);
+  return RK_OK;
+}
+
 }  // namespace
 }  // namespace rk
 
@@ -478,4 +604,61 @@ extern "C" rk_status rk_select_visible_noalloc(const rk_dims* dims, const rk_lay
                                       cudaMemcpyDeviceToDevice, s) != cudaSuccess)
     return RK_ERR_CUDA;
   return RK_OK;
+}
+
+extern "C" rk_status rk_score_query_sizes(const rk_dims* dims, const rk_layout* layout,
+                                          int32_t top_k, rk_score_sizes* out) {
+  if (!out || top_k < 1 || top_k > kScoreMaxTopK) return RK_ERR_INVALID_ARG;
+  rk_status st = check_dims(dims);
+  if (st != RK_OK) return st;
+  if (!layout) return RK_ERR_INVALID_ARG;
+  ScoreLayout sl;
+  score_layout(dims, layout, &sl);
+  Derived dv;
+  if ((st = check_layout(dims, &sl.lay, &dv)) != RK_OK) return st;
+  ScorePlan plan;
+  if ((st = build_score_plan(dims, &sl.lay, dv, top_k, &plan)) != RK_OK) return st;
+  out->n_tables = dv.n_tables;
+  out->max_pages = plan.max_pages;
+  out->workspace_bytes = static_cast<int64_t>(plan.total);
+  return RK_OK;
+}
+
+extern "C" rk_status rk_score_retrieval_pages(const rk_dims* dims, const rk_layout* layout,
+                                              const void* q, const void* k_store, double rope_theta,
+                                              int32_t top_k, int32_t* out_pages,
+                                              int32_t* out_count, float* out_scores,
+                                              int64_t scores_stride, void* workspace,
+                                              size_t workspace_bytes, void* stream) {
+  if (top_k < 1 || top_k > kScoreMaxTopK) return RK_ERR_INVALID_ARG;
+  if (!(rope_theta > 0.0) || !std::isfinite(rope_theta)) return RK_ERR_INVALID_ARG;
+  rk_status st = check_dims(dims);
+  if (st != RK_OK) return st;
+  if (!layout) return RK_ERR_INVALID_ARG;
+  ScoreLayout sl;
+  score_layout(dims, layout, &sl);
+  Derived dv;
+  if ((st = check_layout(dims, &sl.lay, &dv)) != RK_OK) return st;
+  ScorePlan plan;
+  if ((st = build_score_plan(dims, &sl.lay, dv, top_k, &plan)) != RK_OK) return st;
+  if (!q || !k_store || !out_pages || !out_count || !workspace) return RK_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k_store, 16) || !aligned(out_pages, 4) ||
+      !aligned(out_count, 4) || !aligned(out_scores, 4) || !aligned(workspace, 256))
+    return RK_ERR_INVALID_ARG;
+  if (out_scores && scores_stride < plan.max_pages) return RK_ERR_CAPACITY;
+  if (workspace_bytes < plan.total) return RK_ERR_CAPACITY;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (cudaMemcpyAsync(ws, plan.img.data(), 4 * plan.img.size(), cudaMemcpyHostToDevice, s) !=
+      cudaSuccess)
+    return RK_ERR_CUDA;
+  double inv_freq[64];
+  for (int m = 0; m < dims->head_dim / 2; ++m)
+    inv_freq[m] = std::pow(rope_theta, -2.0 * m / dims->head_dim);
+  cudaError_t e = launch_score(reinterpret_cast<const ScoreView*>(ws), plan.sv, q, k_store,
+                               dims->head_dim, dims->page_size, inv_freq,
+                               reinterpret_cast<float*>(ws + plan.off_partials),
+                               reinterpret_cast<float*>(ws + plan.off_cand_scores), out_pages,
+                               out_count, out_scores, out_scores ? scores_stride : 0, s);
+  return e == cudaSuccess ? RK_OK : RK_ERR_CUDA;
 }

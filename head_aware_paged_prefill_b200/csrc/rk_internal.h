@@ -5,6 +5,8 @@
 #include <cstddef>
 #include <cstdint>
 
+#include <cuda_runtime.h>
+
 #include "../../include/rk.h"
 
 namespace rk {
@@ -104,5 +106,43 @@ struct PrefillLaunchArgs {
   int fuse_rope;
   double rope_theta;
 };
+
+// ---- retrieval page scoring (host image read by the scoring kernels)
+
+constexpr int kScoreChunkRows = 64;   // query rows summed by one CTA
+constexpr int kScorePagesPerCta = 8;  // candidate pages per CTA (one warp each)
+constexpr int kScoreMaxCand = 4096;   // candidate pages of one table
+constexpr int kScoreMaxTopK = 64;
+
+struct ScoreTable {  // one retrieval table that has rows
+  int32_t table;     // table id
+  int32_t q_row0;    // layer * T + cu[r]: packed q row of the request's position 0
+  int32_t head0;     // first q head of the kv head
+  int32_t n_rows;    // computed rows (uncached positions)
+  int32_t chunk_begin, chunk_end;  // its query chunks
+  int32_t cand_begin, cand_end;    // its candidate pages
+};
+struct ScoreChunk {  // rows [row_begin, row_begin + n_rows) of one table
+  int32_t st, row_begin, n_rows, pad;
+};
+struct ScoreCand {  // a candidate page of a table
+  int32_t page, phys, delta, n_valid;
+};
+struct ScoreView {
+  int32_t n_st, n_chunks, n_cand, n_blocks, n_tables, top_k;
+  int32_t hq, g;
+  int32_t off_tables;     // ScoreTable[n_st]
+  int32_t off_chunks;     // ScoreChunk[n_chunks]
+  int32_t off_cand;       // ScoreCand[n_cand]
+  int32_t off_blocks;     // int32[n_blocks][2]: (st, first candidate) of each scoring CTA
+  int32_t off_table_map;  // int32[n_tables]: score table of a table, -1 if none
+  int32_t words;
+};
+
+cudaError_t launch_score(const ScoreView* sv_dev, const ScoreView& sv_host, const void* q,
+                         const void* k_store, int D, int P, const double* inv_freq_host,
+                         float* partials, float* cand_scores, int32_t* out_pages,
+                         int32_t* out_count, float* out_scores, int64_t scores_stride,
+                         cudaStream_t stream);
 
 }  // namespace rk

@@ -377,6 +377,16 @@ def random_tiny(rng: np.random.Generator, *, p: Optional[int] = None, d: int = 8
     return lay
 
 
+def with_classes(lay: Layout, class_map, retrieval=None) -> Layout:
+    """The same segments and pages under another head-class map; retrieval
+    lists empty unless given as (indptr, pages)."""
+    indptr, pages = retrieval if retrieval is not None else (
+        np.zeros(lay.n_tables + 1, np.int32), np.zeros(0, np.int32))
+    return dataclasses.replace(lay, class_map=np.asarray(class_map, dtype=np.int8),
+                               retr_indptr=np.asarray(indptr, dtype=np.int32),
+                               retr_pages=np.asarray(pages, dtype=np.int32))
+
+
 def tiny_workload(lay: Layout, seed: int = 0) -> Workload:
     return Workload("tiny", seed, lay, "cpu")
 

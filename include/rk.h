@@ -238,6 +238,60 @@ rk_status rk_selftest_bounded_wait(int32_t* device_word, int32_t wait_ms, void* 
 rk_status rk_select_visible_noalloc(const rk_dims* dims, const rk_layout* layout,
                                     const rk_visible* out, int32_t* device_error, void* stream);
 
+/* ---- retrieval page scoring (the retrieval lists of rk_layout) ----------
+ *
+ * RedKnot's pages say retrieval heads take their cached pages "by query
+ * semantics" (paooo page, "how to use" section, SELECTVISIBLESTATE) and give
+ * no rule.  These calls implement one reading, for every table (request,
+ * layer, kv head) of class RK_RETRIEVAL whose request has uncached rows:
+ *   u        = sum over the kv head's q heads of the mean query over the
+ *              table's rows (the request's uncached positions);
+ *   score_pg = <u, mean over the page's keys of R(delta) K_stored>, for each
+ *              candidate page pg: a page of a cached segment whose first
+ *              position is at most the last uncached position;
+ *   picks    = the top_k candidates by score (ties to the lower page), all
+ *              of them when there are at most top_k, in ascending page order.
+ * The picks are request-logical page numbers, the format of
+ * rk_layout.retr_pages.  Arithmetic: bf16 inputs, fp32 sums, sin / cos of
+ * the relocation angle in fp32 after an fp64 reduction modulo 2 pi. */
+
+typedef struct {
+  int64_t n_tables;
+  int64_t max_pages;       /* pages of the longest request: minimum scores_stride */
+  int64_t workspace_bytes; /* device workspace for rk_score_retrieval_pages */
+} rk_score_sizes;
+
+/* Validates dims + layout (its retrieval lists may be NULL: scoring makes
+ * them) and reports sizes.  top_k: 1 .. 64.  Host only.  Errors:
+ * RK_ERR_INVALID_ARG, RK_ERR_UNALIGNED, RK_ERR_CAPACITY (a table with more
+ * than 4096 candidate pages). */
+rk_status rk_score_query_sizes(const rk_dims* dims, const rk_layout* layout, int32_t top_k,
+                               rk_score_sizes* out);
+
+/* Scores every retrieval table's candidate pages and keeps the top_k.
+ *   q:         device bf16 [n_layers][total_tokens][Hq][D], post-RoPE (as for
+ *              rk_segpaged_prefill).
+ *   k_store:   device bf16 [n_pages][P][D], keys as stored (rotated at their
+ *              stored positions; the call relocates by each page's delta).
+ *   rope_theta: RoPE base.
+ *   out_pages: device int32 [n_tables][top_k]: the picks of table t in
+ *              out_pages[t * top_k .. + out_count[t]).
+ *   out_count: device int32 [n_tables]: picks per table (0 for other classes
+ *              and for tables without rows).
+ *   out_scores: device fp32 [n_tables][scores_stride] or NULL: the score of
+ *              every candidate page at its page number, NaN elsewhere;
+ *              scores_stride >= rk_score_sizes.max_pages.
+ *   workspace: device, >= rk_score_sizes.workspace_bytes, 256-byte aligned;
+ *              not shared with a concurrent call.
+ * Asynchronous on `stream`; the host arrays may be reused once it returns.
+ * Errors (host): RK_ERR_INVALID_ARG, RK_ERR_UNALIGNED, RK_ERR_CAPACITY,
+ * RK_ERR_CUDA. */
+rk_status rk_score_retrieval_pages(const rk_dims* dims, const rk_layout* layout, const void* q,
+                                   const void* k_store, double rope_theta, int32_t top_k,
+                                   int32_t* out_pages, int32_t* out_count, float* out_scores,
+                                   int64_t scores_stride, void* workspace,
+                                   size_t workspace_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

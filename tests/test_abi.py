@@ -156,3 +156,42 @@ def test_relocate_and_prefill_reject_on_host(lib):
     assert lib.rk_segpaged_prefill(*small_ws) == binding.RK_ERR_CAPACITY
     assert lib.rk_get_device_status(None, None, None) == E
 
+
+
+def test_score_calls_validate_on_host(lib):
+    """Retrieval page scoring: sizes follow the layout, and every argument
+    error is returned before any GPU work."""
+    E, C = binding.RK_ERR_INVALID_ARG, binding.RK_ERR_CAPACITY
+    lay = synth.cfg4().layout
+    hl = _hl(lay)
+    s = binding.score_sizes(hl, 16)
+    assert s.n_tables == lay.n_tables and s.max_pages == -(-lay.req_len(0) // lay.p)
+    assert s.workspace_bytes > 0 and s.workspace_bytes % 256 == 0
+    # the layout's retrieval lists are optional here
+    hl.layout.retr_indptr = None
+    hl.layout.retr_pages = None
+    s2 = binding.score_sizes(hl, 16)
+    assert s2.workspace_bytes == s.workspace_bytes
+    out = binding.RkScoreSizes()
+    for k in (0, 65):
+        assert lib.rk_score_query_sizes(ctypes.byref(hl.dims), ctypes.byref(hl.layout), k,
+                                        ctypes.byref(out)) == E
+    fake = ctypes.c_void_p(1 << 20)
+    # (dims, layout, q, k_store, theta, top_k, pages, count, scores, stride, ws, ws_bytes, stream)
+    args = [ctypes.byref(hl.dims), ctypes.byref(hl.layout), fake, fake, 1e6, 16, fake, fake, fake,
+            s.max_pages, fake, s.workspace_bytes, None]
+
+    def call(**kw):
+        a = list(args)
+        for i, v in kw.items():
+            a[int(i[1:])] = v
+        return lib.rk_score_retrieval_pages(*a)
+
+    assert call(a2=None) == E               # q
+    assert call(a3=None) == E               # k_store
+    assert call(a4=-1.0) == E               # theta
+    assert call(a5=0) == E                  # top_k
+    assert call(a6=None) == E               # out_pages
+    assert call(a3=ctypes.c_void_p((1 << 20) + 2)) == E  # unaligned k_store
+    assert call(a9=s.max_pages - 1) == C    # scores row too short
+    assert call(a11=s.workspace_bytes - 1) == C
