@@ -306,6 +306,38 @@ def run_reference(args, rank, world):
     return 0
 
 
+def _bench_scoring(torch, lay, q, k_store, dev, flush, stream, reps, peaks, peak_kind):
+    """rk_score_retrieval_pages on the same layer with every kv head a
+    retrieval head (its cached pages ranked against its tail queries, top
+    16): a bandwidth measurement of the scoring launches."""
+    from head_aware_paged_prefill_b200 import binding, metrics, synth
+    lay_r = synth.with_classes(lay, [synth.RETRIEVAL] * lay.hkv)
+    hl = binding.HostLayout(lay_r)
+    out = binding.ScoreOutputs(binding.score_sizes(hl, 16), 16, dev, with_scores=False)
+    for _ in range(3):
+        binding.score_retrieval_pages(hl, q, k_store, lay.theta, out)
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(reps):
+        flush()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        binding.score_retrieval_pages(hl, q, k_store, lay.theta, out)
+        b.record(stream)
+        ms.append((a, b))
+    torch.cuda.synchronize()
+    t = statistics.mean(x.elapsed_time(y) for x, y in ms)
+    nbytes = metrics.scoring_bytes(lay_r)
+    gbs = nbytes / (t * 1e-3) / 1e9
+    n_tables = int((out.count > 0).sum().item())
+    return {"bound": "hbm", "kernel": "score_query + score_pages + score_topk",
+            "workload": "the same layer, every kv head a retrieval head, top 16",
+            "tables": n_tables, "bytes": nbytes, "achieved": gbs,
+            "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+            "frac": gbs / float(peaks["hbm_gbs"]), "peak_kind": peak_kind, "us": t * 1e3,
+            "launches": 3}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -424,6 +456,8 @@ def main():
     traffic = _recorded_traffic("segpaged_prefill_kernel", wl.name)
 
     reloc = _bench_relocate(torch, lay, k, dev, flush, stream, args.reloc_reps, peaks, peak_kind)
+    scoring = _bench_scoring(torch, lay, q, k, dev, flush, stream, args.reloc_reps, peaks,
+                             peak_kind)
 
     # the other mode of the same path, timed the same way (context)
     other = "relocate" if args.mode == "fused" else "fused"
@@ -495,6 +529,7 @@ def main():
         "mode": args.mode,
         "other_mode": other_mode,
         "relocate_roofline": reloc,
+        "retrieval_scoring_roofline": scoring,
     }
     print(json.dumps(line), flush=True)
     return 0

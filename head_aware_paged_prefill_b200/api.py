@@ -27,8 +27,23 @@ from typing import Optional
 import numpy as np
 import torch
 
-from . import binding
+from . import binding, synth
 from .plan import RelocationPlan, relocation_plan
+
+
+def score_retrieval(layout, q: torch.Tensor, k_store: torch.Tensor, top_k: int = 16,
+                    stream=None):
+    """Chooses every retrieval head's cached pages on the device
+    (rk_score_retrieval_pages: the top_k pages by the score of their mean
+    relocated key against the head's mean tail query) and returns the layout
+    with those retrieval lists, plus the device outputs.  q and k_store are
+    device tensors ([n_layers][T][Hq][D] post-RoPE queries, the K pool as
+    stored).  Reading the picks back synchronises the stream."""
+    hl = binding.HostLayout(layout)
+    out = binding.ScoreOutputs(binding.score_sizes(hl, top_k), top_k, q.device)
+    binding.score_retrieval_pages(hl, q, k_store, layout.theta, out, stream)
+    indptr, pages = out.lists()
+    return synth.with_classes(layout, layout.class_map, (indptr, pages)), out
 
 
 class SegPagedPrefill:

@@ -271,7 +271,7 @@ struct ScorePlan {
   std::vector<int32_t> img;  // ScoreView followed by its arrays
   ScoreView sv{};
   int64_t max_pages = 0;     // pages of the longest request (scores row length)
-  size_t off_partials = 0, off_cand_scores = 0, total = 0;  // workspace byte offsets
+  size_t off_partials = 0, off_kbar = 0, off_urot = 0, total = 0;  // workspace offsets
 };
 
 // A copy of the layout whose retrieval lists are empty when it has none:
@@ -298,7 +298,7 @@ rk_status build_score_plan(const rk_dims* d, const rk_layout* lay, const Derived
   std::vector<ScoreTable> tables;
   std::vector<ScoreChunk> chunks;
   std::vector<ScoreCand> cands;
-  std::vector<int32_t> blocks;  // (st, first candidate) pairs
+  std::vector<ScoreRun> runs;
   std::vector<int32_t> table_map(static_cast<size_t>(dv.n_tables), -1);
   int64_t max_pages = 0;
   for (int r = 0; r < n_req; ++r) {
@@ -333,21 +333,28 @@ rk_status build_score_plan(const rk_dims* d, const rk_layout* lay, const Derived
             chunks.push_back(ScoreChunk{st_idx, a, std::min(kScoreChunkRows, rg.second - a), 0});
         st.chunk_end = static_cast<int32_t>(chunks.size());
         st.cand_begin = static_cast<int32_t>(cands.size());
+        st.run_begin = static_cast<int32_t>(runs.size());
         for (int s = dv.seg_indptr[r]; s < dv.seg_indptr[r + 1]; ++s) {
           const rk_segment& sg = lay->segments[s];
           if (!sg.cached) continue;
           const int32_t base = lay->page_base[static_cast<int64_t>(s) * dv.n_lh + lh];
+          const int32_t delta = sg.logical_start - sg.stored_pos_base;
+          const int32_t first = static_cast<int32_t>(cands.size());
           for (int pos = sg.logical_start; pos < sg.logical_start + sg.len && pos <= last_row;
                pos += P)
-            cands.push_back(ScoreCand{pos / P, base + (pos - sg.logical_start) / P,
-                                      sg.logical_start - sg.stored_pos_base, std::min(P, L - pos)});
+            cands.push_back(ScoreCand{pos / P, base + (pos - sg.logical_start) / P, delta,
+                                      std::min(P, L - pos)});
+          const int32_t last = static_cast<int32_t>(cands.size());
+          if (last == first) continue;
+          if (static_cast<int32_t>(runs.size()) > st.run_begin && runs.back().delta == delta &&
+              runs.back().cand_end == first)
+            runs.back().cand_end = last;
+          else
+            runs.push_back(ScoreRun{first, last, delta, 0});
         }
         st.cand_end = static_cast<int32_t>(cands.size());
+        st.run_end = static_cast<int32_t>(runs.size());
         if (st.cand_end - st.cand_begin > kScoreMaxCand) return RK_ERR_CAPACITY;
-        for (int c = st.cand_begin; c < st.cand_end; c += kScorePagesPerCta) {
-          blocks.push_back(st_idx);
-          blocks.push_back(c);
-        }
         table_map[static_cast<size_t>(t)] = st_idx;
         tables.push_back(st);
       }
@@ -359,22 +366,27 @@ rk_status build_score_plan(const rk_dims* d, const rk_layout* lay, const Derived
   v.n_st = static_cast<int32_t>(tables.size());
   v.n_chunks = static_cast<int32_t>(chunks.size());
   v.n_cand = static_cast<int32_t>(cands.size());
-  v.n_blocks = static_cast<int32_t>(blocks.size() / 2);
+  v.n_runs = static_cast<int32_t>(runs.size());
+  v.n_page_blocks = static_cast<int32_t>((cands.size() + kScorePagesPerCta - 1) / kScorePagesPerCta);
   v.n_tables = static_cast<int32_t>(dv.n_tables);
   v.top_k = top_k;
   v.hq = d->num_q_heads;
   v.g = g;
-  int32_t off = static_cast<int32_t>((sizeof(ScoreView) + 3) / 4);
+  // every array starts on a 16-byte boundary
+  auto al4 = [](int32_t w) { return (w + 3) & ~3; };
+  int32_t off = al4(static_cast<int32_t>((sizeof(ScoreView) + 3) / 4));
   v.off_tables = off;
-  off += static_cast<int32_t>(tables.size() * sizeof(ScoreTable) / 4);
+  off = al4(off + static_cast<int32_t>(tables.size() * sizeof(ScoreTable) / 4));
   v.off_chunks = off;
-  off += static_cast<int32_t>(chunks.size() * sizeof(ScoreChunk) / 4);
+  off = al4(off + static_cast<int32_t>(chunks.size() * sizeof(ScoreChunk) / 4));
   v.off_cand = off;
-  off += static_cast<int32_t>(cands.size() * sizeof(ScoreCand) / 4);
-  v.off_blocks = off;
-  off += static_cast<int32_t>(blocks.size());
+  off = al4(off + static_cast<int32_t>(cands.size() * sizeof(ScoreCand) / 4));
+  v.off_runs = off;
+  off = al4(off + static_cast<int32_t>(runs.size() * sizeof(ScoreRun) / 4));
+  v.off_cand_run = off;
+  off = al4(off + static_cast<int32_t>(cands.size()));
   v.off_table_map = off;
-  off += static_cast<int32_t>(table_map.size());
+  off = al4(off + static_cast<int32_t>(table_map.size()));
   v.words = off;
   out->img.assign(static_cast<size_t>(off), 0);
   int32_t* w = out->img.data();
@@ -382,12 +394,16 @@ rk_status build_score_plan(const rk_dims* d, const rk_layout* lay, const Derived
   if (!tables.empty()) std::memcpy(w + v.off_tables, tables.data(), tables.size() * sizeof(ScoreTable));
   if (!chunks.empty()) std::memcpy(w + v.off_chunks, chunks.data(), chunks.size() * sizeof(ScoreChunk));
   if (!cands.empty()) std::memcpy(w + v.off_cand, cands.data(), cands.size() * sizeof(ScoreCand));
-  if (!blocks.empty()) std::memcpy(w + v.off_blocks, blocks.data(), blocks.size() * 4);
+  if (!runs.empty()) std::memcpy(w + v.off_runs, runs.data(), runs.size() * sizeof(ScoreRun));
+  for (size_t rn = 0; rn < runs.size(); ++rn)
+    for (int x = runs[rn].cand_begin; x < runs[rn].cand_end; ++x)
+      w[v.off_cand_run + x] = static_cast<int32_t>(rn);
   if (!table_map.empty()) std::memcpy(w + v.off_table_map, table_map.data(), table_map.size() * 4);
   out->max_pages = max_pages;
   out->off_partials = align_up(4 * static_cast<size_t>(off), 256);
-  out->off_cand_scores = align_up(out->off_partials + 4 * chunks.size() * D, 256);
-  out->total = align_up(out->off_cand_scores + 4 * cands.size(), 256);
+  out->off_kbar = align_up(out->off_partials + 4 * chunks.size() * D, 256);
+  out->off_urot = align_up(out->off_kbar + 4 * cands.size() * D, 256);
+  out->total = align_up(out->off_urot + 4 * runs.size() * D, 256);
   return RK_OK;
 }
 
@@ -658,7 +674,8 @@ extern "C" rk_status rk_score_retrieval_pages(const rk_dims* dims, const rk_layo
   cudaError_t e = launch_score(reinterpret_cast<const ScoreView*>(ws), plan.sv, q, k_store,
                                dims->head_dim, dims->page_size, inv_freq,
                                reinterpret_cast<float*>(ws + plan.off_partials),
-                               reinterpret_cast<float*>(ws + plan.off_cand_scores), out_pages,
+                               reinterpret_cast<float*>(ws + plan.off_kbar),
+                               reinterpret_cast<float*>(ws + plan.off_urot), out_pages,
                                out_count, out_scores, out_scores ? scores_stride : 0, s);
   return e == cudaSuccess ? RK_OK : RK_ERR_CUDA;
 }

@@ -120,7 +120,9 @@ struct ScoreTable {  // one retrieval table that has rows
   int32_t head0;     // first q head of the kv head
   int32_t n_rows;    // computed rows (uncached positions)
   int32_t chunk_begin, chunk_end;  // its query chunks
-  int32_t cand_begin, cand_end;    // its candidate pages
+  int32_t cand_begin, cand_end;    // its candidate pages (ascending page)
+  int32_t run_begin, run_end;      // its runs of candidates sharing one delta
+  int32_t pad[2];
 };
 struct ScoreChunk {  // rows [row_begin, row_begin + n_rows) of one table
   int32_t st, row_begin, n_rows, pad;
@@ -128,20 +130,28 @@ struct ScoreChunk {  // rows [row_begin, row_begin + n_rows) of one table
 struct ScoreCand {  // a candidate page of a table
   int32_t page, phys, delta, n_valid;
 };
+struct ScoreRun {  // candidates [cand_begin, cand_end) relocated by delta
+  int32_t cand_begin, cand_end, delta, pad;
+};
 struct ScoreView {
-  int32_t n_st, n_chunks, n_cand, n_blocks, n_tables, top_k;
+  int32_t n_st, n_chunks, n_cand, n_runs, n_page_blocks, n_tables, top_k;
   int32_t hq, g;
   int32_t off_tables;     // ScoreTable[n_st]
   int32_t off_chunks;     // ScoreChunk[n_chunks]
   int32_t off_cand;       // ScoreCand[n_cand]
-  int32_t off_blocks;     // int32[n_blocks][2]: (st, first candidate) of each scoring CTA
+  int32_t off_runs;       // ScoreRun[n_runs]
+  int32_t off_cand_run;   // int32[n_cand]: run of each candidate
   int32_t off_table_map;  // int32[n_tables]: score table of a table, -1 if none
   int32_t words;
 };
 
+// One launch sums the queries of every 64-row chunk (the first n_chunks
+// CTAs) and averages the stored keys of every candidate page (the other
+// CTAs, kScorePagesPerCta pages each); a second, one CTA per table, scores
+// and ranks.
 cudaError_t launch_score(const ScoreView* sv_dev, const ScoreView& sv_host, const void* q,
                          const void* k_store, int D, int P, const double* inv_freq_host,
-                         float* partials, float* cand_scores, int32_t* out_pages,
+                         float* partials, float* kbar, float* urot, int32_t* out_pages,
                          int32_t* out_count, float* out_scores, int64_t scores_stride,
                          cudaStream_t stream);
 

@@ -7,6 +7,10 @@ form.  Algorithmic FLOPs of the attention are 4 * D per visible pair
 
 relocate_bytes(jobs, p, d): bytes an rk_relocate_rope pass must move
 (read + write of every page it touches).
+
+scoring_bytes(layout): bytes rk_score_retrieval_pages must read: the
+queries of every retrieval table's rows (all q heads of its kv head) and the
+keys of its candidate pages, each once.
 """
 from __future__ import annotations
 
@@ -61,3 +65,23 @@ def attention_flops(lay) -> int:
 
 def relocate_bytes(n_jobs: int, p: int, d: int) -> int:
     return 2 * n_jobs * p * d * 2
+
+
+def scoring_bytes(lay) -> int:
+    g = lay.hq // lay.hkv
+    P, D = lay.p, lay.d
+    total = 0
+    for r in range(lay.n_req):
+        L = lay.req_len(r)
+        unc = _uncached_mask(lay, r)
+        rows = np.nonzero(unc)[0]
+        if rows.size == 0:
+            continue
+        last = int(rows.max())
+        cand_keys = sum(min(P, L - k * P) for k in range(-(-L // P))
+                        if not unc[k * P] and k * P <= last)
+        for layer in range(lay.n_layers):
+            for kvh in range(lay.hkv):
+                if int(lay.class_map[layer * lay.hkv + kvh]) == RETRIEVAL:
+                    total += 2 * D * (g * rows.size + cand_keys)
+    return int(total)

@@ -96,3 +96,33 @@ def test_score_is_deterministic():
     b = _run(wl.layout, q, k, 16)
     assert torch.equal(a.pages, b.pages) and torch.equal(a.count, b.count)
     assert torch.equal(a.scores.view(torch.int32), b.scores.view(torch.int32))
+
+
+def test_scored_lists_drive_attention():
+    """End to end: the device picks become the layout's retrieval lists, and
+    attention over that layout (select, relocation, attention) matches the
+    oracle on the same layout (sampled rows of the retrieval head)."""
+    from head_aware_paged_prefill_b200.api import SegPagedPrefill, score_retrieval
+    from gpu_util import assert_close, oracle_rows
+    wl = synth.cfg4()
+    q, k, v = wl.materialize("cuda")
+    lay, out = score_retrieval(wl.layout, q, k, top_k=16)
+    t = lay.table_index(0, 0, 1)  # kv head 1 is the retrieval head
+    picks_ref, _ = oracle.score_pages(wl.layout, u16(q), u16(k), 16)
+    assert lay.retr_indptr[t + 1] - lay.retr_indptr[t] == 16
+    np.testing.assert_array_equal(lay.retr_pages[lay.retr_indptr[t]:lay.retr_indptr[t + 1]],
+                                  picks_ref[t])
+    pre = SegPagedPrefill(lay, "cuda")
+    o = pre.run(q, k, v)
+    torch.cuda.synchronize()
+    assert pre.status() == 0
+    g = lay.hq // lay.hkv
+    L = lay.req_len(0)
+    rng = np.random.default_rng(3)
+    rows = np.array([(0, h, int(i)) for h in range(g, 2 * g)
+                     for i in rng.integers(L - 2048, L, 12)], dtype=np.int32)
+    o_ref, _, comp = oracle_rows(lay, q.cpu(), k.cpu(), v.cpu(), rows)
+    assert comp.all()
+    idx = [torch.from_numpy(rows[:, c]).long().cuda() for c in (0, 2, 1)]
+    got = o[idx[0], idx[1], idx[2]].double().cpu().numpy()
+    assert_close(got, o_ref, "scored retrieval o")

@@ -82,3 +82,14 @@ def test_visible_pages_cfg2_counts():
     l_pages = sum(len(v) for (s, lh), v in need.items() if lh > 0 and lay.segments[s, 4])
     assert g_pages == 7 * 64          # the global head reads every cached page
     assert l_pages == 7 * 64          # each local head: the last cached segment (window 4096)
+
+
+def test_scoring_bytes_by_hand():
+    """One retrieval table: 2 cached segments of 2 pages (P 8, D 16) and a
+    10-token tail, 2 q heads: 10 rows x 2 heads of queries and 32 cached
+    keys, 2 bytes each, times D; other classes read nothing."""
+    from head_aware_paged_prefill_b200 import metrics
+    segs = [("a", 16, 3, True), ("b", 16, 9, True), ("t", 10, 0, False)]
+    lay = synth._make_layout(n_layers=1, hq=4, hkv=2, d=16, p=8, theta=1e4, requests=[segs],
+                             class_map=[synth.RETRIEVAL, synth.GLOBAL], window=8, retrieval={})
+    assert metrics.scoring_bytes(lay) == 2 * 16 * (2 * 10 + 32)
