@@ -58,7 +58,8 @@ class RkSizes(ctypes.Structure):
 
 EXPORTS = ("rk_query_sizes", "rk_select_visible", "rk_relocate_rope", "rk_segpaged_prefill",
            "rk_get_device_status", "rk_select_visible_noalloc", "rk_selftest_bounded_wait",
-           "rk_score_query_sizes", "rk_score_retrieval_pages")
+           "rk_score_query_sizes", "rk_score_retrieval_pages", "rk_decode_query_sizes",
+           "rk_segpaged_decode")
 
 _lib = None
 
@@ -82,6 +83,9 @@ def lib() -> ctypes.CDLL:
         L.rk_select_visible_noalloc.argtypes = [vp, vp, vp, vp, vp]
         L.rk_selftest_bounded_wait.argtypes = [vp, i32, vp]
         L.rk_score_query_sizes.argtypes = [vp, vp, i32, vp]
+        L.rk_decode_query_sizes.argtypes = [vp, vp, vp]
+        L.rk_segpaged_decode.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, vp,
+                                         ctypes.c_size_t, vp]
         L.rk_score_retrieval_pages.argtypes = [vp, vp, vp, vp, ctypes.c_double, i32, vp, vp, vp,
                                                i64, vp, ctypes.c_size_t, vp]
         for name in EXPORTS:
@@ -103,6 +107,10 @@ def _stream(stream) -> ctypes.c_void_p:
     if stream is None:
         stream = torch.cuda.current_stream()
     return ctypes.c_void_p(stream.cuda_stream)
+
+
+class RkDecodeSizes(ctypes.Structure):
+    _fields_ = [("max_splits", ctypes.c_int64), ("workspace_bytes", ctypes.c_int64)]
 
 
 class RkScoreSizes(ctypes.Structure):
@@ -263,3 +271,28 @@ def score_retrieval_pages(hl: HostLayout, q: torch.Tensor, k_store: torch.Tensor
         out.top_k, _ptr(out.pages), _ptr(out.count), _ptr(out.scores),
         out.stride if out.scores is not None else 0, _ptr(out.ws), out.ws.numel(),
         _stream(stream)), "rk_score_retrieval_pages")
+
+
+# ------------------------------------------------------------------ decode
+
+def decode_sizes(hl: HostLayout) -> RkDecodeSizes:
+    s = RkDecodeSizes()
+    _check(lib().rk_decode_query_sizes(ctypes.byref(hl.dims), ctypes.byref(hl.layout),
+                                       ctypes.byref(s)), "rk_decode_query_sizes")
+    return s
+
+
+def decode_workspace(sizes: RkDecodeSizes, device) -> torch.Tensor:
+    return torch.zeros(int(sizes.workspace_bytes), dtype=torch.uint8, device=torch.device(device))
+
+
+def segpaged_decode(hl: HostLayout, q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor,
+                    vis: Visible, ws: torch.Tensor, o: torch.Tensor,
+                    lse: Optional[torch.Tensor] = None, stream=None):
+    """q, o: bf16 [n_layers][n_req][Hq][D] (one row per request)."""
+    for t in (q, k_pool, v_pool, o):
+        assert t.dtype == torch.bfloat16 and t.is_contiguous()
+    _check(lib().rk_segpaged_decode(ctypes.byref(hl.dims), ctypes.byref(hl.layout), _ptr(q),
+                                    _ptr(k_pool), _ptr(v_pool), ctypes.byref(vis.struct),
+                                    float(hl.lay.softmax_scale), _ptr(o), _ptr(lse), _ptr(ws),
+                                    ws.numel(), _stream(stream)), "rk_segpaged_decode")

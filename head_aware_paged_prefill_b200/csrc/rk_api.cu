@@ -679,3 +679,104 @@ extern "C" rk_status rk_score_retrieval_pages(const rk_dims* dims, const rk_layo
                                out_count, out_scores, out_scores ? scores_stride : 0, s);
   return e == cudaSuccess ? RK_OK : RK_ERR_CUDA;
 }
+
+// ---- paged decode
+
+namespace rk {
+namespace {
+struct DecodePlan {
+  int max_splits = 0;
+  size_t off_req_len = 0, off_part_o = 0, off_part_ml = 0, total = 0;
+};
+rk_status plan_decode(const rk_dims* d, const Derived& dv, DecodePlan* out) {
+  const int g = d->num_q_heads / d->num_kv_heads;
+  if (g > kDecodeMaxG || dv.n_lh > kDecodeMaxLh) return RK_ERR_INVALID_ARG;
+  int64_t max_pages = 0;
+  for (int r = 0; r < d->n_req; ++r)
+    max_pages = std::max<int64_t>(max_pages, dv.page_prefix[r + 1] - dv.page_prefix[r]);
+  out->max_splits = static_cast<int>((max_pages + kDecodePages - 1) / kDecodePages);
+  const size_t slots = static_cast<size_t>(dv.n_tables) * out->max_splits * g;
+  // the first 256 bytes hold the device error word, then the request lengths
+  out->off_req_len = 256;
+  out->off_part_o = align_up(out->off_req_len + 4 * static_cast<size_t>(d->n_req), 256);
+  out->off_part_ml = align_up(out->off_part_o + 4 * slots * d->head_dim, 256);
+  out->total = align_up(out->off_part_ml + 8 * slots, 256);
+  return RK_OK;
+}
+}  // namespace
+}  // namespace rk
+
+extern "C" rk_status rk_decode_query_sizes(const rk_dims* dims, const rk_layout* layout,
+                                           rk_decode_sizes* out) {
+  if (!out) return RK_ERR_INVALID_ARG;
+  rk_status st = check_dims(dims);
+  if (st != RK_OK) return st;
+  Derived dv;
+  if ((st = check_layout(dims, layout, &dv)) != RK_OK) return st;
+  DecodePlan plan;
+  if ((st = plan_decode(dims, dv, &plan)) != RK_OK) return st;
+  out->max_splits = plan.max_splits;
+  out->workspace_bytes = static_cast<int64_t>(plan.total);
+  return RK_OK;
+}
+
+extern "C" rk_status rk_segpaged_decode(const rk_dims* dims, const rk_layout* layout,
+                                        const void* q, const void* k_pool, const void* v_pool,
+                                        const rk_visible* vis, float softmax_scale, void* o,
+                                        float* lse, void* workspace, size_t workspace_bytes,
+                                        void* stream) {
+  rk_status st = check_dims(dims);
+  if (st != RK_OK) return st;
+  Derived dv;
+  if ((st = check_layout(dims, layout, &dv)) != RK_OK) return st;
+  DecodePlan plan;
+  if ((st = plan_decode(dims, dv, &plan)) != RK_OK) return st;
+  if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return RK_ERR_INVALID_ARG;
+  if (!q || !k_pool || !v_pool || !vis || !o || !workspace || !vis->entries ||
+      !vis->entry_start || !vis->entry_count || !vis->ranges || !vis->range_start ||
+      !vis->range_count)
+    return RK_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k_pool, 16) || !aligned(v_pool, 16) || !aligned(o, 16) ||
+      !aligned(lse, 4) || !aligned(workspace, 256) || !aligned(vis->entries, 16))
+    return RK_ERR_INVALID_ARG;
+  if (vis->entry_capacity < dv.entry_capacity || vis->range_capacity < dv.range_capacity)
+    return RK_ERR_CAPACITY;
+  if (workspace_bytes < plan.total) return RK_ERR_CAPACITY;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  std::vector<int32_t> req_len(static_cast<size_t>(dims->n_req));
+  for (int r = 0; r < dims->n_req; ++r)
+    req_len[r] = layout->cu_seqlens[r + 1] - layout->cu_seqlens[r];
+  if (cudaMemsetAsync(ws, 0, 256, s) != cudaSuccess ||
+      cudaMemcpyAsync(ws + plan.off_req_len, req_len.data(), 4 * req_len.size(),
+                      cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return RK_ERR_CUDA;
+  DecodeLaunchArgs a{};
+  a.q = q;
+  a.k_pool = k_pool;
+  a.v_pool = v_pool;
+  a.entries = vis->entries;
+  a.entry_start = vis->entry_start;
+  a.entry_count = vis->entry_count;
+  a.ranges = vis->ranges;
+  a.range_start = vis->range_start;
+  a.range_count = vis->range_count;
+  a.req_len = reinterpret_cast<const int32_t*>(ws + plan.off_req_len);
+  a.o = o;
+  a.lse = lse;
+  a.part_o = reinterpret_cast<float*>(ws + plan.off_part_o);
+  a.part_ml = reinterpret_cast<float*>(ws + plan.off_part_ml);
+  a.n_pages = dims->n_pages;
+  a.n_req = dims->n_req;
+  a.n_layers = dims->n_layers;
+  a.hq = dims->num_q_heads;
+  a.hkv = dims->num_kv_heads;
+  a.d = dims->head_dim;
+  a.p = dims->page_size;
+  a.max_splits = plan.max_splits;
+  a.window = layout->class_window[RK_LOCAL];
+  a.softmax_scale = softmax_scale;
+  a.cls = layout->class_map;
+  a.error_word = reinterpret_cast<int32_t*>(ws);
+  return launch_decode(a, s) == cudaSuccess ? RK_OK : RK_ERR_CUDA;
+}

@@ -155,4 +155,34 @@ cudaError_t launch_score(const ScoreView* sv_dev, const ScoreView& sv_host, cons
                          int32_t* out_count, float* out_scores, int64_t scores_stride,
                          cudaStream_t stream);
 
+// ---- paged decode
+
+constexpr int kDecodePages = 32;    // pages per split of a table
+constexpr int kDecodeMaxLh = 1024;  // layers x kv heads per call
+constexpr int kDecodeMaxG = 8;      // q heads per kv head
+
+struct DecodeLaunchArgs {
+  const void* q;  // bf16 [n_layers][n_req][hq][d]
+  const void* k_pool;
+  const void* v_pool;
+  const rk_entry* entries;
+  const int32_t* entry_start;
+  const int32_t* entry_count;
+  const rk_range* ranges;
+  const int32_t* range_start;
+  const int32_t* range_count;
+  const int32_t* req_len;  // device [n_req]
+  void* o;     // bf16 [n_layers][n_req][hq][d]
+  float* lse;  // fp32 [n_layers][hq][n_req] or null
+  float* part_o;
+  float* part_ml;
+  int64_t n_pages;
+  int n_req, n_layers, hq, hkv, d, p, max_splits, window;
+  float softmax_scale;
+  const int8_t* cls;  // host [n_layers * hkv]
+  int32_t* error_word;
+};
+
+cudaError_t launch_decode(const DecodeLaunchArgs& a, cudaStream_t stream);
+
 }  // namespace rk

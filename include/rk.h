@@ -292,6 +292,46 @@ rk_status rk_score_retrieval_pages(const rk_dims* dims, const rk_layout* layout,
                                    int64_t scores_stride, void* workspace,
                                    size_t workspace_bytes, void* stream);
 
+/* ---- paged decode -------------------------------------------------------
+ *
+ * One query row per (request, layer, q head): the last position of each
+ * request, a token a decode step appended to the request's uncached tail (its
+ * K / V already in the pools).  The row attends to its table's visible keys
+ * under the class rule, exactly as the prefill's last row would: global /
+ * dense every key, local the last W keys, retrieval the uncached keys and the
+ * listed pages.  Reads relocated pools (as rk_segpaged_prefill with
+ * fuse_rope = 0) and the page tables rk_select_visible built for the same
+ * layout.  bf16 in, fp32 scores and accumulation, bf16 out. */
+
+typedef struct {
+  int64_t max_splits;      /* splits of the longest table (32 pages each) */
+  int64_t workspace_bytes; /* device workspace for rk_segpaged_decode */
+} rk_decode_sizes;
+
+/* Validates dims + layout and reports the workspace size.  Hq / Hkv <= 8 and
+ * n_layers * Hkv <= 1024.  Host only.  Errors: RK_ERR_INVALID_ARG,
+ * RK_ERR_UNALIGNED. */
+rk_status rk_decode_query_sizes(const rk_dims* dims, const rk_layout* layout,
+                                rk_decode_sizes* out);
+
+/*   q:     device bf16 [n_layers][n_req][Hq][D], the new row of each request
+ *          (post-RoPE).
+ *   k_pool, v_pool: device bf16 [n_pages][P][D], relocated.
+ *   vis:   rk_select_visible's output for `layout`.
+ *   o:     device bf16 [n_layers][n_req][Hq][D]; entries of a table whose
+ *          request's last position is not in its row set (a cached last
+ *          segment), or of an empty request, are left untouched.
+ *   lse:   device fp32 [n_layers][Hq][n_req] (natural log) or NULL.
+ *   workspace: device, >= rk_decode_sizes.workspace_bytes, 256-byte aligned;
+ *          its first word is the device error word (RK_DEV_BAD_PAGE), reset
+ *          by this call and read by rk_get_device_status.
+ * Errors (host): RK_ERR_INVALID_ARG, RK_ERR_UNALIGNED, RK_ERR_CAPACITY,
+ * RK_ERR_CUDA. */
+rk_status rk_segpaged_decode(const rk_dims* dims, const rk_layout* layout, const void* q,
+                             const void* k_pool, const void* v_pool, const rk_visible* vis,
+                             float softmax_scale, void* o, float* lse, void* workspace,
+                             size_t workspace_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
