@@ -407,6 +407,52 @@ def _mask_penalty(torch, pre, lay, q, k3_ms, reps=5):
                     "class, the same visible pairs; context for the pages' 4.9-7.6x"}
 
 
+def _bench_decode(torch, lay, pre, dev, flush, stream, reps, peaks, peak_kind, batch):
+    """rk_segpaged_decode on a batch of `batch` requests shaped like the
+    bench's layer, each on its own copy of the relocated pages (so every
+    request's keys come from HBM): one decode row per request and q head."""
+    from head_aware_paged_prefill_b200 import binding, metrics, synth
+    if lay.n_req != 1 or batch < 1:
+        return None
+    lay_b = synth.replicate_requests(lay, batch)
+    n = lay.n_pages
+    k_b = pre.k_work[:n].repeat(batch, 1, 1)
+    v_b = pre.v_work[:n].repeat(batch, 1, 1)
+    hl = binding.HostLayout(lay_b)
+    vis = binding.Visible(hl.sizes(), dev)
+    ws_sel = binding.workspace(hl.sizes(), dev)
+    binding.select_visible(hl, vis, ws_sel)
+    g = torch.Generator(device=dev).manual_seed(7)
+    q_d = torch.randn((lay.n_layers, batch, lay.hq, lay.d), generator=g, device=dev).to(torch.bfloat16)
+    o_d = torch.empty_like(q_d)
+    sizes = binding.decode_sizes(hl)
+    ws = binding.decode_workspace(sizes, dev)
+    for _ in range(3):
+        binding.segpaged_decode(hl, q_d, k_b, v_b, vis, ws, o_d)
+    torch.cuda.synchronize()
+    st = binding.device_status(ws)
+    ms = []
+    for _ in range(reps):
+        flush()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        binding.segpaged_decode(hl, q_d, k_b, v_b, vis, ws, o_d)
+        b.record(stream)
+        ms.append((a, b))
+    torch.cuda.synchronize()
+    t = statistics.mean(x.elapsed_time(y) for x, y in ms)
+    nbytes = metrics.decode_bytes(lay_b)
+    gbs = nbytes / (t * 1e-3) / 1e9
+    del k_b, v_b
+    torch.cuda.empty_cache()
+    return {"bound": "hbm", "kernel": "decode_split + decode_combine",
+            "workload": f"{batch} requests shaped like the bench's layer, own pages each, "
+                        "one decode row per request and q head",
+            "bytes": nbytes, "achieved": gbs, "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+            "frac": gbs / float(peaks["hbm_gbs"]), "peak_kind": peak_kind, "us": t * 1e3,
+            "rows_per_s": batch * lay.n_layers * lay.hq / (t * 1e-3), "device_status": st}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -421,6 +467,7 @@ def main():
     ap.add_argument("--ref-step-s", type=float, default=0.25)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-mask-penalty", action="store_true")
+    ap.add_argument("--decode-batch", type=int, default=32)
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -528,6 +575,9 @@ def main():
     reloc = _bench_relocate(torch, lay, k, dev, flush, stream, args.reloc_reps, peaks, peak_kind)
     scoring = _bench_scoring(torch, lay, q, k, dev, flush, stream, args.reloc_reps, peaks,
                              peak_kind)
+    decode = (_bench_decode(torch, lay, pre, dev, flush, stream, args.reloc_reps, peaks,
+                            peak_kind, args.decode_batch)
+              if args.mode == "relocate" else None)
     mask_penalty = (_mask_penalty(torch, pre, lay, q, k3_mean)
                     if args.mode == "relocate" and not args.no_mask_penalty else None)
 
@@ -603,6 +653,7 @@ def main():
         "relocate_roofline": reloc,
         "retrieval_scoring_roofline": scoring,
         "mask_penalty": mask_penalty,
+        "decode_roofline": decode,
     }
     print(json.dumps(line), flush=True)
     return 0

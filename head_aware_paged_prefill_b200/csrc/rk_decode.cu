@@ -9,10 +9,12 @@
 // HBM bound (every visible key and value is read once per q-head group), so
 // the kernel is a split-K flash decode on the CUDA cores:
 //   1. one CTA per (table, split of kDecodePages pages) for all G q heads of
-//      the kv head: each K and V page is staged in shared memory, the G x P
-//      scores (fp32) are masked by the class rule, an online softmax per head
-//      keeps (m, l) and the partial output in registers; the split writes
-//      (o, m, l) to the workspace;
+//      the kv head: K and V pages are staged in shared memory by cp.async,
+//      two buffers deep; each lane owns D / 32 columns (its slice of the G
+//      queries in registers), each warp a quarter of a page's keys, and the
+//      per-(key, head) partial dots are summed over the lanes 32 values per
+//      transposing butterfly; an online softmax per head keeps (m, l), each
+//      warp its share of the output; the split writes (o, m, l);
 //   2. one CTA per table merges its splits: o = sum_s o_s e^(m_s - M) / L,
 //      lse = M + ln L, written as bf16 / fp32.
 // Relocated pools are read (the cached pages' RoPE delta is applied by
@@ -52,20 +54,52 @@ struct DecodeArgs {
   int32_t* error_word;
 };
 
-// 1. one split of one table
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Sum over the 32 lanes of each of 32 values: after the call, lane l holds in
+// v[0] the total of value index l (five exchange steps, 31 shuffles).
+__device__ __forceinline__ void warp_transpose_sum(float (&v)[32], int lane) {
+#pragma unroll
+  for (int off = 16, n = 32; off >= 1; off >>= 1, n >>= 1) {
+    const bool upper = lane & off;
+#pragma unroll
+    for (int i = 0; i < n / 2; ++i) {
+      const float send = upper ? v[i] : v[i + n / 2];
+      const float keep = upper ? v[i + n / 2] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+}
+
+// 1. one split of one table.  Lane l of every warp owns columns
+// [l * CPL, (l + 1) * CPL) and holds those columns of the G queries; warp w
+// takes keys [w * KPW, (w + 1) * KPW) of each page.  Pages are staged by
+// cp.async, two buffers deep.
 template <int D, int G>
 __global__ void __launch_bounds__(kDecodeThreads)
     decode_split_kernel(const __grid_constant__ DecodeArgs a) {
-  constexpr int NO = (G * D + kDecodeThreads - 1) / kDecodeThreads;  // outputs per thread
+  constexpr int CPL = D / 32;
+  constexpr int NW = kDecodeThreads / 32;
   extern __shared__ __align__(16) uint8_t smem[];
   const int P = a.p;
-  __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(smem);
-  __nv_bfloat16* sV = sK + 64 * D;
-  float* sQ = reinterpret_cast<float*>(sV + 64 * D);  // [G][D]
-  float* sP = sQ + G * D;                             // [G][64] scores, then weights
-  float* sM = sP + G * 64;                            // [G] running max (log2 domain)
-  float* sL = sM + G;                                 // [G] running sum
-  float* sA = sL + G;                                 // [G] rescale of this page
+  const int KPW = P / NW;  // keys of a page per warp (16 at P 64, 4 at P 16)
+  __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(smem);  // [2][64][D]
+  __nv_bfloat16* sV = sK + 2 * 64 * D;                        // [2][64][D]
+  float* sP = reinterpret_cast<float*>(sV + 2 * 64 * D);       // [G][64] scores, then weights
+  float* sM = sP + G * 64;                                    // [G] running max (log2 domain)
+  float* sL = sM + G;                                         // [G] running sum
+  float* sA = sL + G;                                         // [G] rescale of this page
+  float* sO = sA + G;                                         // [NW][G][D] warp partials
   const int t = blockIdx.x, split = blockIdx.y;
   const int kvh = t % a.hkv, layer = (t / a.hkv) % a.n_layers, r = t / (a.hkv * a.n_layers);
   const int n_e = a.entry_count[t], e_first = a.entry_start[t];
@@ -77,67 +111,102 @@ __global__ void __launch_bounds__(kDecodeThreads)
   if (n_e == 0 || rc == 0 || a.ranges[a.range_start[t] + rc - 1].end != row + 1) return;
   const int cls = a.cls[layer * a.hkv + kvh];
   const int lo = cls == RK_LOCAL ? row - a.window + 1 : 0;  // first visible key
-  // this thread's outputs: x = threadIdx.x + 128 k, head x / D, column x % D
-  float acc[NO];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // this lane's columns of the G queries, scaled into the log2 domain
+  float qr[G][CPL];
 #pragma unroll
-  for (int k = 0; k < NO; ++k) acc[k] = 0.f;
-  // the G queries, scaled into the log2 domain
-  for (int x = threadIdx.x; x < G * D; x += kDecodeThreads) {
-    const int h = x / D, c = x % D;
-    const int64_t qi = ((static_cast<int64_t>(layer) * a.n_req + r) * a.hq + kvh * G + h) * D + c;
-    sQ[x] = __bfloat162float(a.q[qi]) * a.scale_log2;
-  }
+  for (int h = 0; h < G; ++h)
+#pragma unroll
+    for (int k = 0; k < CPL; ++k) {
+      const int64_t qi = ((static_cast<int64_t>(layer) * a.n_req + r) * a.hq + kvh * G + h) * D +
+                         lane * CPL + k;
+      qr[h][k] = __bfloat162float(a.q[qi]) * a.scale_log2;
+    }
+  float acc[G][CPL];
+#pragma unroll
+  for (int h = 0; h < G; ++h)
+#pragma unroll
+    for (int k = 0; k < CPL; ++k) acc[h][k] = 0.f;
   if (threadIdx.x < G) {
     sM[threadIdx.x] = -INFINITY;
     sL[threadIdx.x] = 0.f;
   }
-  __syncthreads();
   const int e_end = min(n_e, e0 + kDecodePages);
-  for (int e = e0; e < e_end; ++e) {
+  // stage page e into buffer b (16-byte chunks; a page outside the pool is
+  // not copied and is skipped below, flagged once)
+  auto stage = [&](int e, int b) {
     const rk_entry en = a.entries[e_first + e];
-    const bool ok_page = en.phys_page >= 0 && en.phys_page < a.n_pages;
-    if (!ok_page) {
-      if (threadIdx.x == 0) atomicOr(a.error_word, static_cast<int>(RK_DEV_BAD_PAGE));
-      continue;  // uniform across the CTA
-    }
-    // stage the page's K and V (16-byte chunks)
+    if (en.phys_page < 0 || en.phys_page >= a.n_pages) return;
     const uint4* gk = reinterpret_cast<const uint4*>(a.k_pool + static_cast<int64_t>(en.phys_page) * P * D);
     const uint4* gv = reinterpret_cast<const uint4*>(a.v_pool + static_cast<int64_t>(en.phys_page) * P * D);
-    uint4* k4 = reinterpret_cast<uint4*>(sK);
-    uint4* v4 = reinterpret_cast<uint4*>(sV);
+    uint4* k4 = reinterpret_cast<uint4*>(sK + b * 64 * D);
+    uint4* v4 = reinterpret_cast<uint4*>(sV + b * 64 * D);
     for (int x = threadIdx.x; x < P * D / 8; x += kDecodeThreads) {
-      k4[x] = gk[x];
-      v4[x] = gv[x];
+      cp_async16(k4 + x, gk + x);
+      cp_async16(v4 + x, gv + x);
     }
+  };
+  if (e0 < e_end) stage(e0, 0);
+  cp_async_commit();
+  for (int e = e0; e < e_end; ++e) {
+    const int b = (e - e0) & 1;
+    if (e + 1 < e_end) stage(e + 1, b ^ 1);
+    cp_async_commit();
+    cp_async_wait<1>();  // page e has landed
     __syncthreads();
-    // scores s[h][j] = q_h . k_j (log2 domain), -inf where not visible; a
-    // thread walks the columns from its own offset so the lanes of a warp
-    // read different banks of the key row
-    for (int x = threadIdx.x; x < G * P; x += kDecodeThreads) {
-      const int h = x / P, j = x % P;
-      const int pos = en.logical_pos + j;
-      float s = -INFINITY;
-      if (j < en.n_valid && pos <= row && pos >= lo) {
-        const __nv_bfloat162* kr = reinterpret_cast<const __nv_bfloat162*>(sK + j * D);
-        const float* qh = sQ + h * D;
-        float acc0 = 0.f, acc1 = 0.f;
-        const int rot = (threadIdx.x & 31) % (D / 2);
-#pragma unroll 8
-        for (int c2 = 0; c2 < D / 2; ++c2) {
-          const int cc = (c2 + rot) % (D / 2);
-          const float2 kv = __bfloat1622float2(kr[cc]);
-          acc0 = fmaf(qh[2 * cc], kv.x, acc0);
-          acc1 = fmaf(qh[2 * cc + 1], kv.y, acc1);
+    const rk_entry en = a.entries[e_first + e];
+    if (en.phys_page < 0 || en.phys_page >= a.n_pages) {
+      if (threadIdx.x == 0) atomicOr(a.error_word, static_cast<int>(RK_DEV_BAD_PAGE));
+      __syncthreads();
+      continue;  // uniform across the CTA
+    }
+    const __nv_bfloat16* kb = sK + b * 64 * D;
+    const __nv_bfloat16* vb = sV + b * 64 * D;
+    // scores of this warp's keys: partial dots over the lane's columns,
+    // summed over the lanes 32 values at a time; a group holds KG whole keys
+    // (value kk * G + h), the spare lanes zero
+    constexpr int KG = 32 / G;
+    const int j0 = warp * KPW;
+    for (int kb0 = 0; kb0 < KPW; kb0 += KG) {
+      float v[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = 0.f;
+#pragma unroll
+      for (int kk = 0; kk < KG; ++kk) {
+        if (kb0 + kk < KPW) {
+          const __nv_bfloat16* kr = kb + (j0 + kb0 + kk) * D + lane * CPL;
+          float kf[CPL];
+          if constexpr (CPL == 4) {
+            const uint2 raw = *reinterpret_cast<const uint2*>(kr);
+            const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
+            const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
+            kf[0] = x.x; kf[1] = x.y; kf[2] = y.x; kf[3] = y.y;
+          } else {
+            const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(kr));
+            kf[0] = x.x; kf[1] = x.y;
+          }
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            float d0 = 0.f;
+#pragma unroll
+            for (int k = 0; k < CPL; ++k) d0 = fmaf(qr[h][k], kf[k], d0);
+            v[kk * G + h] = d0;
+          }
         }
-        s = acc0 + acc1;
       }
-      sP[h * 64 + j] = s;
+      warp_transpose_sum(v, lane);
+      const int kk = lane / G, h = lane - kk * G;
+      if (kk < KG && kb0 + kk < KPW) {
+        const int j = j0 + kb0 + kk;
+        const int pos = en.logical_pos + j;
+        const bool vis = j < en.n_valid && pos <= row && pos >= lo;
+        sP[h * 64 + j] = vis ? v[0] : -INFINITY;
+      }
     }
     __syncthreads();
     // per head (one warp each): new running max, weights p = 2^(s - m),
     // rescale factor
-    for (int h = threadIdx.x >> 5; h < G; h += kDecodeThreads / 32) {
-      const int lane = threadIdx.x & 31;
+    for (int h = warp; h < G; h += NW) {
       float mx = -INFINITY;
       for (int j = lane; j < P; j += 32) mx = fmaxf(mx, sP[h * 64 + j]);
 #pragma unroll
@@ -146,8 +215,8 @@ __global__ void __launch_bounds__(kDecodeThreads)
       const float m_new = fmaxf(m_old, mx);
       float sum = 0.f;
       for (int j = lane; j < P; j += 32) {
-        const float s = sP[h * 64 + j];
-        const float w = s == -INFINITY ? 0.f : exp2f(s - m_new);
+        const float sc = sP[h * 64 + j];
+        const float w = sc == -INFINITY ? 0.f : exp2f(sc - m_new);
         sP[h * 64 + j] = w;
         sum += w;
       }
@@ -161,24 +230,47 @@ __global__ void __launch_bounds__(kDecodeThreads)
       }
     }
     __syncthreads();
-    // o[h] = o[h] * alpha + sum_j p[h][j] v_j
+    // this warp's share of o[h] = o[h] * alpha + sum_j p[h][j] v_j
 #pragma unroll
-    for (int k = 0; k < NO; ++k) {
-      const int x = threadIdx.x + kDecodeThreads * k;
-      if (x < G * D) {
-        const int h = x / D, c = x % D;
-        const float* ph = sP + h * 64;
-        float v = acc[k] * sA[h];
-        for (int j = 0; j < P; ++j) v = fmaf(ph[j], __bfloat162float(sV[j * D + c]), v);
-        acc[k] = v;
+    for (int h = 0; h < G; ++h) {
+      const float al = sA[h];
+#pragma unroll
+      for (int k = 0; k < CPL; ++k) acc[h][k] *= al;
+    }
+    for (int jj = 0; jj < KPW; ++jj) {
+      const int j = j0 + jj;
+      const __nv_bfloat16* vr = vb + j * D + lane * CPL;
+      float vf[CPL];
+      if constexpr (CPL == 4) {
+        const uint2 raw = *reinterpret_cast<const uint2*>(vr);
+        const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
+        const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
+        vf[0] = x.x; vf[1] = x.y; vf[2] = y.x; vf[3] = y.y;
+      } else {
+        const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(vr));
+        vf[0] = x.x; vf[1] = x.y;
+      }
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float w = sP[h * 64 + j];
+#pragma unroll
+        for (int k = 0; k < CPL; ++k) acc[h][k] = fmaf(w, vf[k], acc[h][k]);
       }
     }
-    __syncthreads();  // the page buffers are refilled next
+    __syncthreads();  // the weights and this page's buffer are reused next
   }
+  cp_async_wait<0>();
+  // the warps' partial outputs, added in warp order
 #pragma unroll
-  for (int k = 0; k < NO; ++k) {
-    const int x = threadIdx.x + kDecodeThreads * k;
-    if (x < G * D) a.part_o[part * G * D + x] = acc[k];
+  for (int h = 0; h < G; ++h)
+#pragma unroll
+    for (int k = 0; k < CPL; ++k) sO[(warp * G + h) * D + lane * CPL + k] = acc[h][k];
+  __syncthreads();
+  for (int x = threadIdx.x; x < G * D; x += kDecodeThreads) {
+    float tot = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) tot += sO[w * G * D + x];
+    a.part_o[part * G * D + x] = tot;
   }
   if (threadIdx.x < G) {
     a.part_ml[(part * G + threadIdx.x) * 2] = sM[threadIdx.x];
@@ -226,7 +318,8 @@ __global__ void __launch_bounds__(kDecodeThreads)
 
 template <int D, int G>
 cudaError_t launch_decode_typed(const DecodeArgs& a, int n_tables, cudaStream_t stream) {
-  const size_t smem = 2 * 64 * D * sizeof(__nv_bfloat16) + (G * D + G * 64 + 3 * G) * sizeof(float);
+  const size_t smem = 4 * 64 * D * sizeof(__nv_bfloat16) +
+                      (G * 64 + 3 * G + (kDecodeThreads / 32) * G * D) * sizeof(float);
   auto split = decode_split_kernel<D, G>;
   cudaError_t e = cudaFuncSetAttribute(split, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));

@@ -8,6 +8,10 @@ form.  Algorithmic FLOPs of the attention are 4 * D per visible pair
 relocate_bytes(jobs, p, d): bytes an rk_relocate_rope pass must move
 (read + write of every page it touches).
 
+decode_bytes(layout): bytes rk_segpaged_decode must move: the keys and
+values visible to every table's last row (once per kv head), the new rows'
+queries and the outputs.
+
 scoring_bytes(layout): bytes rk_score_retrieval_pages must read: the
 queries of every retrieval table's rows (all q heads of its kv head) and the
 keys of its candidate pages, each once.
@@ -85,3 +89,34 @@ def scoring_bytes(lay) -> int:
                 if int(lay.class_map[layer * lay.hkv + kvh]) == RETRIEVAL:
                     total += 2 * D * (g * rows.size + cand_keys)
     return int(total)
+
+
+def decode_bytes(lay) -> int:
+    """Last-row attention of every table whose last position is a row."""
+    g = lay.hq // lay.hkv
+    W = int(lay.class_window[LOCAL])
+    P, D = lay.p, lay.d
+    keys = 0
+    for r in range(lay.n_req):
+        L = lay.req_len(r)
+        if L == 0:
+            continue
+        unc = _uncached_mask(lay, r)
+        i = L - 1
+        for layer in range(lay.n_layers):
+            for kvh in range(lay.hkv):
+                c = int(lay.class_map[layer * lay.hkv + kvh])
+                if c in (LOCAL, RETRIEVAL) and not unc[i]:
+                    continue
+                if c == LOCAL:
+                    keys += min(L, W)
+                elif c == RETRIEVAL:
+                    t = lay.table_index(r, layer, kvh)
+                    pages = np.unique(lay.retr_pages[lay.retr_indptr[t]:lay.retr_indptr[t + 1]])
+                    pages = pages[(pages >= 0) & (pages * P < L)]
+                    pages = pages[~unc[pages * P]]
+                    keys += int(unc.sum()) + sum(min(P, L - int(k) * P) for k in pages)
+                else:
+                    keys += L
+    rows = sum(1 for r in range(lay.n_req) if lay.req_len(r) > 0) * lay.n_layers * lay.hq
+    return int(2 * D * 2 * keys + 2 * 2 * D * rows)

@@ -387,6 +387,26 @@ def with_classes(lay: Layout, class_map, retrieval=None) -> Layout:
                                retr_pages=np.asarray(pages, dtype=np.int32))
 
 
+def replicate_requests(lay: Layout, n: int) -> Layout:
+    """n requests with the segments and retrieval lists of a one-request
+    layout, each on its own copy of the pages (request r's pages follow the
+    pool r times over)."""
+    assert lay.n_req == 1
+    seg = np.asarray(lay.segments, dtype=np.int32)
+    segs = np.concatenate([np.column_stack([np.full(seg.shape[0], r, np.int32), seg[:, 1:]])
+                           for r in range(n)]).astype(np.int32)
+    pb = np.concatenate([np.asarray(lay.page_base, np.int64) + r * lay.n_pages
+                         for r in range(n)]).astype(np.int32)
+    L = lay.req_len(0)
+    # every request keeps the retrieval lists of the original request's tables
+    counts = np.diff(np.asarray(lay.retr_indptr, np.int64))
+    indptr = np.concatenate([[0], np.cumsum(np.tile(counts, n))]).astype(np.int32)
+    pages = np.tile(np.asarray(lay.retr_pages, np.int32), n)
+    return dataclasses.replace(lay, n_req=n, n_pages=lay.n_pages * n, segments=segs,
+                               page_base=pb, cu_seqlens=(np.arange(n + 1) * L).astype(np.int32),
+                               retr_indptr=indptr, retr_pages=pages, kv_page_scale=None)
+
+
 def tiny_workload(lay: Layout, seed: int = 0) -> Workload:
     return Workload("tiny", seed, lay, "cpu")
 

@@ -93,3 +93,20 @@ def test_scoring_bytes_by_hand():
     lay = synth._make_layout(n_layers=1, hq=4, hkv=2, d=16, p=8, theta=1e4, requests=[segs],
                              class_map=[synth.RETRIEVAL, synth.GLOBAL], window=8, retrieval={})
     assert metrics.scoring_bytes(lay) == 2 * 16 * (2 * 10 + 32)
+
+
+def test_decode_bytes_by_hand():
+    """One request of 40 tokens (2 cached pages of 8 + a 24-token tail), P 8,
+    D 16, 2 q heads per kv head: a global head reads 40 keys, a local head
+    (W 8) 8, a retrieval head the tail (24) plus its listed cached page (8);
+    K and V, 2 bytes each, plus the queries and outputs of 6 rows."""
+    from head_aware_paged_prefill_b200 import metrics
+    segs = [("a", 16, 3, True), ("t", 24, 0, False)]
+    lay = synth._make_layout(n_layers=1, hq=6, hkv=3, d=16, p=8, theta=1e4, requests=[segs],
+                             class_map=[synth.GLOBAL, synth.LOCAL, synth.RETRIEVAL], window=8,
+                             retrieval={2: [1]})
+    keys = 40 + 8 + (24 + 8)
+    assert metrics.decode_bytes(lay) == 2 * 16 * 2 * keys + 2 * 2 * 16 * 6
+    rep = synth.replicate_requests(lay, 3)
+    assert rep.n_req == 3 and rep.n_pages == 3 * lay.n_pages and rep.total_tokens == 120
+    assert metrics.decode_bytes(rep) == 3 * metrics.decode_bytes(lay)
