@@ -1,28 +1,34 @@
 // SegPaged decode: one query row per (request, layer, q head), the last
 // position of each request, over the per-head page tables rk_select_visible
 // built (RedKnot pages: the SegPagedAttention runtime serves the per-head
-// visible windows; paooo page, "how to use": generation streams after the
-// prefill).  A decode step appends a token to each request's uncached tail;
-// its row attends to the table's visible keys under the class rule, as the
-// prefill's last row does.
+// visible windows; paooo page, "application scenarios": in streaming
+// generation the local heads keep reading their recent paged KV).  A decode
+// step appends a token to each request's uncached tail; its row attends to
+// the table's visible keys under the class rule, as the prefill's last row
+// does.
 //
-// HBM bound (every visible key and value is read once per q-head group), so
-// the kernel is a split-K flash decode on the CUDA cores:
-//   1. one CTA per (table, split of kDecodePages pages) for all G q heads of
-//      the kv head: K and V pages are staged in shared memory by cp.async,
-//      two buffers deep; each lane owns D / 32 columns (its slice of the G
-//      queries in registers), each warp a quarter of a page's keys, and the
-//      per-(key, head) partial dots are summed over the lanes 32 values per
-//      transposing butterfly; an online softmax per head keeps (m, l), each
-//      warp its share of the output; the split writes (o, m, l);
-//   2. one CTA per table merges its splits: o = sum_s o_s e^(m_s - M) / L,
-//      lse = M + ln L, written as bf16 / fp32.
+// HBM bound: every visible key and value is read once per kv head, for all
+// G q heads of the group.  Split-K flash decode:
+//   1. one CTA per (table, split of kDecodePages pages); each warp streams
+//      its own 16-key slices through a private cp.async ring and runs
+//      Q K^T and P V of the GQA group as warp-level bf16 MMAs (the G heads
+//      are the rows of a 16-row tile), with its own online softmax; the
+//      warps merge once at the end and the split writes (o, m, l);
+//   2. one CTA per table merges its splits: o = sum_s o_s 2^(m_s - M) / L,
+//      lse = (M + log2 L) ln 2, written as bf16 / fp32.
+// The MMAs are there to cut instruction issue (the CUDA-core form of the
+// same dot products issued ~5x more instructions per byte and reached a
+// third of the HBM bandwidth); the bound stays the HBM stream.  Warp-level
+// MMAs rather than tcgen05: a 16-row tile already wastes 16 / G of the
+// rows, tcgen05's smallest tile has 64, and per-warp tiles keep the warps
+// independent.
 // Relocated pools are read (the cached pages' RoPE delta is applied by
 // rk_relocate_rope beforehand), so the entry's delta is not used here.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <cstdint>
 
 #include "rk_internal.h"
 
@@ -31,6 +37,7 @@ namespace rk {
 namespace {
 
 constexpr int kDecodeThreads = 128;
+constexpr int kDecodeStages = 3;  // ring depth of each warp
 
 struct DecodeArgs {
   const __nv_bfloat16* q;  // [n_layers][n_req][hq][d]
@@ -66,44 +73,110 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// Sum over the 32 lanes of each of 32 values: after the call, lane l holds in
-// v[0] the total of value index l (five exchange steps, 31 shuffles).
-__device__ __forceinline__ void warp_transpose_sum(float (&v)[32], int lane) {
-#pragma unroll
-  for (int off = 16, n = 32; off >= 1; off >>= 1, n >>= 1) {
-    const bool upper = lane & off;
-#pragma unroll
-    for (int i = 0; i < n / 2; ++i) {
-      const float send = upper ? v[i] : v[i + n / 2];
-      const float keep = upper ? v[i + n / 2] : v[i];
-      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-    }
-  }
+__device__ __forceinline__ uint32_t shared_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-// 1. one split of one table.  Lane l of every warp owns columns
-// [l * CPL, (l + 1) * CPL) and holds those columns of the G queries; warp w
-// takes keys [w * KPW, (w + 1) * KPW) of each page.  Pages are staged by
-// cp.async, two buffers deep.
+// Four 8x8 bf16 matrices from shared memory; lanes 8i..8i+7 address the
+// rows of matrix i, and lane l receives row l / 4, columns 2 (l % 4) + {0, 1}
+// of each (.trans: row and column swapped).
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
+
+// c (16 x 8, fp32) += A (16 x 16, bf16) B (16 x 8, bf16).  A's rows 8..15 are
+// zero here (they would be q heads G + 8 and up), so only its fragments for
+// rows 0..7 are passed.
+__device__ __forceinline__ void mma_rows8(float (&c)[4], uint32_t a0, uint32_t a2, uint32_t b0,
+                                          uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// The entries a decode row reads: from the first whose last key is at or
+// after lo (entries are in ascending logical_pos; a local table's list covers
+// the windows of all its rows, the decode row needs only its own) to the
+// table's end.  A warp-wide search: each round probes 32 entries and keeps
+// the interval between the last probe before lo and the first after it.
+// Every lane returns the same index.
+__device__ __forceinline__ int first_entry_at(const rk_entry* en, int n, int lo, int lane) {
+  int a = 0, b = n;  // the answer lies in [a, b] (b = n: no such entry)
+  while (a < b) {
+    const int step = (b - a + 30) / 31;  // probe 31 sits at or past b
+    const int p = a + lane * step;
+    bool at = true;
+    if (p < b) {
+      const rk_entry e = en[p];
+      at = e.logical_pos + e.n_valid - 1 >= lo;
+    }
+    const int f = __ffs(__ballot_sync(0xffffffffu, at)) - 1;
+    if (f == 0) return a;
+    const int nb = min(a + f * step, b);
+    a = a + (f - 1) * step + 1;
+    b = nb;
+  }
+  return b;
+}
+
+// This table's decode entries [first, n_e) cut into n_split balanced splits
+// of at most kDecodePages pages (`per` each, the last one shorter).
+struct DecodeSplits {
+  int first, n_split, per;
+};
+__device__ __forceinline__ DecodeSplits decode_splits(const DecodeArgs& a, int t, int cls, int lo,
+                                                      int lane) {
+  const int n_e = a.entry_count[t];
+  DecodeSplits d;
+  d.first = cls == RK_LOCAL && lo > 0 ? first_entry_at(a.entries + a.entry_start[t], n_e, lo, lane)
+                                      : 0;
+  const int n_vis = n_e - d.first;
+  d.n_split = (n_vis + kDecodePages - 1) / kDecodePages;
+  d.per = d.n_split > 0 ? (n_vis + d.n_split - 1) / d.n_split : 0;
+  return d;
+}
+
+// 1. one split of one table.  The split's pages are cut into 16-key slices
+// (P / 16 per page); warp w takes slices w, w + NW, ... and streams them
+// through its own ring of kDecodeStages shared-memory buffers by cp.async,
+// so the warps never wait for one another inside the loop.  Per slice:
+//   S (G x 16) = Q K^T and O += P V as m16n8k16 bf16 MMAs with fp32
+//   accumulators, the G q heads of the kv head as the rows (padded to 16);
+//   an online softmax per head in the warp (row max over the 4 lanes that
+//   hold a row).
+// Rows of K and V are stored with their 16-byte chunks permuted (chunk c of
+// key k at c ^ (k & 7)), so that the eight rows each ldmatrix reads fall in
+// distinct banks.  At the end the warps' (m, l, o) are merged in shared
+// memory and the split writes (o, m, l).
 template <int D, int G>
 __global__ void __launch_bounds__(kDecodeThreads)
     decode_split_kernel(const __grid_constant__ DecodeArgs a) {
-  constexpr int CPL = D / 32;
   constexpr int NW = kDecodeThreads / 32;
-  extern __shared__ __align__(16) uint8_t smem[];
+  constexpr int KS = D / 16;      // 16-column steps of Q K^T; pairs of 8-column tiles of P V
+  constexpr int CHUNKS = D / 8;   // 16-byte chunks of a key row
+  constexpr int SLICE = 16 * D;   // elements of one slice of K (or V)
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gq = lane >> 2, tq = lane & 3;  // fragment row (q head) and column pair
   const int P = a.p;
-  const int KPW = P / NW;  // keys of a page per warp (16 at P 64, 4 at P 16)
-  __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(smem);  // [2][64][D]
-  __nv_bfloat16* sV = sK + 2 * 64 * D;                        // [2][64][D]
-  float* sP = reinterpret_cast<float*>(sV + 2 * 64 * D);       // [G][64] scores, then weights
-  float* sM = sP + G * 64;                                    // [G] running max (log2 domain)
-  float* sL = sM + G;                                         // [G] running sum
-  float* sA = sL + G;                                         // [G] rescale of this page
-  float* sO = sA + G;                                         // [NW][G][D] warp partials
   const int t = blockIdx.x, split = blockIdx.y;
   const int kvh = t % a.hkv, layer = (t / a.hkv) % a.n_layers, r = t / (a.hkv * a.n_layers);
   const int n_e = a.entry_count[t], e_first = a.entry_start[t];
-  const int e0 = split * kDecodePages;
   const int64_t part = static_cast<int64_t>(t) * a.max_splits + split;
   const int row = a.req_len[r] - 1;  // the request's last position
   // the row must belong to the table's row set (else the combine skips it too)
@@ -111,170 +184,168 @@ __global__ void __launch_bounds__(kDecodeThreads)
   if (n_e == 0 || rc == 0 || a.ranges[a.range_start[t] + rc - 1].end != row + 1) return;
   const int cls = a.cls[layer * a.hkv + kvh];
   const int lo = cls == RK_LOCAL ? row - a.window + 1 : 0;  // first visible key
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // this lane's columns of the G queries, scaled into the log2 domain
-  float qr[G][CPL];
+  const DecodeSplits ds = decode_splits(a, t, cls, lo, lane);
+  if (split >= ds.n_split) return;
+  const int e0 = ds.first + split * ds.per;
+  const int spp = P / 16;
+  const int n_slices = (min(n_e, e0 + ds.per) - e0) * spp;
+  const int my_n = warp < n_slices ? (n_slices - warp + NW - 1) / NW : 0;
+  __nv_bfloat16* ring =
+      reinterpret_cast<__nv_bfloat16*>(smem) + warp * (kDecodeStages * 2 * SLICE);
+  // Q as the A operand, rows = q heads: columns 16 ks + 2 tq (+8) of head gq
+  uint32_t qa[KS][2];
+  {
+    const bool real = gq < G;
+    const uint32_t* q32 = reinterpret_cast<const uint32_t*>(
+        a.q + ((static_cast<int64_t>(layer) * a.n_req + r) * a.hq + kvh * G + (real ? gq : 0)) * D);
 #pragma unroll
-  for (int h = 0; h < G; ++h)
-#pragma unroll
-    for (int k = 0; k < CPL; ++k) {
-      const int64_t qi = ((static_cast<int64_t>(layer) * a.n_req + r) * a.hq + kvh * G + h) * D +
-                         lane * CPL + k;
-      qr[h][k] = __bfloat162float(a.q[qi]) * a.scale_log2;
+    for (int ks = 0; ks < KS; ++ks) {
+      qa[ks][0] = real ? q32[ks * 8 + tq] : 0u;
+      qa[ks][1] = real ? q32[ks * 8 + 4 + tq] : 0u;
     }
-  float acc[G][CPL];
-#pragma unroll
-  for (int h = 0; h < G; ++h)
-#pragma unroll
-    for (int k = 0; k < CPL; ++k) acc[h][k] = 0.f;
-  if (threadIdx.x < G) {
-    sM[threadIdx.x] = -INFINITY;
-    sL[threadIdx.x] = 0.f;
   }
-  const int e_end = min(n_e, e0 + kDecodePages);
-  // stage page e into buffer b (16-byte chunks; a page outside the pool is
-  // not copied and is skipped below, flagged once)
-  auto stage = [&](int e, int b) {
-    const rk_entry en = a.entries[e_first + e];
+  // stage this warp's i-th slice into ring buffer i % kDecodeStages (a page
+  // outside the pool is not copied and is skipped below, flagged once)
+  auto stage = [&](int i) {
+    const int sg = warp + NW * i;
+    const rk_entry en = a.entries[e_first + e0 + sg / spp];
     if (en.phys_page < 0 || en.phys_page >= a.n_pages) return;
-    const uint4* gk = reinterpret_cast<const uint4*>(a.k_pool + static_cast<int64_t>(en.phys_page) * P * D);
-    const uint4* gv = reinterpret_cast<const uint4*>(a.v_pool + static_cast<int64_t>(en.phys_page) * P * D);
-    uint4* k4 = reinterpret_cast<uint4*>(sK + b * 64 * D);
-    uint4* v4 = reinterpret_cast<uint4*>(sV + b * 64 * D);
-    for (int x = threadIdx.x; x < P * D / 8; x += kDecodeThreads) {
-      cp_async16(k4 + x, gk + x);
-      cp_async16(v4 + x, gv + x);
+    const int64_t base = (static_cast<int64_t>(en.phys_page) * P + (sg % spp) * 16) * D;
+    const uint4* gk = reinterpret_cast<const uint4*>(a.k_pool + base);
+    const uint4* gv = reinterpret_cast<const uint4*>(a.v_pool + base);
+    uint4* sk = reinterpret_cast<uint4*>(ring + (i % kDecodeStages) * 2 * SLICE);
+    uint4* sv = sk + SLICE / 8;
+#pragma unroll
+    for (int u = 0; u < 16 * CHUNKS / 32; ++u) {
+      const int x = lane + 32 * u, key = x / CHUNKS, c = x % CHUNKS;
+      const int dst = key * CHUNKS + (c ^ (key & 7));
+      cp_async16(sk + dst, gk + x);
+      cp_async16(sv + dst, gv + x);
     }
   };
-  if (e0 < e_end) stage(e0, 0);
-  cp_async_commit();
-  for (int e = e0; e < e_end; ++e) {
-    const int b = (e - e0) & 1;
-    if (e + 1 < e_end) stage(e + 1, b ^ 1);
+#pragma unroll
+  for (int i = 0; i < kDecodeStages - 1; ++i) {
+    if (i < my_n) stage(i);
     cp_async_commit();
-    cp_async_wait<1>();  // page e has landed
-    __syncthreads();
-    const rk_entry en = a.entries[e_first + e];
+  }
+  float acc[2 * KS][4];
+#pragma unroll
+  for (int n = 0; n < 2 * KS; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+  float m_run = -INFINITY;  // row gq's running max (log2 domain)
+  float l_run = 0.f;        // this lane's share of row gq's running sum
+  // ldmatrix row addresses: for K, matrices (keys 0-7 | 8-15) x (chunk 2ks | 2ks+1);
+  // for V (transposed), (keys 0-7 | 8-15) x (chunk 2np | 2np+1)
+  const int k_key = ((lane >> 4) << 3) | (lane & 7), k_c = (lane >> 3) & 1;
+  const int v_key = (((lane >> 3) & 1) << 3) | (lane & 7), v_c = lane >> 4;
+  for (int i = 0; i < my_n; ++i) {
+    if (i + kDecodeStages - 1 < my_n) stage(i + kDecodeStages - 1);
+    cp_async_commit();
+    cp_async_wait<kDecodeStages - 1>();  // slice i has landed (this lane's copies)
+    __syncwarp();                        // ... and every lane's
+    const int sg = warp + NW * i;
+    const rk_entry en = a.entries[e_first + e0 + sg / spp];
     if (en.phys_page < 0 || en.phys_page >= a.n_pages) {
-      if (threadIdx.x == 0) atomicOr(a.error_word, static_cast<int>(RK_DEV_BAD_PAGE));
-      __syncthreads();
-      continue;  // uniform across the CTA
+      if (lane == 0) atomicOr(a.error_word, static_cast<int>(RK_DEV_BAD_PAGE));
+      continue;  // nothing was read from this buffer
     }
-    const __nv_bfloat16* kb = sK + b * 64 * D;
-    const __nv_bfloat16* vb = sV + b * 64 * D;
-    // scores of this warp's keys: partial dots over the lane's columns,
-    // summed over the lanes 32 values at a time; a group holds KG whole keys
-    // (value kk * G + h), the spare lanes zero
-    constexpr int KG = 32 / G;
-    const int j0 = warp * KPW;
-    for (int kb0 = 0; kb0 < KPW; kb0 += KG) {
-      float v[32];
+    const int k0 = (sg % spp) * 16;
+    const uint32_t sk = shared_addr(ring + (i % kDecodeStages) * 2 * SLICE);
+    const uint32_t sv = sk + SLICE * 2;
+    float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = 0.f;
+    for (int ks = 0; ks < KS; ++ks) {
+      uint32_t b[4];
+      const int c = 2 * ks + k_c;
+      ldsm_x4(sk + (k_key * CHUNKS + (c ^ (k_key & 7))) * 16, b);
+      mma_rows8(s[0], qa[ks][0], qa[ks][1], b[0], b[1]);
+      mma_rows8(s[1], qa[ks][0], qa[ks][1], b[2], b[3]);
+    }
+    // lane holds S[gq][8 nt + 2 tq + cc]
+    float sc[2][2];
+    float mx = -INFINITY;
 #pragma unroll
-      for (int kk = 0; kk < KG; ++kk) {
-        if (kb0 + kk < KPW) {
-          const __nv_bfloat16* kr = kb + (j0 + kb0 + kk) * D + lane * CPL;
-          float kf[CPL];
-          if constexpr (CPL == 4) {
-            const uint2 raw = *reinterpret_cast<const uint2*>(kr);
-            const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
-            const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
-            kf[0] = x.x; kf[1] = x.y; kf[2] = y.x; kf[3] = y.y;
-          } else {
-            const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(kr));
-            kf[0] = x.x; kf[1] = x.y;
-          }
+    for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-          for (int h = 0; h < G; ++h) {
-            float d0 = 0.f;
-#pragma unroll
-            for (int k = 0; k < CPL; ++k) d0 = fmaf(qr[h][k], kf[k], d0);
-            v[kk * G + h] = d0;
-          }
-        }
-      }
-      warp_transpose_sum(v, lane);
-      const int kk = lane / G, h = lane - kk * G;
-      if (kk < KG && kb0 + kk < KPW) {
-        const int j = j0 + kb0 + kk;
+      for (int cc = 0; cc < 2; ++cc) {
+        const int j = k0 + nt * 8 + 2 * tq + cc;  // key within the page
         const int pos = en.logical_pos + j;
         const bool vis = j < en.n_valid && pos <= row && pos >= lo;
-        sP[h * 64 + j] = vis ? v[0] : -INFINITY;
+        sc[nt][cc] = vis ? s[nt][cc] * a.scale_log2 : -INFINITY;
+        mx = fmaxf(mx, sc[nt][cc]);
       }
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    const float m_new = fmaxf(m_run, mx);
+    const float m_use = m_new == -INFINITY ? 0.f : m_new;
+    const float alpha = exp2f(m_run - m_use);
+    float p[2][2];
+    float psum = 0.f;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        p[nt][cc] = exp2f(sc[nt][cc] - m_use);
+        psum += p[nt][cc];
+      }
+    l_run = l_run * alpha + psum;
+    m_run = m_new;
+    // P as the A operand: row gq, keys 2 tq (+8) of the slice
+    const uint32_t pa0 = pack_bf16x2(p[0][0], p[0][1]);
+    const uint32_t pa2 = pack_bf16x2(p[1][0], p[1][1]);
+#pragma unroll
+    for (int n = 0; n < 2 * KS; ++n) {
+      acc[n][0] *= alpha;
+      acc[n][1] *= alpha;
     }
-    __syncthreads();
-    // per head (one warp each): new running max, weights p = 2^(s - m),
-    // rescale factor
-    for (int h = warp; h < G; h += NW) {
-      float mx = -INFINITY;
-      for (int j = lane; j < P; j += 32) mx = fmaxf(mx, sP[h * 64 + j]);
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      const float m_old = sM[h];
-      const float m_new = fmaxf(m_old, mx);
-      float sum = 0.f;
-      for (int j = lane; j < P; j += 32) {
-        const float sc = sP[h * 64 + j];
-        const float w = sc == -INFINITY ? 0.f : exp2f(sc - m_new);
-        sP[h * 64 + j] = w;
-        sum += w;
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-      if (lane == 0) {
-        const float alpha = m_old == -INFINITY ? 0.f : exp2f(m_old - m_new);
-        sA[h] = alpha;
-        sM[h] = m_new;
-        sL[h] = sL[h] * alpha + sum;
-      }
+    for (int np = 0; np < KS; ++np) {
+      uint32_t b[4];
+      const int c = 2 * np + v_c;
+      ldsm_x4_trans(sv + (v_key * CHUNKS + (c ^ (v_key & 7))) * 16, b);
+      mma_rows8(acc[2 * np], pa0, pa2, b[0], b[1]);
+      mma_rows8(acc[2 * np + 1], pa0, pa2, b[2], b[3]);
     }
-    __syncthreads();
-    // this warp's share of o[h] = o[h] * alpha + sum_j p[h][j] v_j
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const float al = sA[h];
-#pragma unroll
-      for (int k = 0; k < CPL; ++k) acc[h][k] *= al;
-    }
-    for (int jj = 0; jj < KPW; ++jj) {
-      const int j = j0 + jj;
-      const __nv_bfloat16* vr = vb + j * D + lane * CPL;
-      float vf[CPL];
-      if constexpr (CPL == 4) {
-        const uint2 raw = *reinterpret_cast<const uint2*>(vr);
-        const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
-        const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
-        vf[0] = x.x; vf[1] = x.y; vf[2] = y.x; vf[3] = y.y;
-      } else {
-        const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(vr));
-        vf[0] = x.x; vf[1] = x.y;
-      }
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float w = sP[h * 64 + j];
-#pragma unroll
-        for (int k = 0; k < CPL; ++k) acc[h][k] = fmaf(w, vf[k], acc[h][k]);
-      }
-    }
-    __syncthreads();  // the weights and this page's buffer are reused next
+    __syncwarp();  // the buffer is restaged next iteration
   }
   cp_async_wait<0>();
-  // the warps' partial outputs, added in warp order
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+  __syncthreads();  // every warp is done with its ring: reuse it for the merge
+  float* sO = reinterpret_cast<float*>(smem);  // [NW][G][D]
+  float* sML = sO + NW * G * D;                // [NW][G][2]
+  if (gq < G) {
 #pragma unroll
-  for (int h = 0; h < G; ++h)
-#pragma unroll
-    for (int k = 0; k < CPL; ++k) sO[(warp * G + h) * D + lane * CPL + k] = acc[h][k];
+    for (int n = 0; n < 2 * KS; ++n) {
+      sO[(warp * G + gq) * D + n * 8 + 2 * tq] = acc[n][0];
+      sO[(warp * G + gq) * D + n * 8 + 2 * tq + 1] = acc[n][1];
+    }
+    if (tq == 0) {
+      sML[(warp * G + gq) * 2] = m_run;
+      sML[(warp * G + gq) * 2 + 1] = l_run;
+    }
+  }
   __syncthreads();
   for (int x = threadIdx.x; x < G * D; x += kDecodeThreads) {
-    float tot = 0.f;
+    const int h = x / D;
+    float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < NW; ++w) tot += sO[w * G * D + x];
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, sML[(w * G + h) * 2]);
+    float tot = 0.f, L = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < NW; ++w) {
+        const float m = sML[(w * G + h) * 2];
+        if (m == -INFINITY) continue;
+        const float f = exp2f(m - M);
+        tot += sO[w * G * D + x] * f;
+        L += sML[(w * G + h) * 2 + 1] * f;
+      }
+    }
     a.part_o[part * G * D + x] = tot;
-  }
-  if (threadIdx.x < G) {
-    a.part_ml[(part * G + threadIdx.x) * 2] = sM[threadIdx.x];
-    a.part_ml[(part * G + threadIdx.x) * 2 + 1] = sL[threadIdx.x];
+    if (x % D == 0) {
+      a.part_ml[(part * G + h) * 2] = M;
+      a.part_ml[(part * G + h) * 2 + 1] = L;
+    }
   }
 }
 
@@ -285,12 +356,15 @@ __global__ void __launch_bounds__(kDecodeThreads)
   const int t = blockIdx.x;
   const int kvh = t % a.hkv, layer = (t / a.hkv) % a.n_layers, r = t / (a.hkv * a.n_layers);
   const int n_e = a.entry_count[t];
+  const int row = a.req_len[r] - 1;
   {
     const int rc = a.range_count[t];
-    if (n_e == 0 || rc == 0 || a.ranges[a.range_start[t] + rc - 1].end != a.req_len[r])
+    if (n_e == 0 || rc == 0 || a.ranges[a.range_start[t] + rc - 1].end != row + 1)
       return;  // the request's last position is not a row of this table
   }
-  const int n_split = (n_e + kDecodePages - 1) / kDecodePages;
+  const int cls = a.cls[layer * a.hkv + kvh];
+  const int lo = cls == RK_LOCAL ? row - a.window + 1 : 0;
+  const int n_split = decode_splits(a, t, cls, lo, threadIdx.x & 31).n_split;
   const int64_t base = static_cast<int64_t>(t) * a.max_splits;
   for (int x = threadIdx.x; x < G * D; x += kDecodeThreads) {
     const int h = x / D, c = x % D;
@@ -318,8 +392,10 @@ __global__ void __launch_bounds__(kDecodeThreads)
 
 template <int D, int G>
 cudaError_t launch_decode_typed(const DecodeArgs& a, int n_tables, cudaStream_t stream) {
-  const size_t smem = 4 * 64 * D * sizeof(__nv_bfloat16) +
-                      (G * 64 + 3 * G + (kDecodeThreads / 32) * G * D) * sizeof(float);
+  constexpr int NW = kDecodeThreads / 32;
+  constexpr size_t ring = static_cast<size_t>(NW) * kDecodeStages * 2 * 16 * D * sizeof(__nv_bfloat16);
+  constexpr size_t merge = static_cast<size_t>(NW) * G * (D + 2) * sizeof(float);
+  const size_t smem = ring > merge ? ring : merge;
   auto split = decode_split_kernel<D, G>;
   cudaError_t e = cudaFuncSetAttribute(split, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
