@@ -78,7 +78,10 @@ def _recorded_traffic(kernel: str, workload: str):
     with open(p) as f:
         d = json.load(f)
     e = d.get(kernel, {})
-    if e.get("source_hash") != _kernel_hash(kernel) or e.get("workload") != workload:
+    # a later source state counts only where its device code was checked
+    # byte-identical to the captured one (recorded beside the figure)
+    hashes = {e.get("source_hash")} | {x["source_hash"] for x in e.get("same_device_code", [])}
+    if _kernel_hash(kernel) not in hashes or e.get("workload") != workload:
         return None
     return e.get("dram_bytes_per_launch")
 

@@ -157,7 +157,7 @@ cudaError_t launch_score(const ScoreView* sv_dev, const ScoreView& sv_host, cons
 
 // ---- paged decode
 
-constexpr int kDecodePages = 32;    // pages per split of a table
+constexpr int kDecodePages = 64;    // pages per split of a table
 constexpr int kDecodeMaxLh = 1024;  // layers x kv heads per call
 constexpr int kDecodeMaxG = 8;      // q heads per kv head
 

@@ -63,6 +63,10 @@ def _load():
                                         ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                         ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
         lib.ora_score_pages.restype = ctypes.c_int
+        lib.ora_importance.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                       ctypes.c_double, ctypes.c_double, ctypes.c_int,
+                                       ctypes.c_int, ctypes.c_void_p]
+        lib.ora_importance.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -188,6 +192,45 @@ def score_pages(lay, q_u16: np.ndarray, k_pool_u16: np.ndarray, top_k: int = 16,
     with ThreadPoolExecutor(_threads(threads)) as ex:
         list(ex.map(one, list(_tables(lay))))
     return picks, scores
+
+
+# ------------------------------------------------- attention importance
+
+def importance(lay, q_u16: np.ndarray, k_pool_u16: np.ndarray, threads=None) -> np.ndarray:
+    """fp64 token importance [n_layers][T] (the reading is stated in
+    ``ora_importance``): per request and layer, the prefill's softmax weights
+    summed over q heads and computed rows.  q: bf16 bits [n_layers][T][Hq][D];
+    k_pool: bf16 bits [n_pages][P][D] (stored, not relocated)."""
+    lib = _load()
+    pref = _ProblemRef(lay)
+    q = np.ascontiguousarray(q_u16.view(np.uint16))
+    k = np.ascontiguousarray(k_pool_u16.view(np.uint16))
+    T = int(lay.cu_seqlens[-1])
+    out = np.zeros((lay.n_layers, T), dtype=np.float64)
+
+    def one(args):
+        r, layer = args
+        L = lay.req_len(r)
+        if L == 0:
+            return
+        buf = np.zeros(L, dtype=np.float64)
+        lib.ora_importance(pref.ptr, q.ctypes.data, k.ctypes.data, float(lay.theta),
+                           float(lay.softmax_scale), r, layer, buf.ctypes.data)
+        c0 = int(lay.cu_seqlens[r])
+        out[layer, c0:c0 + L] = buf
+
+    jobs = [(r, layer) for r in range(lay.n_req) for layer in range(lay.n_layers)]
+    with ThreadPoolExecutor(_threads(threads)) as ex:
+        list(ex.map(one, jobs))
+    return out
+
+
+def select_tokens(imp, top_k: int) -> np.ndarray:
+    """The top_k positions by importance, ties to the lower position, in
+    ascending order (all positions when there are at most top_k)."""
+    vals = [float(x) for x in imp]
+    ranked = sorted(range(len(vals)), key=lambda j: (-vals[j], j))
+    return np.array(sorted(ranked[:max(int(top_k), 0)]), dtype=np.int32)
 
 
 def _uncached_ranges(lay, r) -> List[Tuple[int, int]]:

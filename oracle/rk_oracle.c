@@ -543,3 +543,79 @@ int ora_score_pages(const ora_problem* pr, const uint16_t* q, const uint16_t* k_
   table_close(&t);
   return n_out;
 }
+
+/* ------------------------------------------------- attention importance */
+
+/* Token importance for the sparse FFN.  The RedKnot pages send the tokens with
+ * the highest attention scores through the dense FFN and the rest along the
+ * residual path (README "About", Elastic Sparsity / Sparse FFN; paooo page,
+ * "main functions" and "core advantages"), without a formula.  The reading
+ * implemented here, for request r and one layer:
+ *   I(j) = sum over the layer's q heads h, and over the rows i that the
+ *          table of h's kv head computes, of the softmax weight
+ *          P_h(i, j) = exp(scale * q_h(i) . K'_j - lse_h(i)),
+ *          zero where j is not visible to i,
+ * with K'_j = R(delta_j) K_stored_j the relocated key and lse_h(i) the
+ * row's log-sum-exp over its visible keys: the weight the prefill's own
+ * attention gives key j at row i, summed.  Each row's weights sum to 1, so
+ * the I(j) add up to the number of computed (q head, row) pairs.
+ * q: bf16 [n_layers][T][hq][d]; k_pool: bf16 [n_pages][p][d]; imp_out [L].
+ * fp64 throughout; each row's softmax by definition (max-subtracted). */
+int ora_importance(const ora_problem* pr, const uint16_t* q, const uint16_t* k_pool,
+                   double theta, double scale, int r, int layer, double* imp_out) {
+  int L = req_len(pr, r), d = pr->d, P = pr->p, hh = d / 2;
+  int g = pr->hq / pr->hkv, T = pr->cu_seqlens[pr->n_req];
+  for (int j = 0; j < L; ++j) imp_out[j] = 0.0;
+  double* kr = (double*)malloc(sizeof(double) * ((size_t)L * d + 1));
+  double* s = (double*)malloc(sizeof(double) * ((size_t)L + 1));
+  double* qd = (double*)malloc(sizeof(double) * d);
+  for (int kvh = 0; kvh < pr->hkv; ++kvh) {
+    ora_table t;
+    table_open(&t, pr, r, layer, kvh);
+    int lh = layer * pr->hkv + kvh;
+    /* relocated keys of the whole request for this kv head */
+    for (int j = 0; j < L; ++j) {
+      int sgi = t.seg_of[j];
+      const int32_t* sg = pr->seg + 5 * sgi;
+      int off = j - sg[1];
+      int page = pr->page_base[(size_t)sgi * pr->n_layers * pr->hkv + lh] + off / P;
+      int dpos = sg[1] - sg[3];
+      const uint16_t* ks = k_pool + ((size_t)page * P + off % P) * d;
+      double* kj = kr + (size_t)j * d;
+      for (int m = 0; m < hh; ++m) {
+        double a = (double)dpos * pow(theta, -2.0 * (double)m / (double)d);
+        double x0 = bf16_to_double(ks[m]), x1 = bf16_to_double(ks[m + hh]);
+        kj[m] = x0 * cos(a) - x1 * sin(a);
+        kj[m + hh] = x0 * sin(a) + x1 * cos(a);
+      }
+    }
+    for (int hg = 0; hg < g; ++hg) {
+      int h = kvh * g + hg;
+      for (int i = 0; i < L; ++i) {
+        if (!is_row(&t, i)) continue;
+        const uint16_t* qrow = q + (((size_t)layer * T + pr->cu_seqlens[r] + i) * pr->hq + h) * d;
+        for (int c = 0; c < d; ++c) qd[c] = bf16_to_double(qrow[c]);
+        double mx = -INFINITY;
+        for (int j = 0; j < L; ++j) {
+          if (!visible(&t, i, j)) { s[j] = -INFINITY; continue; }
+          double acc = 0.0;
+          for (int c = 0; c < d; ++c) acc += qd[c] * kr[(size_t)j * d + c];
+          s[j] = acc * scale;
+          if (s[j] > mx) mx = s[j];
+        }
+        if (mx == -INFINITY) continue;
+        double sum = 0.0;
+        for (int j = 0; j < L; ++j)
+          if (s[j] > -INFINITY) sum += exp(s[j] - mx);
+        double lse = mx + log(sum);
+        for (int j = 0; j < L; ++j)
+          if (s[j] > -INFINITY) imp_out[j] += exp(s[j] - lse);
+      }
+    }
+    table_close(&t);
+  }
+  free(kr);
+  free(s);
+  free(qd);
+  return 0;
+}

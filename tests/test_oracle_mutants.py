@@ -13,6 +13,7 @@ import pytest
 import oracle
 import test_oracle_pins as pins
 import test_oracle_scoring as scoring
+import test_oracle_importance as importance
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "rk_oracle.c")
 
@@ -41,6 +42,15 @@ MUTANTS = {
                          "if (best < 0 || scores_out[pg] >= scores_out[best]) best = pg;"),
     "score_uncached_candidates": ("if (t.uncached[j0] || j0 > last_row) continue;",
                                   "if (j0 > last_row) continue;"),
+    # attention importance
+    "importance_unnormalised": ("if (s[j] > -INFINITY) imp_out[j] += exp(s[j] - lse);",
+                                "if (s[j] > -INFINITY) imp_out[j] += exp(s[j] - mx);"),
+    "importance_wrong_head": ("int h = kvh * g + hg;", "int h = hg;"),
+    "importance_shift_sign": ("int dpos = sg[1] - sg[3];", "int dpos = sg[3] - sg[1];"),
+    "importance_sin_sign": ("kj[m] = x0 * cos(a) - x1 * sin(a);",
+                            "kj[m] = x0 * cos(a) + x1 * sin(a);"),
+    "importance_unscaled": ("s[j] = acc * scale;\n          if (s[j] > mx) mx = s[j];\n        }\n        if (mx == -INFINITY) continue;",
+                            "s[j] = acc;\n          if (s[j] > mx) mx = s[j];\n        }\n        if (mx == -INFINITY) continue;"),
 }
 
 PIN_CALLS = [
@@ -56,6 +66,9 @@ PIN_CALLS = [
     scoring.test_planted_pages_win,
     scoring.test_few_candidates_all_picked_and_other_tables_empty,
     scoring.test_ties_go_to_the_lower_page,
+    importance.test_importance_is_dense_softmax_column_sums_cfg1,
+    importance.test_importance_is_dense_softmax_column_sums_retrieval,
+    importance.test_zero_keys_give_harmonic_sums,
 ]
 
 
