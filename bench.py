@@ -456,6 +456,46 @@ def _bench_decode(torch, lay, pre, dev, flush, stream, reps, peaks, peak_kind, b
             "rows_per_s": batch * lay.n_layers * lay.hq / (t * 1e-3), "device_status": st}
 
 
+def _bench_importance(torch, lay, q, k, v, dev, flush, stream, reps, peaks, peak_kind):
+    """rk_attention_importance on the bench's layer after its prefill (with
+    lse): every visible (q head, row, key) pair's weight exp(s - lse) summed
+    per token, then the top L/4 tokens.  One exp per visible pair and a
+    QK^T product: bound by the exp unit (16 results per clock per SM), the
+    roofline given here."""
+    from head_aware_paged_prefill_b200 import metrics
+    from head_aware_paged_prefill_b200.api import SegPagedPrefill
+    pre = SegPagedPrefill(lay, dev, with_lse=True)
+    pre.load(q, k, v)
+    pre.compute()
+    top_k = max(lay.req_len(r) for r in range(lay.n_req)) // 4
+    for _ in range(3):
+        pre.attention_importance(top_k)
+    torch.cuda.synchronize()
+    st = pre.importance_status()
+    ms = []
+    for _ in range(reps):
+        flush()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        pre.attention_importance(top_k)
+        b.record(stream)
+        ms.append((a, b))
+    torch.cuda.synchronize()
+    t = statistics.mean(x.elapsed_time(y) for x, y in ms)
+    pairs = metrics.visible_pairs(lay)
+    sm_mhz = float(peaks.get("sm_max_mhz", 1965.0))
+    exp_peak = 148 * 16 * sm_mhz * 1e6 / 1e9  # G exp / s
+    achieved = pairs / (t * 1e-3) / 1e9
+    del pre
+    torch.cuda.empty_cache()
+    return {"bound": "alu", "kernel": "importance_colsum + importance_select",
+            "workload": f"the bench's layer, top {top_k} tokens", "pairs": pairs,
+            "achieved": achieved, "peak": exp_peak, "unit": "Gexp/s",
+            "frac": achieved / exp_peak, "peak_kind": "derived: 148 SMs x 16 ex2 / clock x max SM clock",
+            "us": t * 1e3, "qk_tflops": 2 * lay.d * pairs / (t * 1e-3) / 1e12,
+            "device_status": st}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -471,6 +511,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-mask-penalty", action="store_true")
     ap.add_argument("--decode-batch", type=int, default=32)
+    ap.add_argument("--no-importance", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -581,6 +622,9 @@ def main():
     decode = (_bench_decode(torch, lay, pre, dev, flush, stream, args.reloc_reps, peaks,
                             peak_kind, args.decode_batch)
               if args.mode == "relocate" else None)
+    importance = (_bench_importance(torch, lay, q, k, v, dev, flush, stream, args.reloc_reps,
+                                    peaks, peak_kind)
+                  if args.mode == "relocate" and not args.no_importance else None)
     mask_penalty = (_mask_penalty(torch, pre, lay, q, k3_mean)
                     if args.mode == "relocate" and not args.no_mask_penalty else None)
 
@@ -657,6 +701,7 @@ def main():
         "retrieval_scoring_roofline": scoring,
         "mask_penalty": mask_penalty,
         "decode_roofline": decode,
+        "importance_roofline": importance,
     }
     print(json.dumps(line), flush=True)
     return 0

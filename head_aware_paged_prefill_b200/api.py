@@ -168,6 +168,38 @@ class SegPagedPrefill:
         if k3_events is not None:
             k3_events[1].record(s)
 
+    def attention_importance(self, top_k: int, stream=None):
+        """Token importance for the sparse FFN from the last compute()
+        (rk_attention_importance: the attention weights each token received,
+        summed over q heads and computed rows, and the top_k tokens per
+        (request, layer)).  Needs relocate mode (relocated K pool) and
+        with_lse=True.  Returns device tensors (importance [n_layers][T] fp32,
+        tokens [n_layers][n_req][top_k] int32, token_count [n_layers][n_req]
+        int32), reused across calls with the same top_k."""
+        if self.mode != "relocate" or self.lse is None:
+            raise ValueError("attention_importance needs mode='relocate' and with_lse=True")
+        lay = self.layout
+        key = int(top_k)
+        if getattr(self, "_imp", None) is None or self._imp[0] != key:
+            sizes = binding.importance_sizes(self.hl)
+            self._imp = (key, binding.importance_workspace(sizes, self.device),
+                         torch.empty((lay.n_layers, lay.total_tokens), dtype=torch.float32,
+                                     device=self.device),
+                         torch.empty((lay.n_layers, lay.n_req, max(key, 1)), dtype=torch.int32,
+                                     device=self.device),
+                         torch.empty((lay.n_layers, lay.n_req), dtype=torch.int32,
+                                     device=self.device))
+        _, ws, imp, tokens, count = self._imp
+        b = self._sets[0]
+        binding.attention_importance(self.hl, b["q"], b["k_work"], self.vis, self.lse, ws, imp,
+                                     key, tokens if key > 0 else None, count if key > 0 else None,
+                                     stream)
+        return imp, tokens, count
+
+    def importance_status(self) -> int:
+        """Device error word of the last attention_importance call."""
+        return binding.device_status(self._imp[1])
+
     def run(self, q, k_pool, v_pool, out: str = "device", host_out: Optional[torch.Tensor] = None):
         self.load(q, k_pool, v_pool)
         self.compute()

@@ -59,7 +59,7 @@ class RkSizes(ctypes.Structure):
 EXPORTS = ("rk_query_sizes", "rk_select_visible", "rk_relocate_rope", "rk_segpaged_prefill",
            "rk_get_device_status", "rk_select_visible_noalloc", "rk_selftest_bounded_wait",
            "rk_score_query_sizes", "rk_score_retrieval_pages", "rk_decode_query_sizes",
-           "rk_segpaged_decode")
+           "rk_segpaged_decode", "rk_importance_query_sizes", "rk_attention_importance")
 
 _lib = None
 
@@ -88,6 +88,9 @@ def lib() -> ctypes.CDLL:
                                          ctypes.c_size_t, vp]
         L.rk_score_retrieval_pages.argtypes = [vp, vp, vp, vp, ctypes.c_double, i32, vp, vp, vp,
                                                i64, vp, ctypes.c_size_t, vp]
+        L.rk_importance_query_sizes.argtypes = [vp, vp, vp]
+        L.rk_attention_importance.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.c_float, i32, vp,
+                                              vp, vp, vp, ctypes.c_size_t, vp]
         for name in EXPORTS:
             getattr(L, name).restype = i32
         _lib = L
@@ -111,6 +114,10 @@ def _stream(stream) -> ctypes.c_void_p:
 
 class RkDecodeSizes(ctypes.Structure):
     _fields_ = [("max_splits", ctypes.c_int64), ("workspace_bytes", ctypes.c_int64)]
+
+
+class RkImportanceSizes(ctypes.Structure):
+    _fields_ = [("max_blocks", ctypes.c_int64), ("workspace_bytes", ctypes.c_int64)]
 
 
 class RkScoreSizes(ctypes.Structure):
@@ -296,3 +303,36 @@ def segpaged_decode(hl: HostLayout, q: torch.Tensor, k_pool: torch.Tensor, v_poo
                                     _ptr(k_pool), _ptr(v_pool), ctypes.byref(vis.struct),
                                     float(hl.lay.softmax_scale), _ptr(o), _ptr(lse), _ptr(ws),
                                     ws.numel(), _stream(stream)), "rk_segpaged_decode")
+
+
+def importance_sizes(hl: HostLayout) -> RkImportanceSizes:
+    s = RkImportanceSizes()
+    _check(lib().rk_importance_query_sizes(ctypes.byref(hl.dims), ctypes.byref(hl.layout),
+                                           ctypes.byref(s)), "rk_importance_query_sizes")
+    return s
+
+
+def importance_workspace(sizes: RkImportanceSizes, device) -> torch.Tensor:
+    return torch.zeros(int(sizes.workspace_bytes), dtype=torch.uint8, device=torch.device(device))
+
+
+def attention_importance(hl: HostLayout, q: torch.Tensor, k_pool: torch.Tensor, vis: Visible,
+                         lse: torch.Tensor, ws: torch.Tensor, importance: torch.Tensor,
+                         top_k: int = 0, tokens: Optional[torch.Tensor] = None,
+                         token_count: Optional[torch.Tensor] = None, stream=None):
+    """q: bf16 [n_layers][T][Hq][D]; k_pool: relocated bf16 [n_pages][P][D];
+    lse: fp32 [n_layers][Hq][T] from the prefill; importance: fp32
+    [n_layers][T]; tokens: int32 [n_layers][n_req][top_k] and token_count:
+    int32 [n_layers][n_req], or both None."""
+    for t in (q, k_pool):
+        assert t.dtype == torch.bfloat16 and t.is_contiguous()
+    for t in (lse, importance):
+        assert t.dtype == torch.float32 and t.is_contiguous()
+    for t in (tokens, token_count):
+        assert t is None or (t.dtype == torch.int32 and t.is_contiguous())
+    _check(lib().rk_attention_importance(ctypes.byref(hl.dims), ctypes.byref(hl.layout), _ptr(q),
+                                         _ptr(k_pool), ctypes.byref(vis.struct), _ptr(lse),
+                                         float(hl.lay.softmax_scale), int(top_k),
+                                         _ptr(importance), _ptr(tokens), _ptr(token_count),
+                                         _ptr(ws), ws.numel(), _stream(stream)),
+           "rk_attention_importance")

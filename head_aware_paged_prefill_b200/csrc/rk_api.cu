@@ -780,3 +780,122 @@ extern "C" rk_status rk_segpaged_decode(const rk_dims* dims, const rk_layout* la
   a.error_word = reinterpret_cast<int32_t*>(ws);
   return launch_decode(a, s) == cudaSuccess ? RK_OK : RK_ERR_CUDA;
 }
+
+// ---- attention importance (sparse FFN token selection)
+
+namespace rk {
+namespace {
+struct ImportancePlan {
+  int max_blocks = 0, n_chunks = 0;
+  size_t off_cu = 0, off_part = 0, part_bytes = 0, total = 0;
+};
+rk_status plan_importance(const rk_dims* d, const rk_layout* lay, const Derived& dv,
+                          ImportancePlan* out) {
+  const int g = d->num_q_heads / d->num_kv_heads;
+  if (g > kImpMaxG || dv.n_lh > kImpMaxLh) return RK_ERR_INVALID_ARG;
+  int64_t max_pages = 0;
+  for (int r = 0; r < d->n_req; ++r)
+    max_pages = std::max<int64_t>(max_pages, dv.page_prefix[r + 1] - dv.page_prefix[r]);
+  const int64_t keys = max_pages * d->page_size;
+  const int64_t blocks = (keys + kImpKeysPerCta - 1) / kImpKeysPerCta;
+  if (blocks > 65535) return RK_ERR_CAPACITY;
+  out->max_blocks = static_cast<int>(blocks);
+  int64_t max_len = 0;
+  for (int r = 0; r < d->n_req; ++r)
+    max_len = std::max<int64_t>(max_len, lay->cu_seqlens[r + 1] - lay->cu_seqlens[r]);
+  const int64_t rows_per_chunk = kImpChunkCols / g;
+  const int64_t chunks = std::max<int64_t>(1, (max_len + rows_per_chunk - 1) / rows_per_chunk);
+  if (chunks > 65535) return RK_ERR_CAPACITY;
+  out->n_chunks = static_cast<int>(chunks);
+  // the first 256 bytes hold the device error word, then cu_seqlens, then the
+  // per-(layer, kv head, row chunk, token) partial sums
+  out->off_cu = 256;
+  out->off_part = align_up(out->off_cu + 4 * static_cast<size_t>(d->n_req + 1), 256);
+  out->part_bytes = 4 * static_cast<size_t>(d->n_layers) * d->num_kv_heads * out->n_chunks *
+                    static_cast<size_t>(d->total_tokens);
+  out->total = align_up(out->off_part + out->part_bytes, 256);
+  return RK_OK;
+}
+}  // namespace
+}  // namespace rk
+
+extern "C" rk_status rk_importance_query_sizes(const rk_dims* dims, const rk_layout* layout,
+                                               rk_importance_sizes* out) {
+  if (!out) return RK_ERR_INVALID_ARG;
+  rk_status st = check_dims(dims);
+  if (st != RK_OK) return st;
+  Derived dv;
+  if ((st = check_layout(dims, layout, &dv)) != RK_OK) return st;
+  ImportancePlan plan;
+  if ((st = plan_importance(dims, layout, dv, &plan)) != RK_OK) return st;
+  out->max_blocks = plan.max_blocks;
+  out->workspace_bytes = static_cast<int64_t>(plan.total);
+  return RK_OK;
+}
+
+extern "C" rk_status rk_attention_importance(const rk_dims* dims, const rk_layout* layout,
+                                             const void* q, const void* k_pool,
+                                             const rk_visible* vis, const float* lse,
+                                             float softmax_scale, int32_t top_k,
+                                             float* importance, int32_t* tokens,
+                                             int32_t* token_count, void* workspace,
+                                             size_t workspace_bytes, void* stream) {
+  rk_status st = check_dims(dims);
+  if (st != RK_OK) return st;
+  Derived dv;
+  if ((st = check_layout(dims, layout, &dv)) != RK_OK) return st;
+  ImportancePlan plan;
+  if ((st = plan_importance(dims, layout, dv, &plan)) != RK_OK) return st;
+  if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale) || top_k < 0)
+    return RK_ERR_INVALID_ARG;
+  if (!q || !k_pool || !vis || !lse || !importance || !workspace || !vis->entries ||
+      !vis->entry_start || !vis->entry_count || !vis->ranges || !vis->range_start ||
+      !vis->range_count)
+    return RK_ERR_INVALID_ARG;
+  if (top_k > 0 && (!tokens) != (!token_count)) return RK_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k_pool, 16) || !aligned(lse, 4) || !aligned(importance, 4) ||
+      !aligned(tokens, 4) || !aligned(token_count, 4) || !aligned(workspace, 256) ||
+      !aligned(vis->entries, 16))
+    return RK_ERR_INVALID_ARG;
+  if (vis->entry_capacity < dv.entry_capacity || vis->range_capacity < dv.range_capacity)
+    return RK_ERR_CAPACITY;
+  if (workspace_bytes < plan.total) return RK_ERR_CAPACITY;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (cudaMemsetAsync(ws, 0, 256, s) != cudaSuccess ||
+      cudaMemcpyAsync(ws + plan.off_cu, layout->cu_seqlens, 4 * static_cast<size_t>(dims->n_req + 1),
+                      cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemsetAsync(ws + plan.off_part, 0, plan.part_bytes, s) != cudaSuccess)
+    return RK_ERR_CUDA;
+  ImportanceLaunchArgs a{};
+  a.q = q;
+  a.k_pool = k_pool;
+  a.entries = vis->entries;
+  a.entry_start = vis->entry_start;
+  a.entry_count = vis->entry_count;
+  a.ranges = vis->ranges;
+  a.range_start = vis->range_start;
+  a.range_count = vis->range_count;
+  a.cu = reinterpret_cast<const int32_t*>(ws + plan.off_cu);
+  a.lse = lse;
+  a.part = reinterpret_cast<float*>(ws + plan.off_part);
+  a.importance = importance;
+  a.tokens = tokens;
+  a.token_count = token_count;
+  a.n_pages = dims->n_pages;
+  a.n_req = dims->n_req;
+  a.n_layers = dims->n_layers;
+  a.hq = dims->num_q_heads;
+  a.hkv = dims->num_kv_heads;
+  a.d = dims->head_dim;
+  a.p = dims->page_size;
+  a.total_tokens = dims->total_tokens;
+  a.window = layout->class_window[RK_LOCAL];
+  a.top_k = top_k;
+  a.max_blocks = plan.max_blocks;
+  a.n_chunks = plan.n_chunks;
+  a.softmax_scale = softmax_scale;
+  a.cls = layout->class_map;
+  a.error_word = reinterpret_cast<int32_t*>(ws);
+  return launch_importance(a, s) == cudaSuccess ? RK_OK : RK_ERR_CUDA;
+}

@@ -185,4 +185,34 @@ struct DecodeLaunchArgs {
 
 cudaError_t launch_decode(const DecodeLaunchArgs& a, cudaStream_t stream);
 
+// ---- attention importance (sparse FFN token selection)
+constexpr int kImpKeysPerCta = 128;  // keys of one table per column-sum CTA
+constexpr int kImpChunkCols = 8192;  // (row, q head) columns per row chunk: 8192 / G rows
+constexpr int kImpMaxLh = 1024;      // layers x kv heads per call
+constexpr int kImpMaxG = 8;          // q heads per kv head
+
+struct ImportanceLaunchArgs {
+  const void* q;       // bf16 [n_layers][T][hq][d], the prefill's queries
+  const void* k_pool;  // bf16 [n_pages][p][d], relocated
+  const rk_entry* entries;
+  const int32_t* entry_start;
+  const int32_t* entry_count;
+  const rk_range* ranges;
+  const int32_t* range_start;
+  const int32_t* range_count;
+  const int32_t* cu;   // device [n_req + 1]
+  const float* lse;    // fp32 [n_layers][hq][T], natural log (the prefill's)
+  float* part;         // fp32 [n_layers][hkv][n_chunks][T], zeroed by the caller
+  float* importance;   // fp32 [n_layers][T]
+  int32_t* tokens;     // [n_layers][n_req][top_k] or null
+  int32_t* token_count;  // [n_layers][n_req] or null
+  int64_t n_pages;
+  int n_req, n_layers, hq, hkv, d, p, total_tokens, window, top_k, max_blocks, n_chunks;
+  float softmax_scale;
+  const int8_t* cls;   // host [n_layers * hkv]
+  int32_t* error_word;
+};
+
+cudaError_t launch_importance(const ImportanceLaunchArgs& a, cudaStream_t stream);
+
 }  // namespace rk

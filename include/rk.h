@@ -332,6 +332,56 @@ rk_status rk_segpaged_decode(const rk_dims* dims, const rk_layout* layout, const
                              float softmax_scale, void* o, float* lse, void* workspace,
                              size_t workspace_bytes, void* stream);
 
+/* ---- attention importance (sparse FFN token selection) ------------------
+ *
+ * RedKnot runs the dense FFN only on the tokens with the highest attention
+ * scores; the others take the residual path (README "About", Elastic
+ * Sparsity / Sparse FFN; paooo page, "main functions").  The pages give no
+ * formula.  This call computes, per request r and layer:
+ *   I(j) = sum over the layer's q heads h and the rows i that the table of
+ *          h's kv head computes of exp(scale q_h(i) . K'_j - lse_h(i)),
+ *          0 where j is not visible to i (the class rules of the prefill),
+ * i.e. the prefill's attention weights summed over heads and rows, and picks
+ * the top_k tokens by I (ties to the lower position), in ascending order.
+ * Each computed row's weights sum to one, so the I(j) of a (request, layer)
+ * add up to the number of its computed (q head, row) pairs.  fp32
+ * accumulation; I is >= 0 (a NaN lse ranks its tokens first). */
+
+typedef struct {
+  int64_t max_blocks;      /* column-sum CTAs per table (128 keys each) */
+  int64_t workspace_bytes; /* device workspace for rk_attention_importance */
+} rk_importance_sizes;
+
+/* Validates dims + layout and reports the workspace size.  Hq / Hkv <= 8,
+ * n_layers * Hkv <= 1024, and a request of at most 65535 * 128 keys.  Host
+ * only.  Errors: RK_ERR_INVALID_ARG, RK_ERR_UNALIGNED, RK_ERR_CAPACITY. */
+rk_status rk_importance_query_sizes(const rk_dims* dims, const rk_layout* layout,
+                                    rk_importance_sizes* out);
+
+/*   q:      device bf16 [n_layers][T][Hq][D], the prefill's queries.
+ *   k_pool: device bf16 [n_pages][P][D], relocated (as rk_segpaged_prefill
+ *           with fuse_rope = 0 reads it).
+ *   vis:    rk_select_visible's output for `layout`.
+ *   lse:    device fp32 [n_layers][Hq][T], natural log: rk_segpaged_prefill's
+ *           lse for the same q, pools, layout and softmax_scale.
+ *   top_k:  >= 0; tokens picked per (request, layer), min(top_k, L_r).
+ *   importance: device fp32 [n_layers][T], written for every position.
+ *   tokens: device int32 [n_layers][n_req][top_k], request-local positions,
+ *           ascending, the first token_count entries of each row written;
+ *           token_count: device int32 [n_layers][n_req].  Both NULL skips
+ *           the selection.
+ *   workspace: device, >= rk_importance_sizes.workspace_bytes, 256-byte
+ *           aligned; its first word is the device error word
+ *           (RK_DEV_BAD_PAGE), reset by this call and read by
+ *           rk_get_device_status.
+ * Errors (host): RK_ERR_INVALID_ARG, RK_ERR_UNALIGNED, RK_ERR_CAPACITY,
+ * RK_ERR_CUDA. */
+rk_status rk_attention_importance(const rk_dims* dims, const rk_layout* layout, const void* q,
+                                  const void* k_pool, const rk_visible* vis, const float* lse,
+                                  float softmax_scale, int32_t top_k, float* importance,
+                                  int32_t* tokens, int32_t* token_count, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -195,3 +195,43 @@ def test_score_calls_validate_on_host(lib):
     assert call(a3=ctypes.c_void_p((1 << 20) + 2)) == E  # unaligned k_store
     assert call(a9=s.max_pages - 1) == C    # scores row too short
     assert call(a11=s.workspace_bytes - 1) == C
+
+
+def test_importance_calls_validate_on_host(lib):
+    """Attention importance: sizes follow the layout, and argument errors are
+    returned before any GPU work."""
+    E, C = binding.RK_ERR_INVALID_ARG, binding.RK_ERR_CAPACITY
+    lay = synth.cfg1().layout
+    hl = _hl(lay)
+    s = binding.importance_sizes(hl)
+    keys = -(-lay.req_len(0) // lay.p) * lay.p
+    assert s.max_blocks == -(-keys // 128)
+    T = int(lay.cu_seqlens[-1])
+    assert s.workspace_bytes >= 256 + 4 * lay.n_layers * lay.hkv * T
+    assert s.workspace_bytes % 256 == 0
+    sz = hl.sizes()
+    fake = ctypes.c_void_p(1 << 20)
+    vis = binding.RkVisible(fake.value, fake.value, fake.value, fake.value, fake.value,
+                            fake.value, sz.entry_capacity, sz.range_capacity)
+    # (dims, layout, q, k_pool, vis, lse, scale, top_k, importance, tokens,
+    #  token_count, ws, ws_bytes, stream)
+    args = [ctypes.byref(hl.dims), ctypes.byref(hl.layout), fake, fake, ctypes.byref(vis), fake,
+            0.125, 8, fake, fake, fake, fake, s.workspace_bytes, None]
+
+    def call(**kw):
+        a = list(args)
+        for i, v in kw.items():
+            a[int(i[1:])] = v
+        return lib.rk_attention_importance(*a)
+
+    assert call(a2=None) == E                # q
+    assert call(a5=None) == E                # lse
+    assert call(a6=0.0) == E                 # softmax scale
+    assert call(a7=-1) == E                  # top_k
+    assert call(a8=None) == E                # importance
+    assert call(a10=None) == E               # tokens without token_count
+    assert call(a3=ctypes.c_void_p((1 << 20) + 8)) == E  # unaligned k_pool
+    assert call(a12=s.workspace_bytes - 1) == C
+    small = binding.RkVisible(fake.value, fake.value, fake.value, fake.value, fake.value,
+                              fake.value, sz.entry_capacity - 1, sz.range_capacity)
+    assert call(a4=ctypes.byref(small)) == C
