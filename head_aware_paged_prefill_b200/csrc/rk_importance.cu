@@ -104,6 +104,14 @@ __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
                : "memory");
 }
 
+// 2^x on the special function unit (flushes results below 2^-126 to 0,
+// which a sum of weights in [0, 1] does not notice)
+__device__ __forceinline__ float ex2_fast(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // c (16 x 8, fp32) += A (16 x 16, bf16) B (16 x 8, bf16)
 __device__ __forceinline__ void mma_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
                                           uint32_t b1) {
@@ -189,6 +197,10 @@ __global__ void __launch_bounds__(kImpThreads)
     if (k0 + gq < en.n_valid) kpos[u][0] = en.logical_pos + k0 + gq;
     if (k0 + gq + 8 < en.n_valid) kpos[u][1] = en.logical_pos + k0 + gq + 8;
   }
+  // every key of the CTA is a real key (then a tile whose rows all see all
+  // keys needs no per-element mask)
+  const bool keys_full = __syncthreads_and(kpos[0][0] != INT_MAX && kpos[0][1] != INT_MAX &&
+                                           kpos[1][0] != INT_MAX && kpos[1][1] != INT_MAX);
   // column tiles: the table's row ranges clipped to [row_lo, row_hi]
   const rk_range* rg = a.ranges + a.range_start[t];
   auto seek = [&](int ri, ColTile& it) -> bool {
@@ -269,48 +281,79 @@ __global__ void __launch_bounds__(kImpThreads)
     }
     const ColTile cur = tiles[buf];
     const uint32_t sq = shared_addr(&sQ[buf][0]);
+    // a full tile whose every row sees every key of the CTA: no mask
+    const bool open = keys_full && cur.f0 + kImpCols <= cur.fend && cur.f0 / G >= pos_hi &&
+                      (!local || (cur.f0 + kImpCols - 1) / G - pos_lo < W);
 #pragma unroll 1
-    for (int nt = 0; nt < kImpCols / 8; ++nt) {
-      // this lane's two columns of the 8-column tile
-      int ci[2];
-      bool cv[2];
-      float l2[2];
+    for (int ng = 0; ng < kImpCols / 32; ++ng) {
+      // four 8-column tiles at a time: 2 slices x 4 tiles = 8 independent
+      // accumulator chains per warp.  Q^T as the B operand: ldmatrix
+      // matrices (columns of tile nt, chunks 4 jj .. 4 jj + 3)
+      uint32_t b[4][KS][2];
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        const int col = nt * 8 + 2 * tq + cc;
-        const int f = cur.f0 + col;
-        cv[cc] = f < cur.fend;
-        ci[cc] = f / G;
-        l2[cc] = sL[buf][col] * kLog2e;
-      }
-      // Q^T as the B operand: matrices (columns nt*8.., chunk 4j + m)
-      uint32_t b[KS][2];
+      for (int q4 = 0; q4 < 4; ++q4)
 #pragma unroll
-      for (int jj = 0; jj < KS / 2; ++jj) {
-        const int line = nt * 8 + (lane & 7), c = 4 * jj + (lane >> 3);
-        uint32_t rr[4];
-        ldsm_x4(sq + (line * CHUNKS + (c ^ (line & 7))) * 16, rr);
-        b[2 * jj][0] = rr[0];
-        b[2 * jj][1] = rr[1];
-        b[2 * jj + 1][0] = rr[2];
-        b[2 * jj + 1][1] = rr[3];
-      }
+        for (int jj = 0; jj < KS / 2; ++jj) {
+          const int line = (ng * 4 + q4) * 8 + (lane & 7), c = 4 * jj + (lane >> 3);
+          uint32_t rr[4];
+          ldsm_x4(sq + (line * CHUNKS + (c ^ (line & 7))) * 16, rr);
+          b[q4][2 * jj][0] = rr[0];
+          b[q4][2 * jj][1] = rr[1];
+          b[q4][2 * jj + 1][0] = rr[2];
+          b[q4][2 * jj + 1][1] = rr[3];
+        }
+      float c[kImpSlices][4][4];
 #pragma unroll
-      for (int u = 0; u < kImpSlices; ++u) {
-        float c[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int u = 0; u < kImpSlices; ++u)
 #pragma unroll
-        for (int ks = 0; ks < KS; ++ks) mma_16816(c, ka[u][ks], b[ks][0], b[ks][1]);
-        // c[kk * 2 + cc]: key gq + 8 kk, column 2 tq + cc
+        for (int q4 = 0; q4 < 4; ++q4) c[u][q4][0] = c[u][q4][1] = c[u][q4][2] = c[u][q4][3] = 0.f;
 #pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {
-          const int pk = kpos[u][kk];
+      for (int ks = 0; ks < KS; ++ks)
+#pragma unroll
+        for (int u = 0; u < kImpSlices; ++u)
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) mma_16816(c[u][q4], ka[u][ks], b[q4][ks][0], b[q4][ks][1]);
+      // c[u][q4][kk * 2 + cc]: key gq + 8 kk of slice u, column 2 tq + cc of tile q4
+      if (open) {
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4)
 #pragma unroll
           for (int cc = 0; cc < 2; ++cc) {
-            const int i = ci[cc];
-            const bool vis = cv[cc] && pk <= i && (!local || i - pk < W);
-            colsum[u][kk] += vis ? exp2f(c[kk * 2 + cc] * a.scale_log2 - l2[cc]) : 0.f;
+            const float l2 = sL[buf][(ng * 4 + q4) * 8 + 2 * tq + cc] * kLog2e;
+#pragma unroll
+            for (int u = 0; u < kImpSlices; ++u)
+#pragma unroll
+              for (int kk = 0; kk < 2; ++kk)
+                colsum[u][kk] += ex2_fast(fmaf(c[u][q4][kk * 2 + cc], a.scale_log2, -l2));
           }
+        continue;
+      }
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        int ci[2];
+        bool cv[2];
+        float l2[2];
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          const int col = (ng * 4 + q4) * 8 + 2 * tq + cc;
+          const int f = cur.f0 + col;
+          cv[cc] = f < cur.fend;
+          ci[cc] = f / G;
+          l2[cc] = sL[buf][col] * kLog2e;
         }
+#pragma unroll
+        for (int u = 0; u < kImpSlices; ++u)
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk) {
+            const int pk = kpos[u][kk];
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+              const int i = ci[cc];
+              const bool vis = cv[cc] && pk <= i && (!local || i - pk < W);
+              colsum[u][kk] += vis ? ex2_fast(fmaf(c[u][q4][kk * 2 + cc], a.scale_log2, -l2[cc]))
+                                   : 0.f;
+            }
+          }
       }
     }
   }
