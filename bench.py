@@ -56,7 +56,9 @@ def _peaks():
 
 
 KERNEL_SOURCES = {"segpaged_prefill_kernel": ("rk_prefill.cu", "sm100.cuh", "rk_internal.h"),
-                  "relocate_kernel": ("rk_relocate.cu", "sm100.cuh", "rk_internal.h")}
+                  "relocate_kernel": ("rk_relocate.cu", "sm100.cuh", "rk_internal.h"),
+                  "decode_split_kernel": ("rk_decode.cu", "rk_internal.h"),
+                  "importance_colsum_kernel": ("rk_importance.cu", "rk_internal.h")}
 
 
 def _kernel_hash(kernel: str = "segpaged_prefill_kernel") -> str:
@@ -453,10 +455,11 @@ def _bench_decode(torch, lay, pre, dev, flush, stream, reps, peaks, peak_kind, b
                         "one decode row per request and q head",
             "bytes": nbytes, "achieved": gbs, "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
             "frac": gbs / float(peaks["hbm_gbs"]), "peak_kind": peak_kind, "us": t * 1e3,
-            "rows_per_s": batch * lay.n_layers * lay.hq / (t * 1e-3), "device_status": st}
+            "rows_per_s": batch * lay.n_layers * lay.hq / (t * 1e-3), "device_status": st,
+            "traffic": _recorded_traffic("decode_split_kernel", f"decode_{batch}req")}
 
 
-def _bench_importance(torch, lay, q, k, v, dev, flush, stream, reps, peaks, peak_kind):
+def _bench_importance(torch, lay, lay_name, q, k, v, dev, flush, stream, reps, peaks, peak_kind):
     """rk_attention_importance on the bench's layer after its prefill (with
     lse): every visible (q head, row, key) pair's weight exp(s - lse) summed
     per token, then the top L/4 tokens.  One exp per visible pair and a
@@ -493,6 +496,7 @@ def _bench_importance(torch, lay, q, k, v, dev, flush, stream, reps, peaks, peak
             "achieved": achieved, "peak": exp_peak, "unit": "Gexp/s",
             "frac": achieved / exp_peak, "peak_kind": "derived: 148 SMs x 16 ex2 / clock x max SM clock",
             "us": t * 1e3, "qk_tflops": 2 * lay.d * pairs / (t * 1e-3) / 1e12,
+            "traffic": _recorded_traffic("importance_colsum_kernel", lay_name),
             "device_status": st}
 
 
@@ -622,8 +626,8 @@ def main():
     decode = (_bench_decode(torch, lay, pre, dev, flush, stream, args.reloc_reps, peaks,
                             peak_kind, args.decode_batch)
               if args.mode == "relocate" else None)
-    importance = (_bench_importance(torch, lay, q, k, v, dev, flush, stream, args.reloc_reps,
-                                    peaks, peak_kind)
+    importance = (_bench_importance(torch, lay, wl.name, q, k, v, dev, flush, stream,
+                                    args.reloc_reps, peaks, peak_kind)
                   if args.mode == "relocate" and not args.no_importance else None)
     mask_penalty = (_mask_penalty(torch, pre, lay, q, k3_mean)
                     if args.mode == "relocate" and not args.no_mask_penalty else None)
