@@ -12,18 +12,20 @@
 // position, in ascending order.
 //
 // Three launches:
-//   1. column sums, one CTA per (table, 128 keys).  Each warp holds two
-//      16-key slices of relocated K in registers as the A operand of warp-level
-//      bf16 MMAs; the CTA streams tiles of 64 (row, q head) columns of Q (and
-//      their lse) through a three-deep cp.async ring, only the rows of the
-//      table's row set that can see its keys (causal from its lowest key, up
-//      to its highest key + W - 1 for local tables).  S = K Q^T, then
-//      P = 2^(S scale log2 e - lse log2 e) masked per element, summed per key
-//      in registers and over the four lanes of a key at the end.  A CTA
-//      takes one chunk of 8192 / G rows (chunks aligned on row 0, so the
-//      CTAs of a chunk read the same Q rows from L2 and no CTA walks a whole
-//      long request); each (layer, kv head, chunk, token) partial is written
-//      by exactly one CTA.
+//   1. column sums on the tensor cores, one 256-thread CTA per (table, 128
+//      keys, row chunk).  The 128 keys of relocated K are the rows of the
+//      A operand (staged once); tiles of 64 (row, q head) columns of Q are
+//      the B operand, streamed with their lse through a four-deep cp.async
+//      ring, only the rows of the table's row set that can see the keys
+//      (causal from the lowest key, up to the highest key + W - 1 for local
+//      tables).  S = K Q^T lands in TMEM, one lane per key; the weights
+//      2^(S scale log2 e - lse log2 e), masked per element where a tile
+//      straddles a causal or window edge, are summed by the thread that
+//      owns the key's lane (two warps per lane quarter, 32 columns each).
+//      A chunk is 8192 / G rows aligned on row 0, so the CTAs of a chunk
+//      read the same Q rows from L2 and no CTA walks a whole long request;
+//      each (layer, kv head, chunk, token) partial is written by exactly one
+//      CTA.
 //   2. the partials added over kv heads and chunks in a fixed order: the
 //      importance.
 //   3. per (request, layer), one 1024-thread CTA: a four-pass radix select
@@ -38,19 +40,14 @@
 #include <cstdint>
 
 #include "rk_internal.h"
+#include "sm100.cuh"
 
 namespace rk {
 
 namespace {
 
-constexpr int kImpThreads = 128;
-constexpr int kImpWarps = kImpThreads / 32;
-constexpr int kImpSlices = 2;  // 16-key slices per warp
-constexpr int kImpCols = 64;   // (row, q head) columns per Q tile
-constexpr int kImpStages = 3;  // Q tiles in flight per CTA
 constexpr int kImpSelectThreads = 1024;
 constexpr float kLog2e = 1.4426950408889634f;
-static_assert(kImpWarps * kImpSlices * 16 == kImpKeysPerCta, "keys per CTA");
 
 struct ImpArgs {
   const __nv_bfloat16* q;
@@ -95,15 +92,6 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// Four 8x8 bf16 matrices from shared memory; lanes 8i..8i+7 address the rows
-// of matrix i, and lane l receives row l / 4, columns 2 (l % 4) + {0, 1}.
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr)
-               : "memory");
-}
-
 // 2^x on the special function unit (flushes results below 2^-126 to 0,
 // which a sum of weights in [0, 1] does not notice)
 __device__ __forceinline__ float ex2_fast(float x) {
@@ -112,44 +100,63 @@ __device__ __forceinline__ float ex2_fast(float x) {
   return y;
 }
 
-// c (16 x 8, fp32) += A (16 x 16, bf16) B (16 x 8, bf16)
-__device__ __forceinline__ void mma_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
-                                          uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
-      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
 // A run of Q tile columns: flat (row, q head) indices [f0, fend), f = row G + h.
 struct ColTile {
   int ri, f0, fend;
 };
 
-// 1. column sums of one table's 128 keys
+// 1. column sums of one table's 128 keys on the 5th-generation tensor cores:
+// the keys are the 128 rows of A (one TMEM lane each), a Q tile of 64
+// (row, q head) columns is B, and S = K Q^T lands in TMEM as 128 lanes x 64
+// fp32 columns (two buffers).  Thread i owns key i: it reads its lane's 64
+// scores and adds their weights without any cross-lane step.  The MMA of
+// tile j + 1 is issued before the weights of tile j are taken, so the
+// tensor work hides under the exponentials.  Operands are staged by
+// cp.async straight into the 128-byte-swizzled K-major layout (16-byte
+// chunk c of row r at c ^ (r & 7) inside 1024-byte atoms).
+constexpr int kTcCols = 64;     // Q tile columns (MMA N)
+constexpr int kTcQBufs = 4;     // Q / lse tiles in flight
+constexpr int kTcTmemCols = 128;  // two S buffers of kTcCols fp32 columns
+constexpr int kTcThreads = 256;   // two warps per TMEM lane quarter, each half the columns
+
+template <int D>
+struct TcSmem {
+  static constexpr int kKBytes = 128 * D * 2;
+  static constexpr int kQBytes = kTcCols * D * 2;
+  static constexpr int kOffQ = kKBytes;
+  static constexpr int kOffL = kOffQ + kTcQBufs * kQBytes;
+  static constexpr int kOffBar = kOffL + kTcQBufs * kTcCols * 4;
+  static constexpr int kBytes = kOffBar + 64;
+  static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024
+};
+
 template <int D, int G>
-__global__ void __launch_bounds__(kImpThreads)
-    importance_colsum_kernel(const __grid_constant__ ImpArgs a) {
-  constexpr int KS = D / 16;
+__global__ void __launch_bounds__(kTcThreads)
+    importance_colsum_tc_kernel(const __grid_constant__ ImpArgs a) {
+  using S = TcSmem<D>;
   constexpr int CHUNKS = D / 8;
-  extern __shared__ __align__(128) uint8_t imp_smem[];
-  // [kImpStages][kImpCols][D] Q columns, then [kImpStages][kImpCols] lse
-  auto sQ = reinterpret_cast<__nv_bfloat16(*)[kImpCols * D]>(imp_smem);
-  auto sL = reinterpret_cast<float(*)[kImpCols]>(imp_smem + kImpStages * kImpCols * D * 2);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int gq = lane >> 2, tq = lane & 3;
+  extern __shared__ uint8_t tc_raw[];
+  uint8_t* sm = tc_raw + ((1024 - (smem_u32(tc_raw) & 1023)) & 1023);
+  uint8_t* sK = sm;
+  uint8_t* sQ = sm + S::kOffQ;
+  float* sL = reinterpret_cast<float*>(sm + S::kOffL);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + S::kOffBar);  // [2] S full
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + S::kOffBar + 16);
+  int* abort_flag = reinterpret_cast<int*>(sm + S::kOffBar + 20);
+  const int warp = threadIdx.x >> 5, tid = threadIdx.x;
+  const int key = tid & 127;      // TMEM lane = row of the K tile
+  const int half = warp >> 2;     // which 32 of the tile's 64 columns
   const int t = blockIdx.x;
   const int kvh = t % a.hkv, layer = (t / a.hkv) % a.n_layers, r = t / (a.hkv * a.n_layers);
   const int n_e = a.entry_count[t], e_first = a.entry_start[t], rc = a.range_count[t];
   const int spp = a.p / 16;
   const int n_sl = n_e * spp;
-  const int s_begin = blockIdx.y * (kImpWarps * kImpSlices);
+  const int s_begin = blockIdx.y * 8;
   if (s_begin >= n_sl || rc == 0) return;
-  const int s_end = min(n_sl, s_begin + kImpWarps * kImpSlices);
+  const int s_end = min(n_sl, s_begin + 8);
   const int t0 = a.cu[r], L = a.cu[r + 1] - t0;
   const bool local = a.cls[layer * a.hkv + kvh] == RK_LOCAL;
   const int W = a.window;
-  // the CTA's lowest and highest key positions (entries ascend)
   int pos_lo, pos_hi;
   {
     const rk_entry e0 = a.entries[e_first + s_begin / spp];
@@ -158,50 +165,41 @@ __global__ void __launch_bounds__(kImpThreads)
     const rk_entry e1 = a.entries[e_first + sl / spp];
     pos_hi = e1.logical_pos + min((sl % spp) * 16 + 16, e1.n_valid) - 1;
   }
-  // rows that can see these keys (causal from the lowest; for a local table,
-  // up to the highest + W - 1), cut to this CTA's chunk of kImpChunkCols / G
-  // rows (chunks are aligned on row 0, so the CTAs of one chunk read the same
-  // Q rows while they are in L2)
   constexpr int RPC = kImpChunkCols / G;
   const int chunk = blockIdx.z;
   const int row_lo = max(pos_lo, chunk * RPC);
   const int row_hi =
       min(local ? min(L - 1, pos_hi + min(W, L) - 1) : L - 1, chunk * RPC + RPC - 1);
   if (row_lo > row_hi) return;
-  // this warp's keys as A fragments (a0: key gq, columns 2 tq; a1: key gq + 8;
-  // a2, a3: columns + 8), and their positions (INT_MAX: no key)
-  uint32_t ka[kImpSlices][KS][4];
-  int kpos[kImpSlices][2];
-#pragma unroll
-  for (int u = 0; u < kImpSlices; ++u) {
-    kpos[u][0] = kpos[u][1] = INT_MAX;
-#pragma unroll
-    for (int ks = 0; ks < KS; ++ks) ka[u][ks][0] = ka[u][ks][1] = ka[u][ks][2] = ka[u][ks][3] = 0u;
-    const int s = s_begin + warp * kImpSlices + u;
-    if (s >= s_end) continue;
-    const rk_entry en = a.entries[e_first + s / spp];
-    const int k0 = (s % spp) * 16;
-    if (en.phys_page < 0 || en.phys_page >= a.n_pages) {
-      if (lane == 0) atomicOr(a.error_word, static_cast<int>(RK_DEV_BAD_PAGE));
-      continue;
+  // this thread's key (TMEM lane `key` = row `key` of the K tile)
+  int kpos = INT_MAX;
+  {
+    const int s = s_begin + key / 16, kk = key % 16;
+    if (s < s_end) {
+      const rk_entry en = a.entries[e_first + s / spp];
+      const int k0 = (s % spp) * 16;
+      if (en.phys_page >= 0 && en.phys_page < a.n_pages && k0 + kk < en.n_valid)
+        kpos = en.logical_pos + k0 + kk;
     }
-    const uint32_t* kr = reinterpret_cast<const uint32_t*>(
-        a.k_pool + (static_cast<int64_t>(en.phys_page) * a.p + k0) * D);
-#pragma unroll
-    for (int ks = 0; ks < KS; ++ks) {
-      ka[u][ks][0] = kr[gq * (D / 2) + ks * 8 + tq];
-      ka[u][ks][1] = kr[(gq + 8) * (D / 2) + ks * 8 + tq];
-      ka[u][ks][2] = kr[gq * (D / 2) + ks * 8 + 4 + tq];
-      ka[u][ks][3] = kr[(gq + 8) * (D / 2) + ks * 8 + 4 + tq];
-    }
-    if (k0 + gq < en.n_valid) kpos[u][0] = en.logical_pos + k0 + gq;
-    if (k0 + gq + 8 < en.n_valid) kpos[u][1] = en.logical_pos + k0 + gq + 8;
   }
-  // every key of the CTA is a real key (then a tile whose rows all see all
-  // keys needs no per-element mask)
-  const bool keys_full = __syncthreads_and(kpos[0][0] != INT_MAX && kpos[0][1] != INT_MAX &&
-                                           kpos[1][0] != INT_MAX && kpos[1][1] != INT_MAX);
-  // column tiles: the table's row ranges clipped to [row_lo, row_hi]
+  // stage the K tile: row rr <- key rr of the CTA (zeros for no key)
+  for (int x = tid; x < 128 * CHUNKS; x += kTcThreads) {
+    const int rr = x / CHUNKS, c = x % CHUNKS;
+    uint8_t* dst = sK + (c >> 3) * (128 * 128) + rr * 128 + (((c & 7) ^ (rr & 7)) << 4);
+    const int s = s_begin + rr / 16;
+    bool copied = false;
+    if (s < s_end) {
+      const rk_entry en = a.entries[e_first + s / spp];
+      if (en.phys_page >= 0 && en.phys_page < a.n_pages) {
+        const int64_t row = static_cast<int64_t>(en.phys_page) * a.p + (s % spp) * 16 + rr % 16;
+        cp_async16(dst, a.k_pool + row * D + c * 8);
+        copied = true;
+      } else if (rr % 16 == 0 && c == 0) {
+        atomicOr(a.error_word, static_cast<int>(RK_DEV_BAD_PAGE));
+      }
+    }
+    if (!copied) *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+  }
   const rk_range* rg = a.ranges + a.range_start[t];
   auto seek = [&](int ri, ColTile& it) -> bool {
     for (; ri < rc; ++ri) {
@@ -218,158 +216,154 @@ __global__ void __launch_bounds__(kImpThreads)
     return false;
   };
   auto advance = [&](ColTile& it) -> bool {
-    it.f0 += kImpCols;
+    it.f0 += kTcCols;
     if (it.f0 < it.fend) return true;
     return seek(it.ri + 1, it);
   };
-  // stage a tile's Q columns (16-byte chunks permuted per column, chunk c of
-  // column n at c ^ (n & 7)) and their lse, all by cp.async
+  // stage a Q tile (its columns' rows, zeros past the run) and its lse
   auto stage = [&](const ColTile& it, int buf) {
-    for (int x = threadIdx.x; x < kImpCols * CHUNKS; x += kImpThreads) {
+    uint8_t* q = sQ + buf * S::kQBytes;
+    for (int x = tid; x < kTcCols * CHUNKS; x += kTcThreads) {
       const int n = x / CHUNKS, c = x % CHUNKS;
+      uint8_t* dst = q + (c >> 3) * (kTcCols * 128) + n * 128 + (((c & 7) ^ (n & 7)) << 4);
       const int f = it.f0 + n;
       if (f < it.fend) {
         const int i = f / G, h = f - i * G;
-        const __nv_bfloat16* src =
-            a.q + ((static_cast<int64_t>(layer) * a.total_tokens + t0 + i) * a.hq + kvh * G + h) * D +
-            c * 8;
-        cp_async16(&sQ[buf][n * D + (c ^ (n & 7)) * 8], src);
+        cp_async16(dst, a.q + ((static_cast<int64_t>(layer) * a.total_tokens + t0 + i) * a.hq +
+                               kvh * G + h) * D + c * 8);
+      } else {
+        *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
       }
     }
-    if (threadIdx.x < kImpCols) {
-      const int f = it.f0 + threadIdx.x;
+    if (tid < kTcCols) {
+      const int f = it.f0 + tid;
       if (f < it.fend) {
         const int i = f / G, h = f - i * G;
-        cp_async4(&sL[buf][threadIdx.x],
+        cp_async4(&sL[buf * kTcCols + tid],
                   a.lse + (static_cast<int64_t>(layer) * a.hq + kvh * G + h) * a.total_tokens + t0 + i);
       }
     }
   };
-  float colsum[kImpSlices][2];
-#pragma unroll
-  for (int u = 0; u < kImpSlices; ++u) colsum[u][0] = colsum[u][1] = 0.f;
-  // a ring of kImpStages tiles: tile j lives in buffer j % kImpStages; one
-  // barrier per tile both publishes tile j and retires tile j - 1's buffer
-  ColTile tiles[kImpStages];  // tiles[j % kImpStages]: the tile staged there
-  bool valid[kImpStages];
+  ColTile tiles[kTcQBufs];
+  int n_staged = 0;
   ColTile it;
   bool more = seek(0, it);
-#pragma unroll
-  for (int j = 0; j < kImpStages - 1; ++j) {
-    valid[j] = more;
+  auto stage_next = [&]() {
     if (more) {
-      tiles[j] = it;
-      stage(it, j);
+      tiles[n_staged % kTcQBufs] = it;
+      stage(it, n_staged % kTcQBufs);
+      ++n_staged;
       more = advance(it);
     }
-    cp_async_commit();
+    cp_async_commit();  // one group per call, empty or not
+  };
+  stage_next();  // group 0: the K tile and Q tile 0
+  stage_next();  // Q tile 1
+  stage_next();  // Q tile 2
+  if (tid == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
   }
-  valid[kImpStages - 1] = false;
-  for (int j = 0; valid[j % kImpStages]; ++j) {
-    const int buf = j % kImpStages;
-    cp_async_wait<kImpStages - 2>();  // tile j has landed (this thread's copies)
-    __syncthreads();                  // ... everyone's; tile j - 1's buffer is free
-    {
-      const int nb = (j + kImpStages - 1) % kImpStages;
-      valid[nb] = more;
-      if (more) {
-        tiles[nb] = it;
-        stage(it, nb);
-        more = advance(it);
-      }
-      cp_async_commit();
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, kTcTmemCols);
+    tmem_relinquish();
+  }
+  const bool keys_full = __syncthreads_and(kpos != INT_MAX);
+  const WaitCtx wc{abort_flag, a.error_word, a.error_word + 1};
+  cp_async_wait<2>();  // K and Q tile 0 have landed (this thread's copies)
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  constexpr uint32_t idesc = idesc_bf16_f32(128, kTcCols, false);
+  const uint32_t sK_u = smem_u32(sK), sQ_u = smem_u32(sQ);
+  auto issue = [&](int j) {  // S buffer j & 1 <- K Q_j^T
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint64_t ad = desc_sw128(sK_u + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024);
+      const uint64_t bd = desc_sw128(
+          sQ_u + (j % kTcQBufs) * S::kQBytes + (kk >> 2) * (kTcCols * 128) + (kk & 3) * 32, 16, 1024);
+      mma_bf16_ss(tmem + (j & 1) * kTcCols, ad, bd, idesc, kk > 0 ? 1u : 0u);
     }
-    const ColTile cur = tiles[buf];
-    const uint32_t sq = shared_addr(&sQ[buf][0]);
-    // a full tile whose every row sees every key of the CTA: no mask
-    const bool open = keys_full && cur.f0 + kImpCols <= cur.fend && cur.f0 / G >= pos_hi &&
-                      (!local || (cur.f0 + kImpCols - 1) / G - pos_lo < W);
-#pragma unroll 1
-    for (int ng = 0; ng < kImpCols / 32; ++ng) {
-      // four 8-column tiles at a time: 2 slices x 4 tiles = 8 independent
-      // accumulator chains per warp.  Q^T as the B operand: ldmatrix
-      // matrices (columns of tile nt, chunks 4 jj .. 4 jj + 3)
-      uint32_t b[4][KS][2];
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4)
-#pragma unroll
-        for (int jj = 0; jj < KS / 2; ++jj) {
-          const int line = (ng * 4 + q4) * 8 + (lane & 7), c = 4 * jj + (lane >> 3);
-          uint32_t rr[4];
-          ldsm_x4(sq + (line * CHUNKS + (c ^ (line & 7))) * 16, rr);
-          b[q4][2 * jj][0] = rr[0];
-          b[q4][2 * jj][1] = rr[1];
-          b[q4][2 * jj + 1][0] = rr[2];
-          b[q4][2 * jj + 1][1] = rr[3];
-        }
-      float c[kImpSlices][4][4];
-#pragma unroll
-      for (int u = 0; u < kImpSlices; ++u)
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) c[u][q4][0] = c[u][q4][1] = c[u][q4][2] = c[u][q4][3] = 0.f;
-#pragma unroll
-      for (int ks = 0; ks < KS; ++ks)
-#pragma unroll
-        for (int u = 0; u < kImpSlices; ++u)
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) mma_16816(c[u][q4], ka[u][ks], b[q4][ks][0], b[q4][ks][1]);
-      // c[u][q4][kk * 2 + cc]: key gq + 8 kk of slice u, column 2 tq + cc of tile q4
+    tc_commit(&bars[j & 1]);
+  };
+  int n_issued = 0, n_waited = 0;
+  if (tid == 0 && n_staged > 0) issue(0);
+  if (n_staged > 0) n_issued = 1;
+  float acc0 = 0.f, acc1 = 0.f;
+  bool ok = true;
+  const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+  for (int j = 0; j < n_staged; ++j) {
+    cp_async_wait<1>();  // tile j + 1 has landed (this thread's copies)
+    fence_proxy_async_smem();
+    tc_fence_before();
+    ok = __syncthreads_and(ok);  // ... everyone's; tile j - 1 is fully consumed
+    if (!ok) break;
+    tc_fence_after();
+    stage_next();  // tile j + 3 into tile j - 1's buffer
+    if (j + 1 < n_staged) {
+      if (tid == 0) issue(j + 1);
+      ++n_issued;
+    }
+    ok = mbar_wait(&bars[j & 1], (j >> 1) & 1, wc, 1);
+    ok = __all_sync(0xffffffffu, ok);
+    if (!ok) continue;  // the next barrier ends the loop for everyone
+    ++n_waited;
+    tc_fence_after();
+    const ColTile cur = tiles[j % kTcQBufs];
+    const float* lse = sL + (j % kTcQBufs) * kTcCols;
+    const bool open = keys_full && cur.f0 + kTcCols <= cur.fend && cur.f0 / G >= pos_hi &&
+                      (!local || (cur.f0 + kTcCols - 1) / G - pos_lo < W);
+    {
+      const int c0 = half * 32;
+      uint32_t v[32];
+      tmem_ld_x32(tmem + lane_base + (j & 1) * kTcCols + c0, v);
+      tmem_ld_wait(v);
       if (open) {
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4)
-#pragma unroll
-          for (int cc = 0; cc < 2; ++cc) {
-            const float l2 = sL[buf][(ng * 4 + q4) * 8 + 2 * tq + cc] * kLog2e;
-#pragma unroll
-            for (int u = 0; u < kImpSlices; ++u)
-#pragma unroll
-              for (int kk = 0; kk < 2; ++kk)
-                colsum[u][kk] += ex2_fast(fmaf(c[u][q4][kk * 2 + cc], a.scale_log2, -l2));
-          }
-        continue;
-      }
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        int ci[2];
-        bool cv[2];
-        float l2[2];
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          const int col = (ng * 4 + q4) * 8 + 2 * tq + cc;
-          const int f = cur.f0 + col;
-          cv[cc] = f < cur.fend;
-          ci[cc] = f / G;
-          l2[cc] = sL[buf][col] * kLog2e;
+        for (int n = 0; n < 32; n += 2) {
+          acc0 += ex2_fast(fmaf(__uint_as_float(v[n]), a.scale_log2, -lse[c0 + n] * kLog2e));
+          acc1 += ex2_fast(fmaf(__uint_as_float(v[n + 1]), a.scale_log2, -lse[c0 + n + 1] * kLog2e));
         }
+      } else {
 #pragma unroll
-        for (int u = 0; u < kImpSlices; ++u)
-#pragma unroll
-          for (int kk = 0; kk < 2; ++kk) {
-            const int pk = kpos[u][kk];
-#pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-              const int i = ci[cc];
-              const bool vis = cv[cc] && pk <= i && (!local || i - pk < W);
-              colsum[u][kk] += vis ? ex2_fast(fmaf(c[u][q4][kk * 2 + cc], a.scale_log2, -l2[cc]))
-                                   : 0.f;
-            }
-          }
+        for (int n = 0; n < 32; ++n) {
+          const int f = cur.f0 + c0 + n;
+          const int i = f / G;
+          const bool vis = f < cur.fend && kpos <= i && (!local || i - kpos < W);
+          const float w =
+              vis ? ex2_fast(fmaf(__uint_as_float(v[n]), a.scale_log2, -lse[c0 + n] * kLog2e)) : 0.f;
+          if (n & 1)
+            acc1 += w;
+          else
+            acc0 += w;
+        }
       }
     }
+    tc_fence_before();
   }
   cp_async_wait<0>();
-  // sum over the four lanes of each key and write this chunk's partial
-  float* part = a.part + ((static_cast<int64_t>(layer) * a.hkv + kvh) * a.n_chunks + chunk) *
-                             a.total_tokens + t0;
-#pragma unroll
-  for (int u = 0; u < kImpSlices; ++u)
-#pragma unroll
-    for (int kk = 0; kk < 2; ++kk) {
-      float v = colsum[u][kk];
-      v += __shfl_xor_sync(0xffffffffu, v, 1);
-      v += __shfl_xor_sync(0xffffffffu, v, 2);
-      if (tq == 0 && kpos[u][kk] != INT_MAX) part[kpos[u][kk]] = v;
-    }
+  if (tid == 0) {
+    // MMAs still in flight after an abort (at most two, one per barrier):
+    // let them finish before the TMEM goes
+    for (int m = n_waited; m < n_issued; ++m) mbar_wait_drain(&bars[m & 1], (m >> 1) & 1);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTcTmemCols);
+  }
+  // the two column halves of each key, added in a fixed order
+  float* red = reinterpret_cast<float*>(sm + S::kOffL);
+  if (half == 1) red[key] = acc0 + acc1;
+  __syncthreads();
+  if (half == 0 && ok && kpos != INT_MAX)
+    a.part[((static_cast<int64_t>(layer) * a.hkv + kvh) * a.n_chunks + chunk) * a.total_tokens +
+           t0 + kpos] = (acc0 + acc1) + red[key];
 }
 
 // 2. importance: the partials added over kv heads and chunks, in that order
@@ -473,12 +467,12 @@ __global__ void __launch_bounds__(kImpSelectThreads)
 template <int D, int G>
 cudaError_t launch_importance_typed(const ImpArgs& a, int n_tables, int max_blocks,
                                     cudaStream_t stream) {
-  constexpr size_t smem = static_cast<size_t>(kImpStages) * kImpCols * (D * 2 + 4);
-  auto colsum = importance_colsum_kernel<D, G>;
+  constexpr size_t smem = TcSmem<D>::kAlloc;
+  auto colsum = importance_colsum_tc_kernel<D, G>;
   cudaError_t e = cudaFuncSetAttribute(colsum, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  colsum<<<dim3(n_tables, max_blocks, a.n_chunks), kImpThreads, smem, stream>>>(a);
+  colsum<<<dim3(n_tables, max_blocks, a.n_chunks), kTcThreads, smem, stream>>>(a);
   if (a.total_tokens > 0)
     importance_reduce_kernel<<<dim3((a.total_tokens + 255) / 256, a.n_layers), 256, 0, stream>>>(a);
   importance_select_kernel<<<a.n_req * a.n_layers, kImpSelectThreads, 0, stream>>>(a);
