@@ -29,10 +29,15 @@
  *     ranges.  Both are derived by brute force over (row, key) pairs.
  *
  *   - Retrieval page scoring (ora_score_pages, a reading stated there).
+ *   - Token importance for the sparse FFN (ora_importance, a reading stated
+ *     there): the prefill's softmax weights summed per token over q heads
+ *     and computed rows.
  *
  * parity pins: see tests/test_oracle_pins.py (RoPE closed form and
  * composition, causal and windowed SDPA special cases, perturbation
- * invariance, sharing, brute-force vs closed-form page tables, pair counts).
+ * invariance, sharing, brute-force vs closed-form page tables, pair counts),
+ * tests/test_oracle_scoring.py and tests/test_oracle_importance.py (dense
+ * restatement, unit row sums, harmonic closed form, selection brute force).
  */
 #include <math.h>
 #include <pthread.h>

@@ -153,6 +153,25 @@ def test_importance_deterministic():
         assert np.array_equal(x, y)
 
 
+def test_importance_through_api():
+    """SegPagedPrefill.attention_importance after a prefill with lse: the
+    same bar against the oracle, and the same invariants."""
+    from head_aware_paged_prefill_b200.api import SegPagedPrefill
+    wl = synth.cfg1()
+    lay = wl.layout
+    q, k, v = wl.materialize("cpu")
+    pre = SegPagedPrefill(lay, "cuda", with_lse=True)
+    pre.load(q.cuda(), k.cuda(), v.cuda())
+    pre.compute()
+    imp, tokens, count = pre.attention_importance(24)
+    torch.cuda.synchronize()
+    assert pre.importance_status() == 0
+    imp = imp.cpu().numpy().astype(np.float64)
+    tokens, count = tokens.cpu().numpy(), count.cpu().numpy()
+    _check_invariants(lay, imp, tokens, count, 24, "api")
+    _check_against_oracle(lay, imp, tokens, count, q, k, 24, "api")
+
+
 def test_importance_rejects_on_host():
     lay = synth.cfg1().layout
     hl = binding.HostLayout(lay)
