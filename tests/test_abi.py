@@ -235,3 +235,17 @@ def test_importance_calls_validate_on_host(lib):
     small = binding.RkVisible(fake.value, fake.value, fake.value, fake.value, fake.value,
                               fake.value, sz.entry_capacity - 1, sz.range_capacity)
     assert call(a4=ctypes.byref(small)) == C
+
+
+@pytest.mark.parametrize("name", ["cfg2", "cfg4"])
+def test_importance_workspace_covers_row_chunks(lib, name):
+    """The column-sum partials are kept per row chunk of 8192 / G rows, so
+    the workspace holds n_layers x Hkv x chunks x T floats."""
+    lay = synth.CONFIGS[name]().layout
+    s = binding.importance_sizes(_hl(lay))
+    g = lay.hq // lay.hkv
+    L = max(lay.req_len(r) for r in range(lay.n_req))
+    chunks = -(-L // (8192 // g))
+    T = int(lay.cu_seqlens[-1])
+    assert s.workspace_bytes >= 256 + 4 * lay.n_layers * lay.hkv * chunks * T
+    assert s.max_blocks == -(-(-(-L // lay.p) * lay.p) // 128)
