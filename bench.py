@@ -184,21 +184,32 @@ def _gpu_id(torch, dev) -> str:
 
 
 def _oracle_sample_rows(lay, n_rows: int, seed: int):
-    """A seeded sample of computed (layer, q_head, token) rows and the number of
-    visible keys of each, for the CPU baseline."""
+    """A seeded sample of computed (layer, q_head, token) rows, uniform over
+    every computed row of the workload, and the number of visible keys of
+    the sampled rows (closed form per class), for the CPU baseline."""
+    from head_aware_paged_prefill_b200 import metrics
     rng = np.random.default_rng(seed)
     g = lay.hq // lay.hkv
-    W = int(lay.class_window[1])
+    tabs, sizes = [], []
+    for r in range(lay.n_req):
+        for layer in range(lay.n_layers):
+            for kvh in range(lay.hkv):
+                rows = metrics.table_rows(lay, r, layer, kvh)
+                if rows.size:
+                    tabs.append((r, layer, kvh, rows))
+                    sizes.append(rows.size)
+    w = np.asarray(sizes, dtype=np.float64)
+    pick = rng.choice(len(tabs), size=n_rows, p=w / w.sum())
     out, pairs = [], 0
-    L = lay.req_len(0)
-    tail0 = int(lay.segments[lay.segments[:, 4] == 0][0, 1])
-    for _ in range(n_rows):
-        h = int(rng.integers(lay.hq))
-        cls = int(lay.class_map[h // g])
-        i = int(rng.integers(L)) if cls in (0, 3) else int(rng.integers(tail0, L))
-        out.append((0, h, i))
-        pairs += (i + 1) if cls in (0, 3) else min(i + 1, W)
-    return np.asarray(out, dtype=np.int32), pairs
+    for ti in np.unique(pick):
+        r, layer, kvh, rows = tabs[ti]
+        n = int((pick == ti).sum())
+        i = rows[rng.integers(rows.size, size=n)]
+        h = kvh * g + rng.integers(g, size=n)
+        pairs += int(metrics.row_visible_keys(lay, r, layer, kvh, i).sum())
+        t0 = int(lay.cu_seqlens[r])
+        out.append(np.column_stack([np.full(n, layer), h, t0 + i]))
+    return np.concatenate(out).astype(np.int32), pairs
 
 
 def _time_oracle(lay, q, k, v, rows):
@@ -208,18 +219,22 @@ def _time_oracle(lay, q, k, v, rows):
     def u16(t):
         return t.contiguous().view(torch.int16).numpy().view(np.uint16)
 
-    idx = torch.from_numpy(rows).long()
-    qr = q[idx[:, 0], idx[:, 2], idx[:, 1]]
+    idx = torch.from_numpy(rows).long().to(q.device)
+    qr = q[idx[:, 0], idx[:, 2], idx[:, 1]].cpu()
     t0 = time.perf_counter()
     oracle.attention(lay, u16(qr), u16(k), u16(v), rows)
     return time.perf_counter() - t0
 
 
-def _bench_relocate(torch, lay, k_pool, dev, flush, stream, reps, peaks, peak_kind):
+def _bench_relocate(torch, lay, k_pool, dev, flush, stream, reps, peaks, peak_kind, copies=4):
     """rk_relocate_rope alone over every page of every cached segment with
     delta != 0 (all (layer, kv_head) pairs, visible or not), from the store
-    into a working pool at the same page ids: a bandwidth measurement of the
-    relocation kernel on a job list larger than the step's own."""
+    into a working pool at the same page ids.  The main figure runs that job
+    list over `copies` distinct copies of the store into as many distinct
+    destination pools, so the pages read and written (several times the
+    126 MB L2) stream from and to HBM; the single-copy figure, whose 50 MB
+    of writes can stay in L2 until after the timed launch, is kept beside
+    it as "in_l2"."""
     from head_aware_paged_prefill_b200 import binding, metrics
     n_lh = lay.n_layers * lay.hkv
     jobs = []
@@ -232,29 +247,43 @@ def _bench_relocate(torch, lay, k_pool, dev, flush, stream, reps, peaks, peak_ki
     if not jobs:
         return None
     jobs = np.asarray(jobs, dtype=np.int32)
-    n = jobs.shape[0]
-    work = torch.empty_like(k_pool)
-    jt = torch.from_numpy(jobs).to(dev)
-    for _ in range(3):
-        binding.relocate_rope(k_pool, work, jt, lay.theta)
-    torch.cuda.synchronize()
-    ms = []
-    for _ in range(reps):
-        flush()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        binding.relocate_rope(k_pool, work, jt, lay.theta)
-        b.record(stream)
-        ms.append((a, b))
-    torch.cuda.synchronize()
-    t = statistics.mean(x.elapsed_time(y) for x, y in ms)
-    byts = metrics.relocate_bytes(n, lay.p, lay.d)
-    gbs = byts / (t * 1e-3) / 1e9
     peak = float(peaks["hbm_gbs"])
-    return {"bound": "hbm", "kernel": "relocate_kernel", "jobs": n, "bytes": byts,
-            "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+
+    def timed(src, dst, jt):
+        for _ in range(3):
+            binding.relocate_rope(src, dst, jt, lay.theta)
+        torch.cuda.synchronize()
+        ms = []
+        for _ in range(reps):
+            flush()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            binding.relocate_rope(src, dst, jt, lay.theta)
+            b.record(stream)
+            ms.append((a, b))
+        torch.cuda.synchronize()
+        return statistics.mean(x.elapsed_time(y) for x, y in ms)
+
+    n = jobs.shape[0]
+    t1 = timed(k_pool, torch.empty_like(k_pool), torch.from_numpy(jobs).to(dev))
+    b1 = metrics.relocate_bytes(n, lay.p, lay.d)
+    npg = int(k_pool.shape[0])
+    big = np.concatenate([jobs + np.asarray([c * npg, c * npg, 0], np.int32) for c in range(copies)])
+    src = k_pool.repeat(copies, 1, 1)
+    dst = torch.empty_like(src)
+    t = timed(src, dst, torch.from_numpy(big).to(dev))
+    del src, dst
+    torch.cuda.empty_cache()
+    byts = metrics.relocate_bytes(big.shape[0], lay.p, lay.d)
+    gbs = byts / (t * 1e-3) / 1e9
+    return {"bound": "hbm", "kernel": "relocate_kernel", "jobs": int(big.shape[0]),
+            "workload": f"every delta != 0 page of the layer's cached segments, {copies} "
+                        "distinct copies (sources and destinations)",
+            "bytes": byts, "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
             "peak_kind": peak_kind, "us": t * 1e3,
-            "traffic": _recorded_traffic("relocate_kernel", "relocate_" + str(n))}
+            "traffic": _recorded_traffic("relocate_kernel", "relocate_" + str(big.shape[0])),
+            "in_l2": {"jobs": n, "bytes": b1, "us": t1 * 1e3,
+                      "achieved": b1 / (t1 * 1e-3) / 1e9, "frac": b1 / (t1 * 1e-3) / 1e9 / peak}}
 
 
 def cpu_values(wl):
@@ -500,6 +529,78 @@ def _bench_importance(torch, lay, lay_name, q, k, v, dev, flush, stream, reps, p
             "device_status": st}
 
 
+def _cpu_baseline(lay, q, kc, vc, seconds: float, total_pairs: int):
+    """The fp64 oracle timed on seeded row samples of the workload (batches of
+    growing size until about `seconds` of oracle time), with the full-run
+    time it implies (labelled as an extrapolation)."""
+    n_rows, tot_rows, tot_pairs, tot_t, seed = 1024, 0, 0, 0.0, 1
+    while tot_t < seconds:
+        rows, pairs = _oracle_sample_rows(lay, n_rows, seed=seed)
+        tot_t += _time_oracle(lay, q, kc, vc, rows)
+        tot_rows += n_rows
+        tot_pairs += pairs
+        seed += 1
+        n_rows = min(2 * n_rows, 65536)
+    return {"value": 4 * lay.d * tot_pairs / tot_t / 1e12, "unit": UNIT,
+            "cores": os.cpu_count() or 1, "kind": "oracle",
+            "sample": f"{tot_rows} seeded (layer, q head, row) samples, uniform over the "
+                      f"workload's computed rows, in {seed - 1} batches: {tot_pairs} visible "
+                      f"pairs in {tot_t:.1f} s",
+            "rows_per_s": tot_rows / tot_t,
+            "full_run_s_extrapolated": tot_t * total_pairs / max(tot_pairs, 1)}
+
+
+def _bench_config(torch, name, dev, flush, stream, steps, warmup, peaks, peak_kind, cpu_s):
+    """One more workload, timed like the headline one in both modes: the
+    attention kernel's TFLOP/s against the bf16 roofline, the whole step's
+    TFLOP/s and tokens/s, and a CPU-oracle baseline on a row sample."""
+    from head_aware_paged_prefill_b200 import metrics, synth
+    from head_aware_paged_prefill_b200.api import SegPagedPrefill
+    wl = synth.CONFIGS[name]()
+    lay = wl.layout
+    q, k, v = wl.materialize(str(dev))
+    flops = metrics.attention_flops(lay)
+    tokens = lay.total_tokens * lay.n_layers
+    peak = float(peaks["bf16_tflops"])
+    out = {"workload": wl.name, "requests": lay.n_req, "layers": lay.n_layers,
+           "tokens": lay.total_tokens, "heads": f"Hq {lay.hq} / Hkv {lay.hkv}",
+           "head_dim": lay.d, "page_size": lay.p, "visible_pairs": flops // (4 * lay.d),
+           "steps": steps, "l2": L2Flush.DESCRIPTION}
+    for mode in ("relocate", "fused"):
+        pre = SegPagedPrefill(lay, dev, mode=mode)
+        pre.load(q, k, v)
+        for _ in range(warmup):
+            pre.compute()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(2 * steps)]
+        for s_ in range(steps):
+            flush()
+            ev[2 * s_][0].record(stream)
+            pre.compute(k3_events=ev[2 * s_ + 1])
+            ev[2 * s_][1].record(stream)
+        torch.cuda.synchronize()
+        step_ms = statistics.mean(ev[2 * i][0].elapsed_time(ev[2 * i][1]) for i in range(steps))
+        k3_ms = statistics.mean(ev[2 * i + 1][0].elapsed_time(ev[2 * i + 1][1])
+                                for i in range(steps))
+        k3 = flops / (k3_ms * 1e-3) / 1e12
+        out[mode] = {"step_tflops": flops / (step_ms * 1e-3) / 1e12, "ms_per_step": step_ms,
+                     "tokens_per_s": tokens / (step_ms * 1e-3), "k3_ms": k3_ms,
+                     "k3_tflops": k3, "k3_frac": k3 / peak, "device_status": pre.status(),
+                     "launches_per_step": pre.launches_per_run}
+        del pre
+        torch.cuda.empty_cache()
+    k3 = out["relocate"]["k3_tflops"]
+    out["roofline"] = {"bound": "tensor", "kernel": "segpaged_prefill_kernel", "mode": "relocate",
+                       "achieved": k3, "peak": peak, "unit": UNIT, "frac": k3 / peak,
+                       "peak_kind": f"bf16 burst, {peak_kind}",
+                       "traffic": _recorded_traffic("segpaged_prefill_kernel", wl.name)}
+    if cpu_s > 0:
+        out["cpu_baseline"] = _cpu_baseline(lay, q, k.cpu(), v.cpu(), cpu_s, flops // (4 * lay.d))
+    del q, k, v
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -516,6 +617,10 @@ def main():
     ap.add_argument("--no-mask-penalty", action="store_true")
     ap.add_argument("--decode-batch", type=int, default=32)
     ap.add_argument("--no-importance", action="store_true")
+    ap.add_argument("--per-config", default="cfg1,cfg3,cfg4,cfg5",
+                    help="other workloads timed after the headline one ('' for none)")
+    ap.add_argument("--pc-steps", type=int, default=20)
+    ap.add_argument("--pc-cpu-seconds", type=float, default=6.0)
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -582,6 +687,7 @@ def main():
     if st != 0:
         raise SystemExit(f"device error word {st:#x} after the timed steps")
     ms_per_step = total_ms / K
+    launches = K * pre.launches_per_run
     value = weak_scaling_value(world, flops, K, total_ms) / 1e12
 
     # end to end through the public API: pinned host inputs in, o back to
@@ -656,21 +762,18 @@ def main():
 
     cpu_baseline = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
-        # batches of seeded rows until about args.cpu_seconds of oracle time
-        n_rows, tot_rows, tot_pairs, tot_t, seed = 1024, 0, 0, 0.0, 1
-        while tot_t < args.cpu_seconds:
-            rows, pairs = _oracle_sample_rows(lay, n_rows, seed=seed)
-            tot_t += _time_oracle(lay, qc, kc, vc, rows)
-            tot_rows += n_rows
-            tot_pairs += pairs
-            seed += 1
-            n_rows = min(2 * n_rows, 65536)
-        cpu_baseline = {"value": 4 * lay.d * tot_pairs / tot_t / 1e12, "unit": UNIT,
-                        "cores": os.cpu_count() or 1, "kind": "oracle",
-                        "sample": f"{tot_rows} seeded (layer, q head, row) samples of the same "
-                                  f"workload in {seed - 1} batches, {tot_pairs} visible pairs, "
-                                  f"{tot_t:.1f} s"}
+        cpu_baseline = _cpu_baseline(lay, q, k.cpu(), v.cpu(), args.cpu_seconds, flops // (4 * lay.d))
+
+    per_config = None
+    if world == 1 and args.per_config:
+        per_config = {}
+        del pre
+        torch.cuda.empty_cache()
+        for name in [c for c in args.per_config.split(",") if c and c != args.config]:
+            per_config[name] = _bench_config(torch, name, dev, flush, stream, min(K, args.pc_steps),
+                                             args.warmup, peaks, peak_kind,
+                                             0.0 if args.no_cpu_baseline else args.pc_cpu_seconds)
+            torch.cuda.empty_cache()
 
     if world > 1:
         dist.barrier()
@@ -697,7 +800,7 @@ def main():
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / E, "pipelined": True,
                 "serial_ms_per_step": serial_ms_per_step},
-        "gpu_launches": K * pre.launches_per_run,
+        "gpu_launches": launches,
         "clocks": clocks,
         "mode": args.mode,
         "other_mode": other_mode,
@@ -706,6 +809,7 @@ def main():
         "mask_penalty": mask_penalty,
         "decode_roofline": decode,
         "importance_roofline": importance,
+        "per_config": per_config,
     }
     print(json.dumps(line), flush=True)
     return 0

@@ -114,20 +114,6 @@ enum : int {
   kBarKFull = 25,  // k_full, k_ready, k_empty [kKStages] each, then v_full, v_empty [kVStages]
 };
 
-// kEmuNum pairs of exponentials in every kEmuDen can go through the FMA-pipe
-// polynomial instead of the MUFU (16 ex2 per clock per SM).  Measured on
-// B200 at D = 128, FP32 work on a sub-partition slows that sub-partition's
-// MUFU, and every emulated fraction tried (1/8 to 5/8) was slower, so the
-// default keeps all exponentials on the MUFU.
-#ifndef RK_EMU_NUM
-#define RK_EMU_NUM 0
-#endif
-#ifndef RK_EMU_DEN
-#define RK_EMU_DEN 4
-#endif
-constexpr int kEmuNum = RK_EMU_NUM;
-constexpr int kEmuDen = RK_EMU_DEN;
-
 // Index of the r-th work item of this CTA, from the producer's two-slot ring
 // (-1 once the list is exhausted).  Every thread of a consuming role reads
 // the slot and arrives on its empty barrier.
@@ -708,12 +694,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           }
 #pragma unroll
           for (int k = 0; k < 32; ++k) {
-            if (k % kEmuDen >= kEmuDen - kEmuNum) {
-              exp2_poly_pair(sh[2 * k], sh[2 * k + 1], sh[2 * k], sh[2 * k + 1]);
-            } else {
-              sh[2 * k] = ex2_approx(sh[2 * k]);
-              sh[2 * k + 1] = ex2_approx(sh[2 * k + 1]);
-            }
+            sh[2 * k] = ex2_approx(sh[2 * k]);
+            sh[2 * k + 1] = ex2_approx(sh[2 * k + 1]);
           }
 #pragma unroll
           for (int k = 0; k < 32; ++k)

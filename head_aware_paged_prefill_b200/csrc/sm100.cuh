@@ -380,29 +380,4 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-// 2^x for a pair on the FMA pipe (keeps the MUFU free for the other
-// elements).  x = n + f with n = round(x) obtained by adding 1.5 * 2^23
-// (round to nearest), f in [-1/2, 1/2]; 2^f by a degree-3 polynomial whose
-// coefficients were fitted for minimum relative error on that interval
-// (max relative error 7.5e-5, far below bf16's 2^-9); 2^n enters through the
-// exponent field.  Inputs below -125 are clamped, so the result is at least
-// 2^-125 instead of 0: negligible next to any finite softmax weight.
-__device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float& y0, float& y1) {
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-  x0 = fmaxf(x0, -125.0f);
-  x1 = fmaxf(x1, -125.0f);
-  const uint64_t x = f2_pack(x0, x1);
-  const uint64_t rnd = f2_pack(kRound, kRound);
-  const uint64_t t = f2_add(x, rnd);
-  const uint64_t f = f2_sub(x, f2_sub(t, rnd));
-  uint64_t p = f2_fma(f2_pack(0.05517166f, 0.05517166f), f, f2_pack(0.24261114f, 0.24261114f));
-  p = f2_fma(p, f, f2_pack(0.69326097f, 0.69326097f));
-  p = f2_fma(p, f, f2_pack(0.99992806f, 0.99992806f));
-  float p0, p1, t0, t1;
-  f2_unpack(p, p0, p1);
-  f2_unpack(t, t0, t1);
-  y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
-  y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
-}
-
 }  // namespace rk

@@ -5,6 +5,9 @@ number of keys the row attends to, counted from each class's rule in closed
 form.  Algorithmic FLOPs of the attention are 4 * D per visible pair
 (2 D for q.k, 2 D for p.v); exp, masking and rotation are not counted.
 
+row_visible_keys / table_rows: the same rules per sampled row (the CPU
+baseline's row samples).
+
 relocate_bytes(jobs, p, d): bytes an rk_relocate_rope pass must move
 (read + write of every page it touches).
 
@@ -61,6 +64,39 @@ def visible_pairs(lay) -> int:
                 else:
                     total += g * L * (L + 1) // 2
     return int(total)
+
+
+def row_visible_keys(lay, r: int, layer: int, kvh: int, rows: np.ndarray) -> np.ndarray:
+    """Visible keys of each request-local row in ``rows`` (rows of the table's
+    row set) for table (r, layer, kvh), from the class rules in closed form."""
+    rows = np.asarray(rows, dtype=np.int64)
+    c = int(lay.class_map[layer * lay.hkv + kvh])
+    if c == LOCAL:
+        return np.minimum(rows + 1, int(lay.class_window[LOCAL]))
+    if c != RETRIEVAL:
+        return rows + 1
+    P, L = lay.p, lay.req_len(r)
+    unc = _uncached_mask(lay, r)
+    n_unc_le = np.cumsum(unc.astype(np.int64))
+    t = lay.table_index(r, layer, kvh)
+    pages = np.unique(lay.retr_pages[lay.retr_indptr[t]:lay.retr_indptr[t + 1]])
+    pages = pages[(pages >= 0) & (pages * P < L)]
+    pages = pages[~unc[pages * P]]
+    cnt = n_unc_le[rows].copy()
+    for k in pages:
+        first, last = int(k) * P, min(int(k) * P + P, L) - 1
+        cnt += np.clip(rows - first + 1, 0, last - first + 1)
+    return cnt
+
+
+def table_rows(lay, r: int, layer: int, kvh: int) -> np.ndarray:
+    """Request-local rows a table computes: every position for global and
+    dense heads, the uncached positions for local and retrieval heads."""
+    c = int(lay.class_map[layer * lay.hkv + kvh])
+    L = lay.req_len(r)
+    if c in (LOCAL, RETRIEVAL):
+        return np.nonzero(_uncached_mask(lay, r))[0].astype(np.int64)
+    return np.arange(L, dtype=np.int64)
 
 
 def attention_flops(lay) -> int:

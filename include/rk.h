@@ -155,7 +155,10 @@ rk_status rk_query_sizes(const rk_dims* dims, const rk_layout* layout, rk_sizes*
  * workspace for rk_segpaged_prefill.  Copies the layout into the workspace
  * (stream-ordered; the host arrays may be reused once the call returns).
  * workspace: device, >= rk_sizes.workspace_bytes, 256-byte aligned; it also
- * holds the device error word, which this call resets.
+ * holds the device error word, which this call resets.  The layout image is
+ * uploaded with cudaMemcpyAsync from a host buffer that the call owns and
+ * frees before it returns, so the call is meant to be issued directly on
+ * the stream, not recorded into a CUDA graph.
  * Errors (host): RK_ERR_INVALID_ARG, RK_ERR_UNALIGNED, RK_ERR_CAPACITY,
  * RK_ERR_CUDA.  Device: RK_DEV_BAD_PAGE, RK_DEV_CAPACITY. */
 rk_status rk_select_visible(const rk_dims* dims, const rk_layout* layout, const rk_visible* out,
@@ -227,7 +230,10 @@ rk_status rk_selftest_bounded_wait(int32_t* device_word, int32_t wait_ms, void* 
  *     item offsets, plus about 8.5 KB of fixed fields) is rejected with
  *     RK_ERR_CAPACITY before any GPU work.
  *   - The first call on a device looks up the scratch's device address with
- *     that device current; make that first call before any stream capture.
+ *     that device current (cudaGetSymbolAddress, once per device); make that
+ *     first call before any stream capture on the device.  This note is
+ *     about the set-up only and says nothing about whether the call itself
+ *     can be captured.
  *   - Every call shares the one scratch array and rewrites all of it that it
  *     reads.  Calls whose GPU work overlaps (other streams, other threads)
  *     race on it: order them on one stream.

@@ -134,6 +134,41 @@ def test_importance_top_k_edges():
             assert tokens[0, 0, :L].tolist() == list(range(L))
 
 
+def _multi_chunk_layout(kind: str):
+    """Layouts whose tables span several row chunks of the column-sum kernel
+    (a chunk holds 8192 (row, q head) columns, 8192 / G rows), so partial
+    sums from different chunks and key blocks must land in the right slots.
+      "g4": Hq 12, Hkv 3 (G 4, 2048-row chunks), L 6220: one global, one
+            local (W 1536) and one retrieval head (16 cached pages), tail
+            ending mid-page.
+      "g8": Hq 16, Hkv 2 (G 8, 1024-row chunks), L 4100: a dense and a local
+            (W 700) head, P 16, D 128."""
+    if kind == "g4":
+        segs = [(f"c{i}", 1024, 512 * i, True) for i in range(5)] + [("tail", 1100, 0, False)]
+        picks = [1, 4, 9, 15, 22, 30, 37, 41, 50, 55, 58, 61, 66, 70, 74, 79]
+        lay = synth._make_layout(n_layers=1, hq=12, hkv=3, d=64, p=64, theta=1e6,
+                                 requests=[segs],
+                                 class_map=[synth.GLOBAL, synth.LOCAL, synth.RETRIEVAL],
+                                 window=1536, retrieval={2: picks})
+    else:
+        segs = [(f"c{i}", 1024, 3000 - 1000 * i, True) for i in range(3)] + [("tail", 1028, 0, False)]
+        lay = synth._make_layout(n_layers=1, hq=16, hkv=2, d=128, p=16, theta=1e4,
+                                 requests=[segs], class_map=[synth.DENSE, synth.LOCAL],
+                                 window=700)
+    return synth.tiny_workload(lay, seed=77 if kind == "g4" else 78)
+
+
+@pytest.mark.parametrize("kind", ["g4", "g8"])
+def test_importance_multi_chunk_against_oracle(kind):
+    """Element by element against the oracle on layouts of 3-4 row chunks
+    (the full-size cases below can only check invariants)."""
+    wl = _multi_chunk_layout(kind)
+    lay = wl.layout
+    g = lay.hq // lay.hkv
+    assert lay.req_len(0) > 2 * (8192 // g)  # at least three chunks
+    _case(wl, lay.req_len(0) // 4, f"multi-chunk {kind}")
+
+
 @pytest.mark.parametrize("name", ["cfg2", "cfg4"])
 def test_importance_full_size_invariants(name):
     wl = synth.CONFIGS[name]()

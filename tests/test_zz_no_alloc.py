@@ -8,6 +8,7 @@ not see anything left over from the first.  This file is collected last so a
 run that stops at the first failure has run every other test before it.
 """
 import ctypes
+import dataclasses
 
 import numpy as np
 import pytest
@@ -60,3 +61,28 @@ def test_noalloc_rejects_layout_beyond_scratch():
     st = binding.lib().rk_select_visible_noalloc(ctypes.byref(hl.dims), ctypes.byref(hl.layout),
                                                  ctypes.byref(vis), None, None)
     assert st == binding.RK_ERR_CAPACITY
+
+
+@pytest.mark.gpu
+def test_noalloc_rejected_call_leaves_no_trace():
+    """A page id outside the pool is caught on the host (RK_ERR_INVALID_ARG)
+    before any GPU work: the caller's error word keeps its old value.  The
+    next, valid call rewrites the shared scratch header and reports 0."""
+    lay = synth.cfg1().layout
+    bad = dataclasses.replace(lay, page_base=lay.page_base.copy())
+    bad.page_base[0, 0] = lay.n_pages  # the segment's pages run past the pool
+    hl = binding.HostLayout(bad)
+    s = binding.HostLayout(lay).sizes()
+    vis = binding.Visible(s, "cuda")
+    err = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    st = binding.lib().rk_select_visible_noalloc(ctypes.byref(hl.dims), ctypes.byref(hl.layout),
+                                                 ctypes.byref(vis.struct), ctypes.c_void_p(err.data_ptr()),
+                                                 None)
+    assert st == binding.RK_ERR_INVALID_ARG
+    torch.cuda.synchronize()
+    assert int(err.item()) == -1
+    got_e, got_r = _tables_with(lay, noalloc=True)
+    want_e, want_r = _tables_with(lay, noalloc=False)
+    for t in range(lay.n_tables):
+        np.testing.assert_array_equal(got_e[t], want_e[t])
+        np.testing.assert_array_equal(got_r[t], want_r[t])
