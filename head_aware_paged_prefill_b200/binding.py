@@ -117,7 +117,7 @@ class RkDecodeSizes(ctypes.Structure):
 
 
 class RkImportanceSizes(ctypes.Structure):
-    _fields_ = [("max_blocks", ctypes.c_int64), ("workspace_bytes", ctypes.c_int64)]
+    _fields_ = [("n_items", ctypes.c_int64), ("workspace_bytes", ctypes.c_int64)]
 
 
 class RkScoreSizes(ctypes.Structure):

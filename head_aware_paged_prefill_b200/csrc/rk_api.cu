@@ -785,35 +785,153 @@ extern "C" rk_status rk_segpaged_decode(const rk_dims* dims, const rk_layout* la
 
 namespace rk {
 namespace {
+// Host plan of one rk_attention_importance call.  The work items of a table
+// are (256-key block, row chunk) pairs: the key block's entries come from the
+// table's page table, which follows the class rule of the select kernel and
+// is therefore known here from the layout alone; the row chunk is one of
+// kImpChunkCols / G rows that holds a row able to see a key of the block.
+// The plan kernel rebuilds the same items from the device page tables and
+// checks the count of every table against tplan.
 struct ImportancePlan {
-  int max_blocks = 0, n_chunks = 0;
-  size_t off_cu = 0, off_part = 0, part_bytes = 0, total = 0;
+  int64_t n_items = 0;
+  int max_kb = 0, max_chunks = 0, max_pages = 0;
+  std::vector<int32_t> upload;  // cu [n_req + 1], padding, tplan [n_tables] (offset, items)
+  size_t off_cu = 0, off_tplan = 0, off_kbinfo = 0, off_chunkinfo = 0, off_inv = 0;
+  size_t off_items = 0, off_part = 0, total = 0;
 };
+
+// Request-logical page starts of table t's entries (ascending), by the rule
+// rk_select_visible applies: every page for global / dense heads; for local
+// heads the pages holding a key of some uncached segment's window
+// [a - W + 1, b - 1]; for retrieval heads the uncached pages and the listed
+// cached pages that start at or before the last uncached position.
+void importance_table_pages(const rk_dims* d, const rk_layout* lay, const Derived& dv, int r,
+                            int lh, int64_t t, std::vector<int>* out) {
+  out->clear();
+  const int P = d->page_size, L = lay->cu_seqlens[r + 1] - lay->cu_seqlens[r];
+  const int cls = lay->class_map[lh];
+  const int W = lay->class_window[RK_LOCAL];
+  const int s0 = dv.seg_indptr[r], s1 = dv.seg_indptr[r + 1];
+  int last_unc = -1;
+  for (int s = s0; s < s1; ++s)
+    if (!lay->segments[s].cached)
+      last_unc = std::max(last_unc, lay->segments[s].logical_start + lay->segments[s].len - 1);
+  std::vector<int> listed;
+  if (cls == RK_RETRIEVAL && lay->retr_indptr)
+    listed.assign(lay->retr_pages + lay->retr_indptr[t], lay->retr_pages + lay->retr_indptr[t + 1]);
+  std::sort(listed.begin(), listed.end());
+  for (int s = s0; s < s1; ++s) {
+    const rk_segment& g = lay->segments[s];
+    for (int pos = g.logical_start; pos < g.logical_start + g.len; pos += P) {
+      const int nv = std::min(P, L - pos);
+      bool flag = false;
+      if (cls == RK_GLOBAL || cls == RK_DENSE) {
+        flag = true;
+      } else if (cls == RK_LOCAL) {
+        for (int u = s0; u < s1 && !flag; ++u) {
+          const rk_segment& x = lay->segments[u];
+          if (x.cached) continue;
+          flag = std::max(pos, x.logical_start - W + 1) <=
+                 std::min(pos + nv - 1, x.logical_start + x.len - 1);
+        }
+      } else {
+        flag = !g.cached ||
+               (pos <= last_unc && std::binary_search(listed.begin(), listed.end(), pos / P));
+      }
+      if (flag) out->push_back(pos);
+    }
+  }
+}
+
 rk_status plan_importance(const rk_dims* d, const rk_layout* lay, const Derived& dv,
                           ImportancePlan* out) {
   const int g = d->num_q_heads / d->num_kv_heads;
   if (g > kImpMaxG || dv.n_lh > kImpMaxLh) return RK_ERR_INVALID_ARG;
-  int64_t max_pages = 0;
-  for (int r = 0; r < d->n_req; ++r)
-    max_pages = std::max<int64_t>(max_pages, dv.page_prefix[r + 1] - dv.page_prefix[r]);
-  const int64_t keys = max_pages * d->page_size;
-  const int64_t blocks = (keys + kImpKeysPerCta - 1) / kImpKeysPerCta;
-  if (blocks > 65535) return RK_ERR_CAPACITY;
-  out->max_blocks = static_cast<int>(blocks);
-  int64_t max_len = 0;
-  for (int r = 0; r < d->n_req; ++r)
-    max_len = std::max<int64_t>(max_len, lay->cu_seqlens[r + 1] - lay->cu_seqlens[r]);
-  const int64_t rows_per_chunk = kImpChunkCols / g;
-  const int64_t chunks = std::max<int64_t>(1, (max_len + rows_per_chunk - 1) / rows_per_chunk);
-  if (chunks > 65535) return RK_ERR_CAPACITY;
-  out->n_chunks = static_cast<int>(chunks);
-  // the first 256 bytes hold the device error word, then cu_seqlens, then the
-  // per-(layer, kv head, row chunk, token) partial sums
+  const int P = d->page_size, EPK = kImpKeysPerBlock / P, RPC = kImpChunkCols / g;
+  const int n_req = d->n_req, hkv = d->num_kv_heads;
+  std::vector<int64_t> items(static_cast<size_t>(dv.n_tables), 0);
+  std::vector<int> pages;
+  std::vector<std::pair<int, int>> rows;
+  int max_kb = 0, max_chunks = 0, max_pages = 0;
+  for (int r = 0; r < n_req; ++r) {
+    const int L = lay->cu_seqlens[r + 1] - lay->cu_seqlens[r];
+    max_pages = std::max(max_pages, (L + P - 1) / P);
+    max_chunks = std::max(max_chunks, (L + RPC - 1) / RPC);
+    std::vector<std::pair<int, int>> unc;  // merged uncached ranges
+    for (int s = dv.seg_indptr[r]; s < dv.seg_indptr[r + 1]; ++s) {
+      const rk_segment& x = lay->segments[s];
+      if (x.cached) continue;
+      if (!unc.empty() && unc.back().second == x.logical_start) unc.back().second += x.len;
+      else unc.emplace_back(x.logical_start, x.logical_start + x.len);
+    }
+    for (int layer = 0; layer < d->n_layers; ++layer)
+      for (int kvh = 0; kvh < hkv; ++kvh) {
+        const int lh = layer * hkv + kvh;
+        const int64_t t = (static_cast<int64_t>(r) * d->n_layers + layer) * hkv + kvh;
+        const int cls = lay->class_map[lh];
+        const bool local = cls == RK_LOCAL;
+        rows.clear();
+        if (cls == RK_GLOBAL || cls == RK_DENSE) {
+          if (L > 0) rows.emplace_back(0, L);
+        } else {
+          rows = unc;
+        }
+        if (rows.empty()) continue;
+        importance_table_pages(d, lay, dv, r, lh, t, &pages);
+        const int n_e = static_cast<int>(pages.size());
+        const int n_kb = (n_e + EPK - 1) / EPK;
+        max_kb = std::max(max_kb, n_kb);
+        int64_t cnt = 0;
+        for (int kb = 0; kb < n_kb; ++kb) {
+          const int e0 = kb * EPK, e1 = std::min(n_e, e0 + EPK);
+          const int pos_lo = pages[e0];
+          const int pos_hi = pages[e1 - 1] + std::min(P, L - pages[e1 - 1]) - 1;
+          const int hi = local ? std::min(L - 1, pos_hi + lay->class_window[RK_LOCAL] - 1) : L - 1;
+          int f = -1, l = -1;
+          for (const auto& x : rows)
+            if (x.second > pos_lo) { f = std::max(x.first, pos_lo); break; }
+          for (auto it = rows.rbegin(); it != rows.rend(); ++it)
+            if (it->first <= hi) { l = std::min(it->second - 1, hi); break; }
+          if (f >= 0 && l >= 0) cnt += std::max(0, l / RPC - f / RPC + 1);
+        }
+        items[static_cast<size_t>(t)] = cnt;
+      }
+  }
+  // the work list: tables with more items first (a longest-first order at
+  // table granularity), each table's items contiguous
+  std::vector<int64_t> order(static_cast<size_t>(dv.n_tables));
+  for (int64_t t = 0; t < dv.n_tables; ++t) order[static_cast<size_t>(t)] = t;
+  std::stable_sort(order.begin(), order.end(),
+                   [&](int64_t x, int64_t y) { return items[x] > items[y]; });
+  std::vector<int64_t> off(static_cast<size_t>(dv.n_tables), 0);
+  int64_t acc = 0;
+  for (int64_t t : order) {
+    off[static_cast<size_t>(t)] = acc;
+    acc += items[static_cast<size_t>(t)];
+  }
+  if (acc >= kMaxI32 / kImpKeysPerBlock) return RK_ERR_CAPACITY;
+  out->n_items = acc;
+  out->max_kb = std::max(max_kb, 1);
+  out->max_chunks = std::max(max_chunks, 1);
+  out->max_pages = std::max(max_pages, 1);
+  const size_t cu_words = align_up(static_cast<size_t>(n_req + 1), 2);
+  out->upload.assign(cu_words + 2 * static_cast<size_t>(dv.n_tables), 0);
+  for (int r = 0; r <= n_req; ++r) out->upload[r] = lay->cu_seqlens[r];
+  for (int64_t t = 0; t < dv.n_tables; ++t) {
+    out->upload[cu_words + 2 * t] = static_cast<int32_t>(off[static_cast<size_t>(t)]);
+    out->upload[cu_words + 2 * t + 1] = static_cast<int32_t>(items[static_cast<size_t>(t)]);
+  }
+  // workspace: header (error word, timeout site, work counter), the upload,
+  // the plan kernel's index arrays, the work list and one partial per item
+  const size_t nt = static_cast<size_t>(dv.n_tables);
   out->off_cu = 256;
-  out->off_part = align_up(out->off_cu + 4 * static_cast<size_t>(d->n_req + 1), 256);
-  out->part_bytes = 4 * static_cast<size_t>(d->n_layers) * d->num_kv_heads * out->n_chunks *
-                    static_cast<size_t>(d->total_tokens);
-  out->total = align_up(out->off_part + out->part_bytes, 256);
+  out->off_tplan = out->off_cu + 4 * cu_words;
+  out->off_kbinfo = align_up(out->off_cu + 4 * out->upload.size(), 256);
+  out->off_chunkinfo = align_up(out->off_kbinfo + 8 * nt * out->max_kb, 256);
+  out->off_inv = align_up(out->off_chunkinfo + 8 * nt * out->max_chunks, 256);
+  out->off_items = align_up(out->off_inv + 4 * nt * out->max_pages, 256);
+  out->off_part = align_up(out->off_items + 16 * static_cast<size_t>(acc), 256);
+  out->total = align_up(out->off_part + 4 * static_cast<size_t>(kImpKeysPerBlock) * acc, 256);
   return RK_OK;
 }
 }  // namespace
@@ -828,7 +946,7 @@ extern "C" rk_status rk_importance_query_sizes(const rk_dims* dims, const rk_lay
   if ((st = check_layout(dims, layout, &dv)) != RK_OK) return st;
   ImportancePlan plan;
   if ((st = plan_importance(dims, layout, dv, &plan)) != RK_OK) return st;
-  out->max_blocks = plan.max_blocks;
+  out->n_items = plan.n_items;
   out->workspace_bytes = static_cast<int64_t>(plan.total);
   return RK_OK;
 }
@@ -863,9 +981,8 @@ extern "C" rk_status rk_attention_importance(const rk_dims* dims, const rk_layou
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   if (cudaMemsetAsync(ws, 0, 256, s) != cudaSuccess ||
-      cudaMemcpyAsync(ws + plan.off_cu, layout->cu_seqlens, 4 * static_cast<size_t>(dims->n_req + 1),
-                      cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemsetAsync(ws + plan.off_part, 0, plan.part_bytes, s) != cudaSuccess)
+      cudaMemcpyAsync(ws + plan.off_cu, plan.upload.data(), 4 * plan.upload.size(),
+                      cudaMemcpyHostToDevice, s) != cudaSuccess)
     return RK_ERR_CUDA;
   ImportanceLaunchArgs a{};
   a.q = q;
@@ -877,11 +994,18 @@ extern "C" rk_status rk_attention_importance(const rk_dims* dims, const rk_layou
   a.range_start = vis->range_start;
   a.range_count = vis->range_count;
   a.cu = reinterpret_cast<const int32_t*>(ws + plan.off_cu);
-  a.lse = lse;
+  a.tplan = reinterpret_cast<const int2*>(ws + plan.off_tplan);
+  a.kbinfo = reinterpret_cast<int2*>(ws + plan.off_kbinfo);
+  a.chunkinfo = reinterpret_cast<int2*>(ws + plan.off_chunkinfo);
+  a.inv = reinterpret_cast<int32_t*>(ws + plan.off_inv);
+  a.items = reinterpret_cast<int4*>(ws + plan.off_items);
   a.part = reinterpret_cast<float*>(ws + plan.off_part);
+  a.lse = lse;
   a.importance = importance;
   a.tokens = tokens;
   a.token_count = token_count;
+  a.work_next = reinterpret_cast<int*>(ws + 8);
+  a.timeout_site = reinterpret_cast<int*>(ws + 4);
   a.n_pages = dims->n_pages;
   a.n_req = dims->n_req;
   a.n_layers = dims->n_layers;
@@ -892,8 +1016,10 @@ extern "C" rk_status rk_attention_importance(const rk_dims* dims, const rk_layou
   a.total_tokens = dims->total_tokens;
   a.window = layout->class_window[RK_LOCAL];
   a.top_k = top_k;
-  a.max_blocks = plan.max_blocks;
-  a.n_chunks = plan.n_chunks;
+  a.n_items = static_cast<int>(plan.n_items);
+  a.max_kb = plan.max_kb;
+  a.max_chunks = plan.max_chunks;
+  a.max_pages = plan.max_pages;
   a.softmax_scale = softmax_scale;
   a.cls = layout->class_map;
   a.error_word = reinterpret_cast<int32_t*>(ws);

@@ -186,10 +186,10 @@ struct DecodeLaunchArgs {
 cudaError_t launch_decode(const DecodeLaunchArgs& a, cudaStream_t stream);
 
 // ---- attention importance (sparse FFN token selection)
-constexpr int kImpKeysPerCta = 128;  // keys of one table per column-sum CTA
-constexpr int kImpChunkCols = 8192;  // (row, q head) columns per row chunk: 8192 / G rows
-constexpr int kImpMaxLh = 1024;      // layers x kv heads per call
-constexpr int kImpMaxG = 8;          // q heads per kv head
+constexpr int kImpKeysPerBlock = 256;  // keys of one table per work item (two MMA halves)
+constexpr int kImpChunkCols = 4096;    // (row, q head) columns per row chunk: 4096 / G rows
+constexpr int kImpMaxLh = 1024;        // layers x kv heads per call
+constexpr int kImpMaxG = 8;            // q heads per kv head
 
 struct ImportanceLaunchArgs {
   const void* q;       // bf16 [n_layers][T][hq][d], the prefill's queries
@@ -200,14 +200,22 @@ struct ImportanceLaunchArgs {
   const rk_range* ranges;
   const int32_t* range_start;
   const int32_t* range_count;
-  const int32_t* cu;   // device [n_req + 1]
-  const float* lse;    // fp32 [n_layers][hq][T], natural log (the prefill's)
-  float* part;         // fp32 [n_layers][hkv][n_chunks][T], zeroed by the caller
-  float* importance;   // fp32 [n_layers][T]
-  int32_t* tokens;     // [n_layers][n_req][top_k] or null
+  const int32_t* cu;     // device [n_req + 1]
+  const int2* tplan;     // device [n_tables]: (work-list offset, items) of each table
+  int2* kbinfo;          // device [n_tables][max_kb]
+  int2* chunkinfo;       // device [n_tables][max_chunks]
+  int32_t* inv;          // device [n_tables][max_pages]
+  int4* items;           // device [n_items]
+  float* part;           // device [n_items][kImpKeysPerBlock]
+  const float* lse;      // fp32 [n_layers][hq][T], natural log (the prefill's)
+  float* importance;     // fp32 [n_layers][T]
+  int32_t* tokens;       // [n_layers][n_req][top_k] or null
   int32_t* token_count;  // [n_layers][n_req] or null
+  int* work_next;        // zeroed by the caller
+  int* timeout_site;
   int64_t n_pages;
-  int n_req, n_layers, hq, hkv, d, p, total_tokens, window, top_k, max_blocks, n_chunks;
+  int n_req, n_layers, hq, hkv, d, p, total_tokens, window, top_k;
+  int n_items, max_kb, max_chunks, max_pages;
   float softmax_scale;
   const int8_t* cls;   // host [n_layers * hkv]
   int32_t* error_word;

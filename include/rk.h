@@ -354,13 +354,18 @@ rk_status rk_segpaged_decode(const rk_dims* dims, const rk_layout* layout, const
  * accumulation; I is >= 0 (a NaN lse ranks its tokens first). */
 
 typedef struct {
-  int64_t max_blocks;      /* column-sum CTAs per table (128 keys each) */
+  /* work items: (table, block of 256 page-table keys, row chunk of 4096 / G
+   * rows) triples whose rows can see a key of the block; the workspace keeps
+   * one 256-float partial sum per item */
+  int64_t n_items;
   int64_t workspace_bytes; /* device workspace for rk_attention_importance */
 } rk_importance_sizes;
 
-/* Validates dims + layout and reports the workspace size.  Hq / Hkv <= 8,
- * n_layers * Hkv <= 1024, and a request of at most 65535 * 128 keys.  Host
- * only.  Errors: RK_ERR_INVALID_ARG, RK_ERR_UNALIGNED, RK_ERR_CAPACITY. */
+/* Validates dims + layout and reports the workspace size (exact: the items
+ * follow from the layout's page tables, which the class rule fixes).
+ * Hq / Hkv <= 8 and n_layers * Hkv <= 1024.  Host only.  Errors:
+ * RK_ERR_INVALID_ARG, RK_ERR_UNALIGNED, RK_ERR_CAPACITY (more than 2^23
+ * items). */
 rk_status rk_importance_query_sizes(const rk_dims* dims, const rk_layout* layout,
                                     rk_importance_sizes* out);
 
@@ -378,8 +383,10 @@ rk_status rk_importance_query_sizes(const rk_dims* dims, const rk_layout* layout
  *           the selection.
  *   workspace: device, >= rk_importance_sizes.workspace_bytes, 256-byte
  *           aligned; its first word is the device error word
- *           (RK_DEV_BAD_PAGE), reset by this call and read by
- *           rk_get_device_status.
+ *           (RK_DEV_BAD_PAGE; RK_DEV_CAPACITY if the page tables in `vis`
+ *           do not belong to `layout`; RK_DEV_TIMEOUT), reset by this call
+ *           and read by rk_get_device_status.  Not shared with a concurrent
+ *           call.
  * Errors (host): RK_ERR_INVALID_ARG, RK_ERR_UNALIGNED, RK_ERR_CAPACITY,
  * RK_ERR_CUDA. */
 rk_status rk_attention_importance(const rk_dims* dims, const rk_layout* layout, const void* q,

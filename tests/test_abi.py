@@ -7,6 +7,7 @@ import re
 import numpy as np
 import pytest
 
+import oracle
 from head_aware_paged_prefill_b200 import binding, synth
 from head_aware_paged_prefill_b200.csrc import build as build_mod
 
@@ -204,10 +205,8 @@ def test_importance_calls_validate_on_host(lib):
     lay = synth.cfg1().layout
     hl = _hl(lay)
     s = binding.importance_sizes(hl)
-    keys = -(-lay.req_len(0) // lay.p) * lay.p
-    assert s.max_blocks == -(-keys // 128)
-    T = int(lay.cu_seqlens[-1])
-    assert s.workspace_bytes >= 256 + 4 * lay.n_layers * lay.hkv * T
+    assert s.n_items == _importance_items_brute(lay)
+    assert s.workspace_bytes >= 256 + 4 * 256 * s.n_items
     assert s.workspace_bytes % 256 == 0
     sz = hl.sizes()
     fake = ctypes.c_void_p(1 << 20)
@@ -237,15 +236,84 @@ def test_importance_calls_validate_on_host(lib):
     assert call(a4=ctypes.byref(small)) == C
 
 
-@pytest.mark.parametrize("name", ["cfg2", "cfg4"])
-def test_importance_workspace_covers_row_chunks(lib, name):
-    """The column-sum partials are kept per row chunk of 8192 / G rows, so
-    the workspace holds n_layers x Hkv x chunks x T floats."""
+KB = 256          # keys per importance work item
+CHUNK_COLS = 4096  # (row, q head) columns per row chunk
+
+
+def _importance_items_brute(lay) -> int:
+    """Importance work items by brute force: for every table and every block
+    of 256 consecutive page-table keys, the row chunks (CHUNK_COLS / G rows)
+    from the one holding the first row that sees a key of the block to the
+    one holding the last such row (visibility from the oracle's brute-force
+    page tables and the class rule)."""
+    entries, ranges = oracle.page_tables(lay)
+    g = lay.hq // lay.hkv
+    rpc = CHUNK_COLS // g
+    W = int(lay.class_window[synth.LOCAL])
+    n = 0
+    for t in range(lay.n_tables):
+        r, rem = divmod(t, lay.n_layers * lay.hkv)
+        cls = int(lay.class_map[rem])
+        rows = [i for a, b in ranges[t] for i in range(a, b)]
+        epk = KB // lay.p
+        ent = entries[t]
+        for kb in range(-(-ent.shape[0] // epk)):
+            blk = [int(e[1]) + k for e in ent[kb * epk: kb * epk + epk] for k in range(int(e[3]))]
+            seeing = [i for i in rows
+                      if any(k <= i and (cls != synth.LOCAL or i - k < W) for k in blk)]
+            if seeing:
+                n += seeing[-1] // rpc - seeing[0] // rpc + 1
+    return n
+
+
+def _importance_items_tail_layout(lay) -> int:
+    """The same count in closed form for layouts whose only uncached segment
+    is each request's last (the full-size workloads)."""
+    P, g, W = lay.p, lay.hq // lay.hkv, int(lay.class_window[synth.LOCAL])
+    rpc = CHUNK_COLS // g
+    entries, _ = oracle.page_tables_closed_form(lay)
+    n = 0
+    for t in range(lay.n_tables):
+        r, rem = divmod(t, lay.n_layers * lay.hkv)
+        cls = int(lay.class_map[rem])
+        L = lay.req_len(r)
+        segs = lay.segments_of(r)
+        unc = segs[segs[:, 4] == 0]
+        assert unc.shape[0] <= 1 and (unc.shape[0] == 0 or int(unc[0, 1] + unc[0, 2]) == L)
+        a = int(unc[0, 1]) if unc.shape[0] else L
+        rows = (0, L) if cls in (synth.GLOBAL, synth.DENSE) else (a, L)
+        if rows[0] >= rows[1]:
+            continue
+        e = entries[t]
+        epk = KB // P
+        for kb in range(-(-e.shape[0] // epk)):
+            blk = e[kb * epk: kb * epk + epk]
+            lo, hi = int(blk[0, 1]), int(blk[-1, 1] + blk[-1, 3] - 1)
+            first = max(lo, rows[0])
+            last = min(L - 1, hi + W - 1) if cls == synth.LOCAL else L - 1
+            if first <= last:
+                n += last // rpc - first // rpc + 1
+    return n
+
+
+def test_importance_items_match_brute_force(lib):
+    """The library's exact item count equals the brute-force count on random
+    small layouts (every class, windows, uncached segments anywhere)."""
+    rng = np.random.default_rng(12)
+    for _ in range(40):
+        lay = synth.random_small(rng, max_pages=40)
+        assert binding.importance_sizes(_hl(lay)).n_items == _importance_items_brute(lay)
+
+
+@pytest.mark.parametrize("name", ["cfg2", "cfg3", "cfg4", "cfg5"])
+def test_importance_workspace_exact(lib, name):
+    """The workspace holds one 1 KB partial per work item plus small index
+    arrays: no dense per-(chunk, token) buffer (the serving mix needs about
+    260 MB, not GBs)."""
     lay = synth.CONFIGS[name]().layout
     s = binding.importance_sizes(_hl(lay))
+    assert s.n_items == _importance_items_tail_layout(lay)
     g = lay.hq // lay.hkv
-    L = max(lay.req_len(r) for r in range(lay.n_req))
-    chunks = -(-L // (8192 // g))
-    T = int(lay.cu_seqlens[-1])
-    assert s.workspace_bytes >= 256 + 4 * lay.n_layers * lay.hkv * chunks * T
-    assert s.max_blocks == -(-(-(-L // lay.p) * lay.p) // 128)
+    max_pages = max(-(-lay.req_len(r) // lay.p) for r in range(lay.n_req))
+    index = 8 * lay.n_tables * (max_pages * lay.p // KB + 1 + max_pages // 8 + 1) + 4 * lay.n_tables * max_pages
+    assert 1024 * s.n_items <= s.workspace_bytes <= 1040 * s.n_items + index + 4096 + 8 * lay.n_tables

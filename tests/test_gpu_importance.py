@@ -169,7 +169,7 @@ def test_importance_multi_chunk_against_oracle(kind):
     _case(wl, lay.req_len(0) // 4, f"multi-chunk {kind}")
 
 
-@pytest.mark.parametrize("name", ["cfg2", "cfg4"])
+@pytest.mark.parametrize("name", ["cfg2", "cfg3", "cfg4", "cfg5"])
 def test_importance_full_size_invariants(name):
     wl = synth.CONFIGS[name]()
     lay = wl.layout
@@ -177,6 +177,8 @@ def test_importance_full_size_invariants(name):
     top_k = lay.req_len(0) // 4
     imp, tokens, count = _run(lay, q, k, v, top_k)
     _check_invariants(lay, imp, tokens, count, top_k, name)
+    del q, k, v
+    torch.cuda.empty_cache()
 
 
 def test_importance_deterministic():
