@@ -67,6 +67,10 @@ def _load():
                                        ctypes.c_double, ctypes.c_double, ctypes.c_int,
                                        ctypes.c_int, ctypes.c_void_p]
         lib.ora_importance.restype = ctypes.c_int
+        lib.ora_sparse_ffn.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p,
+                                       ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+                                       ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_int]
+        lib.ora_sparse_ffn.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -362,3 +366,24 @@ def attention(lay, q_rows_u16: np.ndarray, k_pool_u16: np.ndarray, v_pool_u16: n
                           float(lay.theta), float(lay.softmax_scale), rows.ctypes.data, n,
                           o.ctypes.data, lse.ctypes.data, comp.ctypes.data, _threads(threads))
     return o, lse, comp
+
+
+# ------------------------------------------------------------ sparse FFN
+
+def sparse_ffn(x_u16: np.ndarray, rows, w_gate_u16: np.ndarray, w_up_u16: np.ndarray,
+               w_down_u16: np.ndarray, threads=None) -> np.ndarray:
+    """fp64 token-selective FFN (rk_oracle.c, ora_sparse_ffn): for each listed
+    row i of x [., d_model], y_i = x_i + W_down (silu(W_gate x_i) * W_up x_i).
+    Weights are bf16 bits [d_ff][d_model] (gate, up) and [d_model][d_ff]
+    (down).  Returns fp64 [len(rows)][d_model]; unlisted rows are x itself."""
+    x = np.ascontiguousarray(x_u16.view(np.uint16))
+    wg = np.ascontiguousarray(w_gate_u16.view(np.uint16))
+    wu = np.ascontiguousarray(w_up_u16.view(np.uint16))
+    wd = np.ascontiguousarray(w_down_u16.view(np.uint16))
+    d_ff, d_model = wg.shape
+    assert x.shape[-1] == d_model and wu.shape == wg.shape and wd.shape == (d_model, d_ff)
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int32))
+    y = np.zeros((rows.shape[0], d_model), dtype=np.float64)
+    _load().ora_sparse_ffn(x.ctypes.data, d_model, rows.ctypes.data, rows.shape[0], wg.ctypes.data,
+                           wu.ctypes.data, wd.ctypes.data, d_ff, y.ctypes.data, _threads(threads))
+    return y

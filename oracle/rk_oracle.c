@@ -32,12 +32,16 @@
  *   - Token importance for the sparse FFN (ora_importance, a reading stated
  *     there): the prefill's softmax weights summed per token over q heads
  *     and computed rows.
+ *   - The token-selective FFN itself (ora_sparse_ffn, a reading stated
+ *     there): the gated SiLU MLP on the listed rows, residual elsewhere.
  *
  * parity pins: see tests/test_oracle_pins.py (RoPE closed form and
  * composition, causal and windowed SDPA special cases, perturbation
  * invariance, sharing, brute-force vs closed-form page tables, pair counts),
  * tests/test_oracle_scoring.py and tests/test_oracle_importance.py (dense
- * restatement, unit row sums, harmonic closed form, selection brute force).
+ * restatement, unit row sums, harmonic closed form, selection brute force),
+ * tests/test_oracle_ffn.py (hand-computed values, silu's odd-part identity,
+ * zero-gate and scaled-down-projection special cases).
  */
 #include <math.h>
 #include <pthread.h>
@@ -622,5 +626,92 @@ int ora_importance(const ora_problem* pr, const uint16_t* q, const uint16_t* k_p
   free(kr);
   free(s);
   free(qd);
+  return 0;
+}
+
+/* ------------------------------------------------------------ sparse FFN */
+
+/* Token-selective FFN (README "About", Elastic Sparsity / Sparse FFN; paooo
+ * page, "main functions": the tokens with the highest attention scores run
+ * the dense FFN, the others take the residual path).  The pages name the
+ * Mistral-7B and Qwen3 families, whose FFN is the gated SiLU MLP; the
+ * reading implemented here, for every listed row i of the hidden state x:
+ *   g_f = sum_c x_ic Wg_fc,   u_f = sum_c x_ic Wu_fc        (f < d_ff)
+ *   h_f = silu(g_f) u_f,      silu(z) = z / (1 + exp(-z))
+ *   y_in = x_in + sum_f h_f Wd_nf                           (n < d_model)
+ * and y_i = x_i for every other row (the residual path, not computed here).
+ * x: bf16 [.][d_model]; Wg, Wu: bf16 [d_ff][d_model]; Wd: bf16
+ * [d_model][d_ff] (rows are output features, as in a linear layer's
+ * weight); rows: the listed row indices; y_out: fp64 [n_rows][d_model].
+ * fp64 throughout, no intermediate rounding. */
+typedef struct {
+  const uint16_t *x, *wg, *wu, *wd;
+  const int32_t* rows;
+  int n_rows, d_model, d_ff;
+  double* y;
+  int next;
+  pthread_mutex_t mu;
+} ffn_job;
+
+static void ffn_row(ffn_job* j, int k) {
+  int dm = j->d_model, df = j->d_ff;
+  const uint16_t* xr = j->x + (size_t)j->rows[k] * dm;
+  double* xd = (double*)malloc(sizeof(double) * dm);
+  double* h = (double*)malloc(sizeof(double) * df);
+  for (int c = 0; c < dm; ++c) xd[c] = bf16_to_double(xr[c]);
+  for (int f = 0; f < df; ++f) {
+    const uint16_t* wgr = j->wg + (size_t)f * dm;
+    const uint16_t* wur = j->wu + (size_t)f * dm;
+    double g = 0.0, u = 0.0;
+    for (int c = 0; c < dm; ++c) {
+      g += xd[c] * bf16_to_double(wgr[c]);
+      u += xd[c] * bf16_to_double(wur[c]);
+    }
+    h[f] = g / (1.0 + exp(-g)) * u;
+  }
+  double* y = j->y + (size_t)k * dm;
+  for (int n = 0; n < dm; ++n) {
+    const uint16_t* wdr = j->wd + (size_t)n * df;
+    double acc = 0.0;
+    for (int f = 0; f < df; ++f) acc += h[f] * bf16_to_double(wdr[f]);
+    y[n] = xd[n] + acc;
+  }
+  free(xd);
+  free(h);
+}
+
+static void* ffn_worker(void* arg) {
+  ffn_job* j = (ffn_job*)arg;
+  for (;;) {
+    pthread_mutex_lock(&j->mu);
+    int k = j->next++;
+    pthread_mutex_unlock(&j->mu);
+    if (k >= j->n_rows) return NULL;
+    ffn_row(j, k);
+  }
+}
+
+int ora_sparse_ffn(const uint16_t* x, int d_model, const int32_t* rows, int n_rows,
+                   const uint16_t* wg, const uint16_t* wu, const uint16_t* wd, int d_ff,
+                   double* y_out, int n_threads) {
+  ffn_job j;
+  j.x = x;
+  j.wg = wg;
+  j.wu = wu;
+  j.wd = wd;
+  j.rows = rows;
+  j.n_rows = n_rows;
+  j.d_model = d_model;
+  j.d_ff = d_ff;
+  j.y = y_out;
+  j.next = 0;
+  pthread_mutex_init(&j.mu, NULL);
+  if (n_threads < 1) n_threads = 1;
+  if (n_threads > n_rows) n_threads = n_rows > 0 ? n_rows : 1;
+  pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * n_threads);
+  for (int k = 0; k < n_threads; ++k) pthread_create(&th[k], NULL, ffn_worker, &j);
+  for (int k = 0; k < n_threads; ++k) pthread_join(th[k], NULL);
+  free(th);
+  pthread_mutex_destroy(&j.mu);
   return 0;
 }

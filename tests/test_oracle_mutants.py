@@ -14,6 +14,7 @@ import oracle
 import test_oracle_pins as pins
 import test_oracle_scoring as scoring
 import test_oracle_importance as importance
+import test_oracle_ffn as ffn
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "rk_oracle.c")
 
@@ -51,6 +52,13 @@ MUTANTS = {
                             "kj[m] = x0 * cos(a) + x1 * sin(a);"),
     "importance_unscaled": ("s[j] = acc * scale;\n          if (s[j] > mx) mx = s[j];\n        }\n        if (mx == -INFINITY) continue;",
                             "s[j] = acc;\n          if (s[j] > mx) mx = s[j];\n        }\n        if (mx == -INFINITY) continue;"),
+    # token-selective FFN
+    "ffn_gate_up_swapped": ("h[f] = g / (1.0 + exp(-g)) * u;", "h[f] = u / (1.0 + exp(-u)) * g;"),
+    "ffn_no_residual": ("y[n] = xd[n] + acc;", "y[n] = acc;"),
+    "ffn_relu": ("h[f] = g / (1.0 + exp(-g)) * u;", "h[f] = (g > 0.0 ? g : 0.0) * u;"),
+    "ffn_sigmoid_sign": ("h[f] = g / (1.0 + exp(-g)) * u;", "h[f] = g / (1.0 + exp(g)) * u;"),
+    "ffn_down_transposed": ("const uint16_t* wdr = j->wd + (size_t)n * df;\n    double acc = 0.0;\n    for (int f = 0; f < df; ++f) acc += h[f] * bf16_to_double(wdr[f]);",
+                            "double acc = 0.0;\n    for (int f = 0; f < df; ++f) acc += h[f] * bf16_to_double(j->wd[(size_t)f * dm + n % dm]);"),
 }
 
 PIN_CALLS = [
@@ -69,6 +77,11 @@ PIN_CALLS = [
     importance.test_importance_is_dense_softmax_column_sums_cfg1,
     importance.test_importance_is_dense_softmax_column_sums_retrieval,
     importance.test_zero_keys_give_harmonic_sums,
+    ffn.test_one_feature_by_hand,
+    ffn.test_two_features_by_hand,
+    ffn.test_mirrored_features_give_a_bilinear_form,
+    ffn.test_zero_gate_is_the_residual_path,
+    ffn.test_down_projection_scales_the_update_and_rows_follow_the_list,
 ]
 
 
