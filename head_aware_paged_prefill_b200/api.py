@@ -200,6 +200,27 @@ class SegPagedPrefill:
         """Device error word of the last attention_importance call."""
         return binding.device_status(self._imp[1])
 
+    def sparse_ffn(self, x: torch.Tensor, tokens: torch.Tensor, top_k: int, w_gate: torch.Tensor,
+                   w_up: torch.Tensor, w_down: torch.Tensor, stream=None) -> torch.Tensor:
+        """The token-selective FFN of one layer (rk_sparse_ffn): the picked
+        tokens (``tokens`` [n_req][top_k], one layer of attention_importance's
+        output) of the hidden state x [T][d_model] take x + W_down (silu(W_gate
+        x) * W_up x), every other row keeps x.  Updates x in place and returns
+        it; the workspace is kept across calls of the same shape."""
+        lay = self.layout
+        key = (int(top_k), int(x.shape[1]), int(w_gate.shape[0]))
+        if getattr(self, "_ffn", None) is None or self._ffn[0] != key:
+            sizes = binding.ffn_sizes(lay.total_tokens, x.shape[1], w_gate.shape[0],
+                                      lay.cu_seqlens, top_k)
+            self._ffn = (key, binding.ffn_workspace(sizes, self.device))
+        binding.sparse_ffn(x, lay.cu_seqlens, tokens, top_k, w_gate, w_up, w_down, self._ffn[1],
+                           stream)
+        return x
+
+    def ffn_status(self) -> int:
+        """Device error word of the last sparse_ffn call."""
+        return binding.device_status(self._ffn[1])
+
     def run(self, q, k_pool, v_pool, out: str = "device", host_out: Optional[torch.Tensor] = None):
         self.load(q, k_pool, v_pool)
         self.compute()

@@ -59,7 +59,8 @@ class RkSizes(ctypes.Structure):
 EXPORTS = ("rk_query_sizes", "rk_select_visible", "rk_relocate_rope", "rk_segpaged_prefill",
            "rk_get_device_status", "rk_select_visible_noalloc", "rk_selftest_bounded_wait",
            "rk_score_query_sizes", "rk_score_retrieval_pages", "rk_decode_query_sizes",
-           "rk_segpaged_decode", "rk_importance_query_sizes", "rk_attention_importance")
+           "rk_segpaged_decode", "rk_importance_query_sizes", "rk_attention_importance",
+           "rk_ffn_query_sizes", "rk_sparse_ffn")
 
 _lib = None
 
@@ -91,6 +92,8 @@ def lib() -> ctypes.CDLL:
         L.rk_importance_query_sizes.argtypes = [vp, vp, vp]
         L.rk_attention_importance.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.c_float, i32, vp,
                                               vp, vp, vp, ctypes.c_size_t, vp]
+        L.rk_ffn_query_sizes.argtypes = [vp, i32, vp, i32, vp]
+        L.rk_sparse_ffn.argtypes = [vp, i32, vp, vp, i32, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
         for name in EXPORTS:
             getattr(L, name).restype = i32
         _lib = L
@@ -114,6 +117,15 @@ def _stream(stream) -> ctypes.c_void_p:
 
 class RkDecodeSizes(ctypes.Structure):
     _fields_ = [("max_splits", ctypes.c_int64), ("workspace_bytes", ctypes.c_int64)]
+
+
+class RkFfnDims(ctypes.Structure):
+    _fields_ = [("n_rows", ctypes.c_int32), ("d_model", ctypes.c_int32), ("d_ff", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
+
+
+class RkFfnSizes(ctypes.Structure):
+    _fields_ = [("n_selected", ctypes.c_int64), ("workspace_bytes", ctypes.c_int64)]
 
 
 class RkImportanceSizes(ctypes.Structure):
@@ -336,3 +348,40 @@ def attention_importance(hl: HostLayout, q: torch.Tensor, k_pool: torch.Tensor, 
                                          _ptr(importance), _ptr(tokens), _ptr(token_count),
                                          _ptr(ws), ws.numel(), _stream(stream)),
            "rk_attention_importance")
+
+
+# ------------------------------------------------------ token-selective FFN
+
+def _ffn_args(n_rows: int, d_model: int, d_ff: int, cu_seqlens):
+    cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
+    return RkFfnDims(int(n_rows), int(d_model), int(d_ff), 0), cu
+
+
+def ffn_sizes(n_rows: int, d_model: int, d_ff: int, cu_seqlens, top_k: int) -> RkFfnSizes:
+    dims, cu = _ffn_args(n_rows, d_model, d_ff, cu_seqlens)
+    s = RkFfnSizes()
+    _check(lib().rk_ffn_query_sizes(ctypes.byref(dims), cu.shape[0] - 1, cu.ctypes.data,
+                                    int(top_k), ctypes.byref(s)), "rk_ffn_query_sizes")
+    return s
+
+
+def ffn_workspace(sizes: RkFfnSizes, device) -> torch.Tensor:
+    return torch.empty(max(256, int(sizes.workspace_bytes)), dtype=torch.uint8,
+                       device=torch.device(device))
+
+
+def sparse_ffn(x: torch.Tensor, cu_seqlens, tokens: Optional[torch.Tensor], top_k: int,
+               w_gate: torch.Tensor, w_up: torch.Tensor, w_down: torch.Tensor, ws: torch.Tensor,
+               stream=None):
+    """rk_sparse_ffn: x [n_rows][d_model] bf16 (updated in place at the
+    selected rows); tokens int32 [n_req][top_k] request-local picks (one
+    layer of rk_attention_importance's output); w_gate / w_up [d_ff][d_model],
+    w_down [d_model][d_ff] bf16."""
+    n_rows, d_model = x.shape
+    d_ff = w_gate.shape[0]
+    assert x.dtype == w_gate.dtype == w_up.dtype == w_down.dtype == torch.bfloat16
+    assert w_up.shape == w_gate.shape == (d_ff, d_model) and w_down.shape == (d_model, d_ff)
+    dims, cu = _ffn_args(n_rows, d_model, d_ff, cu_seqlens)
+    _check(lib().rk_sparse_ffn(ctypes.byref(dims), cu.shape[0] - 1, cu.ctypes.data, _ptr(tokens),
+                               int(top_k), _ptr(x), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
+                               _ptr(ws), ws.numel(), _stream(stream)), "rk_sparse_ffn")

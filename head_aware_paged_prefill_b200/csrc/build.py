@@ -18,7 +18,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 PKG = os.path.dirname(HERE)
 ROOT = os.path.dirname(PKG)
 SOURCES = ["rk_api.cu", "rk_select.cu", "rk_relocate.cu", "rk_prefill.cu", "rk_selftest.cu",
-           "rk_score.cu", "rk_decode.cu", "rk_importance.cu"]
+           "rk_score.cu", "rk_decode.cu", "rk_importance.cu", "rk_ffn.cu"]
 HEADERS = ["rk_internal.h", "sm100.cuh", os.path.join("..", "..", "include", "rk.h")]
 LIB = os.path.join(PKG, "librk.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -1025,3 +1025,95 @@ extern "C" rk_status rk_attention_importance(const rk_dims* dims, const rk_layou
   a.error_word = reinterpret_cast<int32_t*>(ws);
   return launch_importance(a, s) == cudaSuccess ? RK_OK : RK_ERR_CUDA;
 }
+
+// ---- token-selective FFN
+
+namespace rk {
+namespace {
+struct FfnPlan {
+  int64_t m = 0;
+  std::vector<int32_t> upload;  // cu [n_req + 1], selection prefix [n_req + 1]
+  size_t off_up = 0, off_rows = 0, off_xs = 0, off_h = 0, total = 0;
+};
+rk_status plan_ffn(const rk_ffn_dims* d, int32_t n_req, const int32_t* cu, int32_t top_k,
+                   FfnPlan* out) {
+  if (!d || !cu || n_req < 1 || top_k < 0 || d->reserved != 0 || d->n_rows < 0)
+    return RK_ERR_INVALID_ARG;
+  if (d->d_model < 256 || d->d_model % 256 != 0 || d->d_ff < 128 || d->d_ff % 128 != 0 ||
+      d->d_model > (1 << 16) || d->d_ff > (1 << 18))
+    return RK_ERR_INVALID_ARG;
+  if (cu[0] != 0 || cu[n_req] != d->n_rows) return RK_ERR_INVALID_ARG;
+  out->upload.assign(2 * static_cast<size_t>(n_req + 1), 0);
+  int64_t m = 0;
+  for (int r = 0; r < n_req; ++r) {
+    if (cu[r + 1] < cu[r]) return RK_ERR_INVALID_ARG;
+    out->upload[r] = cu[r];
+    out->upload[n_req + 1 + r] = static_cast<int32_t>(m);
+    m += std::min<int64_t>(top_k, cu[r + 1] - cu[r]);
+  }
+  out->upload[n_req] = cu[n_req];
+  out->upload[2 * n_req + 1] = static_cast<int32_t>(m);
+  if (m >= kMaxI32 / 2) return RK_ERR_INVALID_ARG;
+  out->m = m;
+  out->off_up = 256;
+  out->off_rows = align_up(out->off_up + 4 * out->upload.size(), 256);
+  out->off_xs = align_up(out->off_rows + 4 * static_cast<size_t>(m), 256);
+  out->off_h = align_up(out->off_xs + 2 * static_cast<size_t>(m) * d->d_model, 256);
+  out->total = align_up(out->off_h + 2 * static_cast<size_t>(m) * d->d_ff, 256);
+  return RK_OK;
+}
+}  // namespace
+}  // namespace rk
+
+extern "C" rk_status rk_ffn_query_sizes(const rk_ffn_dims* dims, int32_t n_req,
+                                        const int32_t* cu_seqlens, int32_t top_k,
+                                        rk_ffn_sizes* out) {
+  if (!out) return RK_ERR_INVALID_ARG;
+  FfnPlan plan;
+  rk_status st = plan_ffn(dims, n_req, cu_seqlens, top_k, &plan);
+  if (st != RK_OK) return st;
+  out->n_selected = plan.m;
+  out->workspace_bytes = static_cast<int64_t>(plan.total);
+  return RK_OK;
+}
+
+extern "C" rk_status rk_sparse_ffn(const rk_ffn_dims* dims, int32_t n_req,
+                                   const int32_t* cu_seqlens, const int32_t* tokens, int32_t top_k,
+                                   void* x, const void* w_gate, const void* w_up,
+                                   const void* w_down, void* workspace, size_t workspace_bytes,
+                                   void* stream) {
+  FfnPlan plan;
+  rk_status st = plan_ffn(dims, n_req, cu_seqlens, top_k, &plan);
+  if (st != RK_OK) return st;
+  if (!x || !w_gate || !w_up || !w_down || !workspace || (plan.m > 0 && !tokens))
+    return RK_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(w_gate, 16) || !aligned(w_up, 16) || !aligned(w_down, 16) ||
+      !aligned(tokens, 4) || !aligned(workspace, 256))
+    return RK_ERR_INVALID_ARG;
+  if (workspace_bytes < plan.total) return RK_ERR_CAPACITY;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (cudaMemsetAsync(ws, 0, 256, s) != cudaSuccess ||
+      cudaMemcpyAsync(ws + plan.off_up, plan.upload.data(), 4 * plan.upload.size(),
+                      cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return RK_ERR_CUDA;
+  FfnLaunchArgs a{};
+  a.x = x;
+  a.w_gate = w_gate;
+  a.w_up = w_up;
+  a.w_down = w_down;
+  a.cu = reinterpret_cast<const int32_t*>(ws + plan.off_up);
+  a.sel_prefix = a.cu + (n_req + 1);
+  a.tokens = tokens;
+  a.xs = ws + plan.off_xs;
+  a.h = ws + plan.off_h;
+  a.rows = reinterpret_cast<int32_t*>(ws + plan.off_rows);
+  a.error_word = reinterpret_cast<int32_t*>(ws);
+  a.timeout_site = reinterpret_cast<int*>(ws + 4);
+  a.m = static_cast<int>(plan.m);
+  a.n_req = n_req;
+  a.top_k = top_k;
+  a.d_model = dims->d_model;
+  a.d_ff = dims->d_ff;
+  return launch_sparse_ffn(a, s) == cudaSuccess ? RK_OK : RK_ERR_CUDA;
+}

@@ -224,3 +224,26 @@ struct ImportanceLaunchArgs {
 cudaError_t launch_importance(const ImportanceLaunchArgs& a, cudaStream_t stream);
 
 }  // namespace rk
+
+namespace rk {
+
+// ---- token-selective FFN
+struct FfnLaunchArgs {
+  void* x;                    // bf16 [n_rows][d_model], updated in place
+  const void* w_gate;         // bf16 [d_ff][d_model]
+  const void* w_up;           // bf16 [d_ff][d_model]
+  const void* w_down;         // bf16 [d_model][d_ff]
+  const int32_t* cu;          // device [n_req + 1]
+  const int32_t* sel_prefix;  // device [n_req + 1]: selection entries before request r
+  const int32_t* tokens;      // device [n_req][top_k], request-local
+  void* xs;                   // workspace bf16 [m][d_model]
+  void* h;                    // workspace bf16 [m][d_ff]
+  int32_t* rows;              // workspace [m]
+  int32_t* error_word;
+  int* timeout_site;
+  int m, n_req, top_k, d_model, d_ff;
+};
+
+cudaError_t launch_sparse_ffn(const FfnLaunchArgs& a, cudaStream_t stream);
+
+}  // namespace rk

@@ -460,3 +460,20 @@ def random_small(rng: np.random.Generator, *, p: Optional[int] = None, d: Option
     return _make_layout(n_layers=n_layers, hq=hkv * g, hkv=hkv, d=d, p=p,
                         theta=float(rng.choice([1e4, 1e6])), requests=requests, class_map=cmap,
                         window=int(rng.integers(1, 4 * p + 1)), retrieval=retrieval)
+
+
+def ffn_inputs(n_rows: int, d_model: int, d_ff: int, seed: int, device="cpu"):
+    """Synthetic hidden state and FFN weights for the token-selective FFN:
+    x ~ N(0, 1) [n_rows][d_model]; W_gate, W_up ~ N(0, 1 / d_model)
+    [d_ff][d_model]; W_down ~ N(0, 1 / d_ff) [d_model][d_ff] (so every
+    product is of unit scale), all drawn in fp32 in that order from
+    torch.Generator(device).manual_seed(seed) and rounded to bf16.  The
+    width of the bench's FFN is Mistral-7B's (d_model 4096, d_ff 14336)."""
+    dev = torch.device(device)
+    g = torch.Generator(device=dev).manual_seed(seed)
+    bf = torch.bfloat16
+    x = torch.randn((n_rows, d_model), generator=g, device=dev).to(bf)
+    wg = (torch.randn((d_ff, d_model), generator=g, device=dev) * d_model ** -0.5).to(bf)
+    wu = (torch.randn((d_ff, d_model), generator=g, device=dev) * d_model ** -0.5).to(bf)
+    wd = (torch.randn((d_model, d_ff), generator=g, device=dev) * d_ff ** -0.5).to(bf)
+    return x, wg, wu, wd

@@ -13,6 +13,9 @@
  *   - rk_segpaged_prefill <- EXECUTE's attention (paooo page, "how to use" and
  *                            "technical principles": a fused varlen kernel over
  *                            per-head pages that never builds an attn_mask).
+ * and, beside the hot path, retrieval page scoring, paged decode, the
+ * attention importance and the token-selective FFN it feeds (each section
+ * below cites its passage).
  *
  * Conventions shared by every call
  *   - All pointers are caller-owned.  The library never allocates or frees
@@ -394,6 +397,61 @@ rk_status rk_attention_importance(const rk_dims* dims, const rk_layout* layout, 
                                   float softmax_scale, int32_t top_k, float* importance,
                                   int32_t* tokens, int32_t* token_count, void* workspace,
                                   size_t workspace_bytes, void* stream);
+
+
+/* ---- token-selective FFN (sparse FFN) ------------------------------------
+ *
+ * RedKnot runs the dense FFN only on the tokens with the highest attention
+ * scores and sends the others along the residual path (README "About",
+ * Elastic Sparsity / Sparse FFN; paooo page, "main functions").  The pages
+ * name the Mistral-7B and Qwen3 families, whose FFN is the gated SiLU MLP;
+ * the reading implemented, for each selected row i of the hidden state x:
+ *   h   = silu(W_gate x_i) * (W_up x_i)      (d_ff values, rounded to bf16)
+ *   x_i = x_i + W_down h                     (fp32 sum, rounded to bf16)
+ * and every other row of x is left as it is.  The selection is
+ * rk_attention_importance's output for one layer: request r contributes its
+ * first min(top_k, L_r) tokens.  bf16 inputs, fp32 accumulation on the
+ * tensor cores. */
+
+typedef struct {
+  int32_t n_rows;   /* rows of x: the batch's total tokens */
+  int32_t d_model;  /* hidden width: a multiple of 256 */
+  int32_t d_ff;     /* FFN width: a multiple of 128 */
+  int32_t reserved; /* must be 0 */
+} rk_ffn_dims;
+
+typedef struct {
+  int64_t n_selected;      /* rows the call updates: sum_r min(top_k, L_r) */
+  int64_t workspace_bytes; /* device workspace for rk_sparse_ffn */
+} rk_ffn_sizes;
+
+/* Validates the shapes and reports the workspace size.  cu_seqlens: host
+ * [n_req + 1] (cu_seqlens[0] = 0, non-decreasing, cu_seqlens[n_req] =
+ * n_rows).  Host only.  Errors: RK_ERR_INVALID_ARG. */
+rk_status rk_ffn_query_sizes(const rk_ffn_dims* dims, int32_t n_req, const int32_t* cu_seqlens,
+                             int32_t top_k, rk_ffn_sizes* out);
+
+/*   x:       device bf16 [n_rows][d_model], updated in place at the selected
+ *            rows.
+ *   tokens:  device int32 [n_req][top_k], request-local positions (the
+ *            `tokens` of rk_attention_importance for one layer); the first
+ *            min(top_k, L_r) of request r are used and must be distinct.  A
+ *            position outside the request is skipped and sets
+ *            RK_DEV_BAD_PAGE.
+ *   w_gate, w_up: device bf16 [d_ff][d_model]; w_down: device bf16
+ *            [d_model][d_ff] (rows are output features, as in a linear
+ *            layer's weight).
+ *   workspace: device, >= rk_ffn_sizes.workspace_bytes, 256-byte aligned;
+ *            its first word is the device error word (RK_DEV_BAD_PAGE,
+ *            RK_DEV_TIMEOUT), reset by this call and read by
+ *            rk_get_device_status.  It holds the gathered rows and the
+ *            bf16 activations h between the two GEMMs.
+ * Asynchronous on `stream`.  Errors (host): RK_ERR_INVALID_ARG,
+ * RK_ERR_CAPACITY, RK_ERR_CUDA. */
+rk_status rk_sparse_ffn(const rk_ffn_dims* dims, int32_t n_req, const int32_t* cu_seqlens,
+                        const int32_t* tokens, int32_t top_k, void* x, const void* w_gate,
+                        const void* w_up, const void* w_down, void* workspace,
+                        size_t workspace_bytes, void* stream);
 
 #ifdef __cplusplus
 }

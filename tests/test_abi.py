@@ -317,3 +317,34 @@ def test_importance_workspace_exact(lib, name):
     max_pages = max(-(-lay.req_len(r) // lay.p) for r in range(lay.n_req))
     index = 8 * lay.n_tables * (max_pages * lay.p // KB + 1 + max_pages // 8 + 1) + 4 * lay.n_tables * max_pages
     assert 1024 * s.n_items <= s.workspace_bytes <= 1040 * s.n_items + index + 4096 + 8 * lay.n_tables
+
+
+def test_ffn_calls_validate_on_host(lib):
+    """Token-selective FFN: sizes follow the selection, and bad shapes or
+    pointers are refused before any GPU work."""
+    E, C = binding.RK_ERR_INVALID_ARG, binding.RK_ERR_CAPACITY
+    s = binding.ffn_sizes(700, 256, 384, [0, 300, 700], 200)
+    assert s.n_selected == 400
+    assert s.workspace_bytes >= 2 * 400 * (256 + 384) and s.workspace_bytes % 256 == 0
+    assert binding.ffn_sizes(700, 256, 384, [0, 300, 700], 1000).n_selected == 700
+    for bad in ((700, 200, 384), (700, 256, 100), (699, 256, 384)):
+        with pytest.raises(binding.RkError):
+            binding.ffn_sizes(*bad, [0, 300, 700], 8)
+    fake = ctypes.c_void_p(1 << 20)
+    dims = binding.RkFfnDims(700, 256, 384, 0)
+    cu = np.asarray([0, 300, 700], dtype=np.int32)
+    args = [ctypes.byref(dims), 2, cu.ctypes.data, fake, 200, fake, fake, fake, fake, fake,
+            s.workspace_bytes, None]
+
+    def call(**kw):
+        a = list(args)
+        for i, v in kw.items():
+            a[int(i[1:])] = v
+        return lib.rk_sparse_ffn(*a)
+
+    assert call(a3=None) == E                           # tokens
+    assert call(a5=None) == E                           # x
+    assert call(a5=ctypes.c_void_p((1 << 20) + 2)) == E  # unaligned x
+    assert call(a9=ctypes.c_void_p((1 << 20) + 16)) == E  # unaligned workspace
+    assert call(a4=-1) == E                             # top_k
+    assert call(a10=s.workspace_bytes - 1) == C
