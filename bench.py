@@ -58,7 +58,8 @@ def _peaks():
 KERNEL_SOURCES = {"segpaged_prefill_kernel": ("rk_prefill.cu", "sm100.cuh", "rk_internal.h"),
                   "relocate_kernel": ("rk_relocate.cu", "sm100.cuh", "rk_internal.h"),
                   "decode_split_kernel": ("rk_decode.cu", "rk_internal.h"),
-                  "importance_colsum_kernel": ("rk_importance.cu", "rk_internal.h")}
+                  "importance_colsum_kernel": ("rk_importance.cu", "rk_internal.h"),
+                  "ffn_gemm_kernel": ("rk_ffn.cu", "sm100.cuh", "rk_internal.h")}
 
 
 def _kernel_hash(kernel: str = "segpaged_prefill_kernel") -> str:
@@ -529,6 +530,53 @@ def _bench_importance(torch, lay, lay_name, q, k, v, dev, flush, stream, reps, p
             "device_status": st}
 
 
+def _bench_ffn(torch, lay, dev, flush, stream, reps, peaks, peak_kind, d_model=4096, d_ff=14336):
+    """rk_sparse_ffn on the layer's rows at Mistral-7B's FFN width with the
+    top quarter of each request's tokens selected (seeded synthetic hidden
+    state and weights): three GEMM-sized products (gate, up, down) on the
+    selected rows only, bound by the tensor cores."""
+    from head_aware_paged_prefill_b200 import binding, synth
+    T = lay.total_tokens
+    top_k = max(lay.req_len(r) for r in range(lay.n_req)) // 4
+    x, wg, wu, wd = synth.ffn_inputs(T, d_model, d_ff, seed=21, device=dev)
+    rng = np.random.default_rng(22)
+    tok = np.zeros((lay.n_req, top_k), dtype=np.int32)
+    for r in range(lay.n_req):
+        L = lay.req_len(r)
+        k = min(top_k, L)
+        tok[r, :k] = np.sort(rng.choice(L, size=k, replace=False))
+    tok = torch.from_numpy(tok).to(dev)
+    sizes = binding.ffn_sizes(T, d_model, d_ff, lay.cu_seqlens, top_k)
+    ws = binding.ffn_workspace(sizes, dev)
+    for _ in range(3):
+        binding.sparse_ffn(x, lay.cu_seqlens, tok, top_k, wg, wu, wd, ws)
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(reps):
+        flush()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        binding.sparse_ffn(x, lay.cu_seqlens, tok, top_k, wg, wu, wd, ws)
+        b.record(stream)
+        ms.append((a, b))
+    torch.cuda.synchronize()
+    t = statistics.mean(x_.elapsed_time(y_) for x_, y_ in ms)
+    m = int(sizes.n_selected)
+    flops = 2 * m * d_model * d_ff * 3
+    achieved = flops / (t * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    st = binding.device_status(ws)
+    del x, wg, wu, wd, ws
+    torch.cuda.empty_cache()
+    return {"bound": "tensor", "kernel": "ffn_gather + ffn_gemm (gate/up, SwiGLU) + ffn_gemm (down, residual)",
+            "workload": f"the layer's {T} rows, top {top_k} per request selected, d_model {d_model}, "
+                        f"d_ff {d_ff} (Mistral-7B's FFN), seeded synthetic x and weights",
+            "selected_rows": m, "flops": flops, "achieved": achieved, "peak": peak,
+            "unit": UNIT, "frac": achieved / peak, "peak_kind": f"bf16 burst, {peak_kind}",
+            "us": t * 1e3, "launches": 3, "device_status": st,
+            "traffic": _recorded_traffic("ffn_gemm_kernel", f"ffn_{m}x{d_model}x{d_ff}")}
+
+
 def _cpu_baseline(lay, q, kc, vc, seconds: float, total_pairs: int):
     """The fp64 oracle timed on seeded row samples of the workload (batches of
     growing size until about `seconds` of oracle time), with the full-run
@@ -601,6 +649,39 @@ def _bench_config(torch, name, dev, flush, stream, steps, warmup, peaks, peak_ki
     return out
 
 
+def _bench_e2e(torch, pre, q, k, v, stream, E, world, dist, dev, flops):
+    """The same metric end to end through SegPagedPrefill with host buffers:
+    pinned q / K / V in and o out every step, E steps pipelined."""
+    q_h = q.cpu().pin_memory()
+    k_h = k.cpu().pin_memory()
+    v_h = v.cpu().pin_memory()
+    o_h = torch.empty(pre.o.shape, dtype=pre.o.dtype, pin_memory=True)
+    pre.run_host_pipelined([(q_h, k_h, v_h)] * 2, [o_h] * 2)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    pre.run_host_pipelined([(q_h, k_h, v_h)] * E, [o_h] * E)
+    b.record(stream)
+    b.synchronize()
+    e2e_ms = a.elapsed_time(b)
+    # the same steps one after another (copy in, compute, copy out), for context
+    a2, b2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a2.record(stream)
+    for _ in range(min(E, 5)):
+        pre.run(q_h, k_h, v_h, out="host", host_out=o_h)
+    b2.record(stream)
+    b2.synchronize()
+    serial_ms_per_step = a2.elapsed_time(b2) / min(E, 5)
+    e2e_ms = max_over_ranks(e2e_ms, dist if world > 1 else None, dev)
+    e2e_value = weak_scaling_value(world, flops, E, e2e_ms) / 1e12
+    h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h))
+    d2h = o_h.numel() * o_h.element_size()
+    del q_h, k_h, v_h, o_h
+    return {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / E, "pipelined": True,
+            "serial_ms_per_step": serial_ms_per_step}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -617,6 +698,8 @@ def main():
     ap.add_argument("--no-mask-penalty", action="store_true")
     ap.add_argument("--decode-batch", type=int, default=32)
     ap.add_argument("--no-importance", action="store_true")
+    ap.add_argument("--no-ffn", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--per-config", default="cfg1,cfg3,cfg4,cfg5",
                     help="other workloads timed after the headline one ('' for none)")
     ap.add_argument("--pc-steps", type=int, default=20)
@@ -694,32 +777,8 @@ def main():
     # host, E steps pipelined (step n + 1's inputs and step n - 1's o cross
     # the host link while step n computes); every step moves its full inputs
     # and output, each larger than L2
-    q_h = q.cpu().pin_memory()
-    k_h = k.cpu().pin_memory()
-    v_h = v.cpu().pin_memory()
-    o_h = torch.empty(pre.o.shape, dtype=pre.o.dtype, pin_memory=True)
-    pre.run_host_pipelined([(q_h, k_h, v_h)] * 2, [o_h] * 2)
-    torch.cuda.synchronize()
-    E = args.e2e_steps
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    pre.run_host_pipelined([(q_h, k_h, v_h)] * E, [o_h] * E)
-    b.record(stream)
-    b.synchronize()
-    e2e_ms = a.elapsed_time(b)
-    # the same steps one after another (copy in, compute, copy out), for context
-    a2, b2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a2.record(stream)
-    for _ in range(min(E, 5)):
-        pre.run(q_h, k_h, v_h, out="host", host_out=o_h)
-    b2.record(stream)
-    b2.synchronize()
-    serial_ms_per_step = a2.elapsed_time(b2) / min(E, 5)
-    e2e_ms = max_over_ranks(e2e_ms, dist if world > 1 else None, dev)
-    e2e_value = weak_scaling_value(world, flops, E, e2e_ms) / 1e12
-    h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h))
-    d2h = o_h.numel() * o_h.element_size()
-
+    e2e = _bench_e2e(torch, pre, q, k, v, stream, args.e2e_steps, world, dist, dev, flops) \
+        if not args.no_e2e else None
     peaks, peak_kind = _peaks()
     k3_mean = statistics.mean(k3_ms)
     achieved = flops / (k3_mean * 1e-3) / 1e12
@@ -735,6 +794,8 @@ def main():
     importance = (_bench_importance(torch, lay, wl.name, q, k, v, dev, flush, stream,
                                     args.reloc_reps, peaks, peak_kind)
                   if args.mode == "relocate" and not args.no_importance else None)
+    ffn = (_bench_ffn(torch, lay, dev, flush, stream, args.reloc_reps, peaks, peak_kind)
+           if args.mode == "relocate" and not args.no_ffn else None)
     mask_penalty = (_mask_penalty(torch, pre, lay, q, k3_mean)
                     if args.mode == "relocate" and not args.no_mask_penalty else None)
 
@@ -797,9 +858,7 @@ def main():
                      "peak_kind": f"bf16 burst, {peak_kind}", "traffic": traffic,
                      "k3_ms": k3_mean},
         "cpu_baseline": cpu_baseline,
-        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / E, "pipelined": True,
-                "serial_ms_per_step": serial_ms_per_step},
+        "e2e": e2e,
         "gpu_launches": launches,
         "clocks": clocks,
         "mode": args.mode,
@@ -809,6 +868,7 @@ def main():
         "mask_penalty": mask_penalty,
         "decode_roofline": decode,
         "importance_roofline": importance,
+        "sparse_ffn_roofline": ffn,
         "per_config": per_config,
     }
     print(json.dumps(line), flush=True)

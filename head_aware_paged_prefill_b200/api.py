@@ -11,8 +11,8 @@ C-ABI calls on the current CUDA stream.  Two modes:
               K pool (same page id; pages reused at two offsets get an
               appended copy, V copied alongside), then rk_select_visible and
               rk_segpaged_prefill(fuse_rope=0) read the working pools.  The
-              jobs come from the page tables, built once on the device when
-              the object is created.
+              jobs and the relocated layout come from rk_relocation_plan
+              (host only), once, when the object is created.
 
 Inputs may live on the host (pinned tensors are copied asynchronously) or on
 the device; ``run(..., out="host")`` returns o on the host.
@@ -28,7 +28,6 @@ import numpy as np
 import torch
 
 from . import binding, synth
-from .plan import RelocationPlan, relocation_plan
 
 
 def score_retrieval(layout, q: torch.Tensor, k_store: torch.Tensor, top_k: int = 16,
@@ -54,16 +53,15 @@ class SegPagedPrefill:
         self.mode = mode
         self.device = torch.device(device)
         lay = layout
-        entries, ranges = self._tables(layout)
         # attention work items: 128-row tiles of each table's row ranges x
-        # pairs of q heads (the library's own rule)
+        # pairs of q heads (the library's own rule), for the launch count
         npairs = (layout.hq // layout.hkv + 1) // 2
-        self.n_items = npairs * sum(-(-(int(b) - int(a)) // 128) for rr in ranges for a, b in rr)
+        self.n_items = npairs * sum(-(-(b - a) // 128) for a, b in self._row_ranges(layout))
         if mode == "relocate":
-            self.plan = relocation_plan(layout, entries)
+            self.plan = binding.relocation_plan(layout)
         else:
             empty = np.zeros((0, 3), np.int32)
-            self.plan = RelocationPlan(empty, empty, layout, 0)
+            self.plan = binding.RelocationPlan(empty, empty, layout, 0)
         self.rel_layout = self.plan.layout
         self.hl = binding.HostLayout(self.rel_layout)
         self.sizes = self.hl.sizes()
@@ -97,20 +95,26 @@ class SegPagedPrefill:
                         if self.mode == "relocate" else None),
         }
 
-    def _tables(self, layout):
-        """Page tables and row ranges of the original layout, built once by
-        the library on the device and read back (relocation jobs, item
-        count)."""
-        hl = binding.HostLayout(layout)
-        sizes = hl.sizes()
-        vis = binding.Visible(sizes, self.device)
-        ws = binding.workspace(sizes, self.device)
-        binding.select_visible(hl, vis, ws)
-        torch.cuda.current_stream(self.device).synchronize()
-        st = binding.device_status(ws)
-        if st:
-            raise binding.RkError(binding.RK_ERR_DEVICE, f"rk_select_visible (device {st:#x})")
-        return vis.tables()
+    @staticmethod
+    def _row_ranges(lay):
+        """Every table's row ranges by the class rule: the whole request for
+        global and dense heads, the merged uncached segments otherwise."""
+        out = []
+        for r in range(lay.n_req):
+            L = lay.req_len(r)
+            unc = []
+            for seg in lay.segments_of(r):
+                if not seg[4]:
+                    a, b = int(seg[1]), int(seg[1] + seg[2])
+                    if unc and unc[-1][1] == a:
+                        unc[-1] = (unc[-1][0], b)
+                    else:
+                        unc.append((a, b))
+            for lh in range(lay.n_layers * lay.hkv):
+                c = int(lay.class_map[lh])
+                out.extend([(0, L)] if c in (synth.GLOBAL, synth.DENSE) and L > 0 else
+                           ([] if c in (synth.GLOBAL, synth.DENSE) else unc))
+        return out
 
     # Number of library kernel launches one run() makes.
     @property

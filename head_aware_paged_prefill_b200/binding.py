@@ -6,7 +6,9 @@ library is missing, every call raises; there is no fallback.
 """
 from __future__ import annotations
 
+import copy
 import ctypes
+import dataclasses
 import os
 from typing import Optional
 
@@ -60,7 +62,8 @@ EXPORTS = ("rk_query_sizes", "rk_select_visible", "rk_relocate_rope", "rk_segpag
            "rk_get_device_status", "rk_select_visible_noalloc", "rk_selftest_bounded_wait",
            "rk_score_query_sizes", "rk_score_retrieval_pages", "rk_decode_query_sizes",
            "rk_segpaged_decode", "rk_importance_query_sizes", "rk_attention_importance",
-           "rk_ffn_query_sizes", "rk_sparse_ffn")
+           "rk_ffn_query_sizes", "rk_sparse_ffn", "rk_relocation_query_sizes",
+           "rk_relocation_plan")
 
 _lib = None
 
@@ -93,6 +96,8 @@ def lib() -> ctypes.CDLL:
         L.rk_attention_importance.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.c_float, i32, vp,
                                               vp, vp, vp, ctypes.c_size_t, vp]
         L.rk_ffn_query_sizes.argtypes = [vp, i32, vp, i32, vp]
+        L.rk_relocation_query_sizes.argtypes = [vp, vp, vp]
+        L.rk_relocation_plan.argtypes = [vp, vp, vp, i64, vp, i64, vp, vp]
         L.rk_sparse_ffn.argtypes = [vp, i32, vp, vp, i32, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
         for name in EXPORTS:
             getattr(L, name).restype = i32
@@ -117,6 +122,11 @@ def _stream(stream) -> ctypes.c_void_p:
 
 class RkDecodeSizes(ctypes.Structure):
     _fields_ = [("max_splits", ctypes.c_int64), ("workspace_bytes", ctypes.c_int64)]
+
+
+class RkRelocationSizes(ctypes.Structure):
+    _fields_ = [("n_jobs_k", ctypes.c_int64), ("n_jobs_v", ctypes.c_int64),
+                ("n_extra_pages", ctypes.c_int64)]
 
 
 class RkFfnDims(ctypes.Structure):
@@ -385,3 +395,36 @@ def sparse_ffn(x: torch.Tensor, cu_seqlens, tokens: Optional[torch.Tensor], top_
     _check(lib().rk_sparse_ffn(ctypes.byref(dims), cu.shape[0] - 1, cu.ctypes.data, _ptr(tokens),
                                int(top_k), _ptr(x), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
                                _ptr(ws), ws.numel(), _stream(stream)), "rk_sparse_ffn")
+
+
+# ------------------------------------------------------ relocation plan
+
+@dataclasses.dataclass
+class RelocationPlan:
+    jobs_k: np.ndarray   # int32 [n, 3] (src_page in the K store, dst_page in the working K pool, delta)
+    jobs_v: np.ndarray   # int32 [m, 3] (src_page, dst_page >= n_pages, 0) within the working V pool
+    layout: object       # the relocated layout: every segment at delta 0, appended runs in page_base
+    n_extra: int         # pages appended to both working pools
+
+
+def relocation_plan(lay) -> RelocationPlan:
+    """rk_relocation_plan (host only): the relocate-mode step's job lists and
+    relocated layout for a layout (an object with synth.Layout's fields)."""
+    hl = HostLayout(lay)
+    sz = RkRelocationSizes()
+    _check(lib().rk_relocation_query_sizes(ctypes.byref(hl.dims), ctypes.byref(hl.layout),
+                                           ctypes.byref(sz)), "rk_relocation_query_sizes")
+    nk, nv = int(sz.n_jobs_k), int(sz.n_jobs_v)
+    jk = np.zeros((max(nk, 1), 3), dtype=np.int32)
+    jv = np.zeros((max(nv, 1), 3), dtype=np.int32)
+    n_seg = int(np.asarray(lay.segments).reshape(-1, 5).shape[0])
+    segs = np.zeros((max(n_seg, 1), 5), dtype=np.int32)
+    pb = np.zeros((max(n_seg, 1), lay.n_layers * lay.hkv), dtype=np.int32)
+    _check(lib().rk_relocation_plan(ctypes.byref(hl.dims), ctypes.byref(hl.layout), jk.ctypes.data,
+                                    nk, jv.ctypes.data, nv, segs.ctypes.data, pb.ctypes.data),
+           "rk_relocation_plan")
+    out = copy.copy(lay)
+    out.segments = segs[:n_seg].copy()
+    out.page_base = pb[:n_seg].copy()
+    out.n_pages = int(lay.n_pages) + int(sz.n_extra_pages)
+    return RelocationPlan(jk[:nk].copy(), jv[:nv].copy(), out, int(sz.n_extra_pages))

@@ -1117,3 +1117,130 @@ extern "C" rk_status rk_sparse_ffn(const rk_ffn_dims* dims, int32_t n_req,
   a.d_ff = dims->d_ff;
   return launch_sparse_ffn(a, s) == cudaSuccess ? RK_OK : RK_ERR_CUDA;
 }
+
+// ---- relocation plan (the relocate-mode step's job lists)
+
+namespace rk {
+namespace {
+struct RelocPlan {
+  std::vector<int32_t> jobs_k, jobs_v;  // [n][3] (src_page, dst_page, delta)
+  std::vector<int32_t> page_base;       // [n_segments][n_lh]
+  int64_t n_extra = 0;
+};
+
+// Pages attention reads are the page-table entries, which follow from the
+// layout by the class rule (importance_table_pages).  Every visible page of
+// a cached instance with delta != 0 is rotated into the working pool at its
+// own id; a physical page visible through two instances at different
+// deltas keeps its id for the first and gets a fresh run of pages appended
+// to both pools for the later one (K rotated, V copied).
+rk_status plan_relocation(const rk_dims* d, const rk_layout* lay, const Derived& dv,
+                          RelocPlan* out) {
+  const int P = d->page_size, hkv = d->num_kv_heads;
+  const int64_t n_lh = dv.n_lh;
+  const int n_seg = lay->n_segments;
+  // need[s * n_lh + lh]: page offsets within segment s that a table lists
+  std::vector<std::vector<int>> need(static_cast<size_t>(n_seg) * n_lh);
+  std::vector<int> pages;
+  for (int r = 0; r < d->n_req; ++r) {
+    const int s0 = dv.seg_indptr[r], s1 = dv.seg_indptr[r + 1];
+    if (s0 == s1) continue;
+    for (int layer = 0; layer < d->n_layers; ++layer)
+      for (int kvh = 0; kvh < hkv; ++kvh) {
+        const int lh = layer * hkv + kvh;
+        const int64_t t = (static_cast<int64_t>(r) * d->n_layers + layer) * hkv + kvh;
+        importance_table_pages(d, lay, dv, r, lh, t, &pages);
+        int s = s0;
+        for (int pos : pages) {
+          while (s + 1 < s1 && lay->segments[s + 1].logical_start <= pos) ++s;
+          need[static_cast<size_t>(s) * n_lh + lh].push_back((pos - lay->segments[s].logical_start) / P);
+        }
+      }
+  }
+  out->page_base.assign(lay->page_base, lay->page_base + static_cast<size_t>(n_seg) * n_lh);
+  std::vector<int64_t> claim(static_cast<size_t>(d->n_pages), INT64_MIN);  // delta held per page
+  int64_t nxt = d->n_pages;
+  for (int s = 0; s < n_seg; ++s) {
+    const rk_segment& g = lay->segments[s];
+    const int delta = g.cached ? g.logical_start - g.stored_pos_base : 0;
+    const int npg = (g.len + P - 1) / P;
+    for (int64_t lh = 0; lh < n_lh; ++lh) {
+      std::vector<int>& ks = need[static_cast<size_t>(s) * n_lh + lh];
+      if (ks.empty()) continue;
+      std::sort(ks.begin(), ks.end());
+      ks.erase(std::unique(ks.begin(), ks.end()), ks.end());
+      const int64_t base = lay->page_base[static_cast<size_t>(s) * n_lh + lh];
+      bool clash = false;
+      for (int k : ks) {
+        const int64_t c = claim[static_cast<size_t>(base + k)];
+        clash |= c != INT64_MIN && c != delta;
+      }
+      if (clash) {
+        if (nxt + npg >= kMaxI32 / P) return RK_ERR_CAPACITY;
+        out->page_base[static_cast<size_t>(s) * n_lh + lh] = static_cast<int32_t>(nxt);
+        for (int k : ks) {
+          out->jobs_k.insert(out->jobs_k.end(), {static_cast<int32_t>(base + k),
+                                                 static_cast<int32_t>(nxt + k), delta});
+          out->jobs_v.insert(out->jobs_v.end(), {static_cast<int32_t>(base + k),
+                                                 static_cast<int32_t>(nxt + k), 0});
+        }
+        nxt += npg;
+        continue;
+      }
+      for (int k : ks) {
+        int64_t& c = claim[static_cast<size_t>(base + k)];
+        if (c != INT64_MIN) continue;
+        c = delta;
+        if (delta != 0)
+          out->jobs_k.insert(out->jobs_k.end(), {static_cast<int32_t>(base + k),
+                                                 static_cast<int32_t>(base + k), delta});
+      }
+    }
+  }
+  out->n_extra = nxt - d->n_pages;
+  return RK_OK;
+}
+}  // namespace
+}  // namespace rk
+
+extern "C" rk_status rk_relocation_query_sizes(const rk_dims* dims, const rk_layout* layout,
+                                               rk_relocation_sizes* out) {
+  if (!out) return RK_ERR_INVALID_ARG;
+  rk_status st = check_dims(dims);
+  if (st != RK_OK) return st;
+  Derived dv;
+  if ((st = check_layout(dims, layout, &dv)) != RK_OK) return st;
+  RelocPlan plan;
+  if ((st = plan_relocation(dims, layout, dv, &plan)) != RK_OK) return st;
+  out->n_jobs_k = static_cast<int64_t>(plan.jobs_k.size() / 3);
+  out->n_jobs_v = static_cast<int64_t>(plan.jobs_v.size() / 3);
+  out->n_extra_pages = plan.n_extra;
+  return RK_OK;
+}
+
+extern "C" rk_status rk_relocation_plan(const rk_dims* dims, const rk_layout* layout,
+                                        int32_t* jobs_k, int64_t cap_k, int32_t* jobs_v,
+                                        int64_t cap_v, rk_segment* segments_out,
+                                        int32_t* page_base_out) {
+  rk_status st = check_dims(dims);
+  if (st != RK_OK) return st;
+  Derived dv;
+  if ((st = check_layout(dims, layout, &dv)) != RK_OK) return st;
+  if ((layout->n_segments > 0 && (!segments_out || !page_base_out)) || cap_k < 0 || cap_v < 0)
+    return RK_ERR_INVALID_ARG;
+  RelocPlan plan;
+  if ((st = plan_relocation(dims, layout, dv, &plan)) != RK_OK) return st;
+  const int64_t nk = static_cast<int64_t>(plan.jobs_k.size() / 3);
+  const int64_t nv = static_cast<int64_t>(plan.jobs_v.size() / 3);
+  if (nk > cap_k || nv > cap_v) return RK_ERR_CAPACITY;
+  if ((nk > 0 && !jobs_k) || (nv > 0 && !jobs_v)) return RK_ERR_INVALID_ARG;
+  if (nk > 0) std::memcpy(jobs_k, plan.jobs_k.data(), 4 * plan.jobs_k.size());
+  if (nv > 0) std::memcpy(jobs_v, plan.jobs_v.data(), 4 * plan.jobs_v.size());
+  for (int s = 0; s < layout->n_segments; ++s) {
+    segments_out[s] = layout->segments[s];
+    segments_out[s].stored_pos_base = layout->segments[s].logical_start;
+  }
+  if (layout->n_segments > 0)
+    std::memcpy(page_base_out, plan.page_base.data(), 4 * plan.page_base.size());
+  return RK_OK;
+}

@@ -203,6 +203,49 @@ rk_status rk_segpaged_prefill(const rk_dims* dims, const void* q, const void* k_
                               double rope_theta, float softmax_scale, void* o, float* lse,
                               void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---- relocation plan (host only) ------------------------------------------
+ *
+ * The relocate-mode step: rk_relocate_rope rotates, from the K store into a
+ * working K pool with the same page ids, every page that a page table lists
+ * and that belongs to a cached segment instance with a non-zero delta; then
+ * rk_select_visible and rk_segpaged_prefill(fuse_rope = 0) run on a layout
+ * whose segments all sit at delta 0 (README excerpt, "Offline KV Reuse +
+ * RoPE Relocation"; paooo page, "how to use": BUILDSTATE relocates reused
+ * KV, SELECTVISIBLESTATE chooses it).  Attention reads no other page, so no
+ * other page needs rotating.  A physical page visible through two instances
+ * at different offsets keeps its id for the first instance (in segment
+ * order) and gets a fresh run of pages for the later one: the run is
+ * appended after the pool (ids n_pages, n_pages + 1, ...) in both the K and
+ * the V working pool, filled by K jobs (rotated) and V jobs (delta 0: a
+ * copy).  The page tables follow from the layout by the class rule, so the
+ * plan is computed on the host from the layout alone. */
+
+typedef struct {
+  int64_t n_jobs_k;      /* rk_relocate_rope jobs from the K store into the working K pool */
+  int64_t n_jobs_v;      /* jobs within the working V pool (copies into appended pages) */
+  int64_t n_extra_pages; /* pages appended to both working pools */
+} rk_relocation_sizes;
+
+/* Host only.  Errors: RK_ERR_INVALID_ARG, RK_ERR_UNALIGNED, RK_ERR_CAPACITY. */
+rk_status rk_relocation_query_sizes(const rk_dims* dims, const rk_layout* layout,
+                                    rk_relocation_sizes* out);
+
+/* Host only: writes the plan into host buffers.
+ *   jobs_k: int32 [cap_k][3] (src_page in the K store, dst_page in the
+ *           working K pool, delta); jobs_v: int32 [cap_v][3] (src_page,
+ *           dst_page >= n_pages, 0) within the working V pool, whose first
+ *           n_pages pages are the caller's V pool.
+ *   segments_out [n_segments], page_base_out [n_segments][n_layers * Hkv]:
+ *           the relocated layout (every segment at delta 0, appended runs in
+ *           page_base); with n_pages + n_extra_pages pages, the same
+ *           cu_seqlens, class map, windows and retrieval lists it describes
+ *           what the working pools hold.
+ * Errors: RK_ERR_INVALID_ARG, RK_ERR_UNALIGNED, RK_ERR_CAPACITY (cap_k or
+ * cap_v below rk_relocation_query_sizes). */
+rk_status rk_relocation_plan(const rk_dims* dims, const rk_layout* layout, int32_t* jobs_k,
+                             int64_t cap_k, int32_t* jobs_v, int64_t cap_v,
+                             rk_segment* segments_out, int32_t* page_base_out);
+
 /* Waits for the stream, then copies the device error word of the workspace
  * into *status (host).  Returns RK_OK when the word is 0, RK_ERR_DEVICE
  * otherwise, RK_ERR_CUDA if the copy failed. */

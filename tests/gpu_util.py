@@ -7,7 +7,6 @@ import torch
 
 import oracle
 from head_aware_paged_prefill_b200 import binding
-from head_aware_paged_prefill_b200.plan import relocation_plan
 
 # tolerances for bf16-in / fp32-accumulate outputs (max abs, mean relative)
 MAX_ABS = 2e-2
@@ -61,11 +60,10 @@ def run_select(lay, device="cuda"):
 class PrefillRun:
     """One pass of the CUDA path through the C ABI.
 
-    mode "relocate": rk_select_visible on the original layout gives the
-    page tables the relocation plan is built from; rk_relocate_rope rotates
-    the visible cached K pages from the input pool (the store) into a working
-    copy, then rk_select_visible and rk_segpaged_prefill(fuse_rope=0) run on
-    the relocated layout.  mode "fused": rk_select_visible and
+    mode "relocate": rk_relocation_plan gives the jobs and the relocated
+    layout; rk_relocate_rope rotates the visible cached K pages from the
+    input pool (the store) into a working copy, then rk_select_visible and
+    rk_segpaged_prefill(fuse_rope=0) run on the relocated layout.  mode "fused": rk_select_visible and
     rk_segpaged_prefill(fuse_rope=1) on the original layout.
     ``o`` starts filled with the sentinel so untouched rows can be checked."""
 
@@ -76,10 +74,8 @@ class PrefillRun:
             rel, self.plan = lay, None
             self.k_rel, self.v_rel = k_pool, v_pool
         else:
-            # page tables of the original layout -> relocation jobs
-            _, vis0, _ = run_select(lay, dev)
-            torch.cuda.synchronize()
-            self.plan = relocation_plan(lay, vis0.tables()[0])
+            # relocation jobs and the relocated layout (rk_relocation_plan)
+            self.plan = binding.relocation_plan(lay)
             rel = self.plan.layout
             extra = self.plan.n_extra
             pad = torch.zeros((extra,) + tuple(k_pool.shape[1:]), dtype=k_pool.dtype, device=dev)

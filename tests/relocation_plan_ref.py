@@ -1,4 +1,7 @@
-"""Host-side planning for the relocation pass (BUILDSTATE's relocation part in
+"""Python restatement of the relocation plan, kept as a CPU cross-check of
+the library's rk_relocation_plan (tests only).
+
+Host-side planning for the relocation pass (BUILDSTATE's relocation part in
 the RedKnot pages: cached segment KV is re-rotated to the offset it is reused
 at, "Offline KV Reuse + RoPE Relocation" in the README excerpt).
 

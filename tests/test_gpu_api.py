@@ -76,3 +76,45 @@ def test_pipelined_one_step_and_reuse():
         assert torch.equal(got.view(torch.int16), w.view(torch.int16))
     with pytest.raises(ValueError):
         pre.run_host_pipelined(steps, o2[:1])
+
+
+def test_c_abi_relocate_step_cfg3():
+    """The step the bench times in relocate mode, written with the C ABI's
+    calls only (through the ctypes binding): rk_relocation_plan ->
+    rk_relocate_rope (K store -> working K pool; V copies into the pages
+    appended for the duplicated segment) -> rk_select_visible ->
+    rk_segpaged_prefill(fuse_rope = 0).  On cfg3 (a segment placed twice,
+    sharing pages) its output matches the oracle on sampled rows, and
+    SegPagedPrefill gives the same bytes."""
+    import oracle
+    from head_aware_paged_prefill_b200 import binding
+    from gpu_util import assert_close, oracle_rows, sample_rows
+    wl = synth.cfg3()
+    lay = wl.layout
+    q, k, v = wl.materialize("cuda")
+    plan = binding.relocation_plan(lay)
+    assert plan.n_extra > 0 and plan.jobs_v.shape[0] > 0
+    n, extra = lay.n_pages, plan.n_extra
+    pad = torch.zeros((extra, lay.p, lay.d), dtype=torch.bfloat16, device="cuda")
+    k_work, v_work = torch.cat([k, pad]), torch.cat([v, pad])
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    binding.relocate_rope(k, k_work, torch.from_numpy(plan.jobs_k).cuda(), lay.theta, err)
+    binding.relocate_rope(v_work, v_work, torch.from_numpy(plan.jobs_v).cuda(), lay.theta, err)
+    hl = binding.HostLayout(plan.layout)
+    s = hl.sizes()
+    vis, ws = binding.Visible(s, "cuda"), binding.workspace(s, "cuda")
+    binding.select_visible(hl, vis, ws)
+    o = torch.full_like(q, float("nan"))
+    binding.segpaged_prefill(hl, q, k_work, v_work, vis, ws, o, None, fuse_rope=False)
+    torch.cuda.synchronize()
+    assert binding.device_status(ws) == 0 and int(err.item()) == 0
+    rows = sample_rows(lay, per_table=12, seed=31)
+    want, _, _ = oracle_rows(lay, q.cpu(), k.cpu(), v.cpu(), rows)
+    idx = [torch.from_numpy(rows[:, c]).long().cuda() for c in (0, 2, 1)]
+    assert_close(o[idx[0], idx[1], idx[2]].double().cpu().numpy(), want, "cfg3 C-ABI step")
+    pre = SegPagedPrefill(lay, "cuda")
+    pre.load(q, k, v)
+    pre.compute()
+    torch.cuda.synchronize()
+    got = pre.o[idx[0], idx[1], idx[2]]
+    assert torch.equal(got.view(torch.int16), o[idx[0], idx[1], idx[2]].view(torch.int16))

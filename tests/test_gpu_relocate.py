@@ -7,7 +7,6 @@ import torch
 
 import oracle
 from head_aware_paged_prefill_b200 import binding, synth
-from head_aware_paged_prefill_b200.plan import relocation_plan
 from gpu_util import assert_bf16_rounded, assert_close, run_select, u16
 
 pytestmark = pytest.mark.gpu
@@ -98,15 +97,13 @@ def test_relocate_many_jobs_delta_runs(d):
 
 @pytest.mark.parametrize("name", ["cfg2", "cfg3"])
 def test_relocate_full_plan_sampled(name):
-    """The plan of the full-size layout (from the library's page tables): the
+    """The plan of the full-size layout (rk_relocation_plan): the
     rotated pages match the oracle, and every page no K job writes still holds
     the store's bits."""
     wl = synth.CONFIGS[name]()
     lay = wl.layout
     _, k_pool, _ = wl.materialize("cuda")
-    _, vis, _ = run_select(lay)
-    torch.cuda.synchronize()
-    plan = relocation_plan(lay, vis.tables()[0])
+    plan = binding.relocation_plan(lay)
     jobs = plan.jobs_k
     work = torch.cat([k_pool, torch.zeros((plan.n_extra, lay.p, lay.d), dtype=torch.bfloat16,
                                           device="cuda")])

@@ -1,17 +1,20 @@
-"""The relocation plan (host logic, no GPU): built from the oracle's page
-tables, its jobs must leave, in the working pools, exactly the rotated pages
-that the relocated layout's page tables point at, and nothing more."""
+"""The relocation plan (rk_relocation_plan, host only, no GPU): its jobs must
+leave, in the working pools, exactly the rotated pages that the relocated
+layout's page tables point at, and nothing more.  The library's plan is
+also compared with a Python restatement (relocation_plan_ref) built from
+the oracle's page tables."""
 import numpy as np
 import pytest
 
 import oracle
-from head_aware_paged_prefill_b200 import synth
-from head_aware_paged_prefill_b200.plan import relocation_plan, visible_pages
+from head_aware_paged_prefill_b200 import binding, synth
+from relocation_plan_ref import relocation_plan, visible_pages
 
 
-def _check(lay):
+def _check(lay, plan=None):
     entries, _ = oracle.page_tables(lay)
-    plan = relocation_plan(lay, entries)
+    if plan is None:
+        plan = binding.relocation_plan(lay)
     n = int(lay.n_pages)
     n_all = n + plan.n_extra
     assert plan.layout.n_pages == n_all
@@ -49,15 +52,42 @@ def _check(lay):
 
 
 @pytest.mark.parametrize("seed", range(40))
-def test_plan_random_tiny(seed):
-    _check(synth.random_tiny(np.random.default_rng(1000 + seed)))
+def test_reference_plan_random_tiny(seed):
+    """The Python restatement on the oracle's page tables of tiny layouts
+    (page sizes 1-4, below the library's)."""
+    lay = synth.random_tiny(np.random.default_rng(1000 + seed))
+    _check(lay, relocation_plan(lay, oracle.page_tables(lay)[0]))
+
+
+def _same_plan(a, b):
+    np.testing.assert_array_equal(a.jobs_k, b.jobs_k)
+    np.testing.assert_array_equal(a.jobs_v, b.jobs_v)
+    np.testing.assert_array_equal(a.layout.segments, b.layout.segments)
+    np.testing.assert_array_equal(a.layout.page_base, b.layout.page_base)
+    assert a.n_extra == b.n_extra and a.layout.n_pages == b.layout.n_pages
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_library_plan_random_small(seed):
+    """rk_relocation_plan on random layouts of the library's page sizes:
+    the symbolic pool check, and the same jobs as the Python restatement."""
+    lay = synth.random_small(np.random.default_rng(2000 + seed), max_pages=16)
+    plan = _check(lay)
+    _same_plan(plan, relocation_plan(lay, oracle.page_tables(lay)[0]))
 
 
 def test_plan_some_random_layout_needs_appended_pages():
     # shared contents reused at two offsets must occur in the random family
-    extra = sum(_check(synth.random_tiny(np.random.default_rng(1000 + s))).n_extra
-                for s in range(40))
+    extra = sum(binding.relocation_plan(
+        synth.random_small(np.random.default_rng(2000 + s), max_pages=16)).n_extra for s in range(40))
     assert extra > 0
+
+
+@pytest.mark.parametrize("name", ["cfg2", "cfg3", "cfg4", "cfg5"])
+def test_library_plan_full_size_matches_reference(name):
+    lay = synth.CONFIGS[name]().layout
+    _same_plan(binding.relocation_plan(lay),
+               relocation_plan(lay, oracle.page_tables_closed_form(lay)[0]))
 
 
 def test_plan_cfg1():
