@@ -347,7 +347,7 @@ def _bench_scoring(torch, lay, q, k_store, dev, flush, stream, reps, peaks, peak
     retrieval head (its cached pages ranked against its tail queries, top
     16): a bandwidth measurement of the scoring launches."""
     from head_aware_paged_prefill_b200 import binding, metrics, synth
-    lay_r = synth.with_classes(lay, [synth.RETRIEVAL] * lay.hkv)
+    lay_r = synth.with_classes(lay, [synth.RETRIEVAL] * (lay.n_layers * lay.hkv))
     hl = binding.HostLayout(lay_r)
     out = binding.ScoreOutputs(binding.score_sizes(hl, 16), 16, dev, with_scores=False)
     for _ in range(3):
