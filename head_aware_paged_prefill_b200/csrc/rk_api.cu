@@ -295,27 +295,31 @@ rk_status build_score_plan(const rk_dims* d, const rk_layout* lay, const Derived
                            int top_k, ScorePlan* out) {
   const int P = d->page_size, D = d->head_dim, n_req = d->n_req;
   const int hkv = d->num_kv_heads, g = d->num_q_heads / hkv;
+  // candidates and chunks are described by runs and row ranges, so the host
+  // work is O(tables x segments); the kernels expand them
   std::vector<ScoreTable> tables;
-  std::vector<ScoreChunk> chunks;
-  std::vector<ScoreCand> cands;
   std::vector<ScoreRun> runs;
+  std::vector<ScoreRange> ranges;
   std::vector<int32_t> table_map(static_cast<size_t>(dv.n_tables), -1);
-  int64_t max_pages = 0;
+  int64_t max_pages = 0, n_chunks = 0, n_cand = 0;
   for (int r = 0; r < n_req; ++r) {
     const int L = lay->cu_seqlens[r + 1] - lay->cu_seqlens[r];
     max_pages = std::max<int64_t>(max_pages, (L + P - 1) / P);
     // the request's rows for retrieval heads: its uncached positions, merged
-    std::vector<std::pair<int, int>> rows;
-    int last_row = -1, n_rows = 0;
+    const int32_t range_begin = static_cast<int32_t>(ranges.size());
+    int last_row = -1, n_rows = 0, req_chunks = 0;
     for (int s = dv.seg_indptr[r]; s < dv.seg_indptr[r + 1]; ++s) {
       const rk_segment& sg = lay->segments[s];
       if (sg.cached || sg.len == 0) continue;
       const int a = sg.logical_start, b = a + sg.len;
-      if (!rows.empty() && rows.back().second == a) rows.back().second = b;
-      else rows.emplace_back(a, b);
+      if (static_cast<int32_t>(ranges.size()) > range_begin && ranges.back().end == a) ranges.back().end = b;
+      else ranges.push_back(ScoreRange{a, b});
       last_row = b - 1;
       n_rows += sg.len;
     }
+    const int32_t range_end = static_cast<int32_t>(ranges.size());
+    for (int32_t x = range_begin; x < range_end; ++x)
+      req_chunks += (ranges[x].end - ranges[x].begin + kScoreChunkRows - 1) / kScoreChunkRows;
     for (int layer = 0; layer < d->n_layers; ++layer)
       for (int kvh = 0; kvh < hkv; ++kvh) {
         const int lh = layer * hkv + kvh;
@@ -326,65 +330,54 @@ rk_status build_score_plan(const rk_dims* d, const rk_layout* lay, const Derived
         st.q_row0 = layer * d->total_tokens + lay->cu_seqlens[r];
         st.head0 = kvh * g;
         st.n_rows = n_rows;
-        st.chunk_begin = static_cast<int32_t>(chunks.size());
-        const int st_idx = static_cast<int>(tables.size());
-        for (const auto& rg : rows)
-          for (int a = rg.first; a < rg.second; a += kScoreChunkRows)
-            chunks.push_back(ScoreChunk{st_idx, a, std::min(kScoreChunkRows, rg.second - a), 0});
-        st.chunk_end = static_cast<int32_t>(chunks.size());
-        st.cand_begin = static_cast<int32_t>(cands.size());
+        st.range_begin = range_begin;
+        st.range_end = range_end;
+        st.req_len = L;
+        st.chunk_begin = static_cast<int32_t>(n_chunks);
+        n_chunks += req_chunks;
+        st.chunk_end = static_cast<int32_t>(n_chunks);
+        st.cand_begin = static_cast<int32_t>(n_cand);
         st.run_begin = static_cast<int32_t>(runs.size());
         for (int s = dv.seg_indptr[r]; s < dv.seg_indptr[r + 1]; ++s) {
           const rk_segment& sg = lay->segments[s];
-          if (!sg.cached) continue;
+          if (!sg.cached || sg.logical_start > last_row) continue;
           const int32_t base = lay->page_base[static_cast<int64_t>(s) * dv.n_lh + lh];
           const int32_t delta = sg.logical_start - sg.stored_pos_base;
-          const int32_t first = static_cast<int32_t>(cands.size());
-          for (int pos = sg.logical_start; pos < sg.logical_start + sg.len && pos <= last_row;
-               pos += P)
-            cands.push_back(ScoreCand{pos / P, base + (pos - sg.logical_start) / P, delta,
-                                      std::min(P, L - pos)});
-          const int32_t last = static_cast<int32_t>(cands.size());
-          if (last == first) continue;
-          if (static_cast<int32_t>(runs.size()) > st.run_begin && runs.back().delta == delta &&
-              runs.back().cand_end == first)
-            runs.back().cand_end = last;
-          else
-            runs.push_back(ScoreRun{first, last, delta, 0});
+          // pages of the segment that start at or before the last row
+          const int last_pos = std::min(sg.logical_start + sg.len - 1, last_row);
+          const int cnt = (last_pos - sg.logical_start) / P + 1;
+          runs.push_back(ScoreRun{static_cast<int32_t>(n_cand), static_cast<int32_t>(n_cand + cnt),
+                                  delta, sg.logical_start / P, base, L, {0, 0}});
+          n_cand += cnt;
         }
-        st.cand_end = static_cast<int32_t>(cands.size());
+        st.cand_end = static_cast<int32_t>(n_cand);
         st.run_end = static_cast<int32_t>(runs.size());
         if (st.cand_end - st.cand_begin > kScoreMaxCand) return RK_ERR_CAPACITY;
-        table_map[static_cast<size_t>(t)] = st_idx;
+        table_map[static_cast<size_t>(t)] = static_cast<int32_t>(tables.size());
         tables.push_back(st);
       }
   }
-  if (cands.size() >= static_cast<size_t>(kMaxI32 / 8) ||
-      chunks.size() >= static_cast<size_t>(kMaxI32 / 8))
-    return RK_ERR_INVALID_ARG;
+  if (n_cand >= kMaxI32 / 8 || n_chunks >= kMaxI32 / 8) return RK_ERR_INVALID_ARG;
   ScoreView& v = out->sv;
   v.n_st = static_cast<int32_t>(tables.size());
-  v.n_chunks = static_cast<int32_t>(chunks.size());
-  v.n_cand = static_cast<int32_t>(cands.size());
+  v.n_chunks = static_cast<int32_t>(n_chunks);
+  v.n_cand = static_cast<int32_t>(n_cand);
   v.n_runs = static_cast<int32_t>(runs.size());
-  v.n_page_blocks = static_cast<int32_t>((cands.size() + kScorePagesPerCta - 1) / kScorePagesPerCta);
+  v.n_page_blocks = static_cast<int32_t>((n_cand + kScorePagesPerCta - 1) / kScorePagesPerCta);
   v.n_tables = static_cast<int32_t>(dv.n_tables);
   v.top_k = top_k;
   v.hq = d->num_q_heads;
   v.g = g;
+  v.n_ranges = static_cast<int32_t>(ranges.size());
   // every array starts on a 16-byte boundary
   auto al4 = [](int32_t w) { return (w + 3) & ~3; };
   int32_t off = al4(static_cast<int32_t>((sizeof(ScoreView) + 3) / 4));
   v.off_tables = off;
   off = al4(off + static_cast<int32_t>(tables.size() * sizeof(ScoreTable) / 4));
-  v.off_chunks = off;
-  off = al4(off + static_cast<int32_t>(chunks.size() * sizeof(ScoreChunk) / 4));
-  v.off_cand = off;
-  off = al4(off + static_cast<int32_t>(cands.size() * sizeof(ScoreCand) / 4));
   v.off_runs = off;
   off = al4(off + static_cast<int32_t>(runs.size() * sizeof(ScoreRun) / 4));
-  v.off_cand_run = off;
-  off = al4(off + static_cast<int32_t>(cands.size()));
+  v.off_ranges = off;
+  off = al4(off + static_cast<int32_t>(ranges.size() * sizeof(ScoreRange) / 4));
   v.off_table_map = off;
   off = al4(off + static_cast<int32_t>(table_map.size()));
   v.words = off;
@@ -392,17 +385,13 @@ rk_status build_score_plan(const rk_dims* d, const rk_layout* lay, const Derived
   int32_t* w = out->img.data();
   std::memcpy(w, &v, sizeof v);
   if (!tables.empty()) std::memcpy(w + v.off_tables, tables.data(), tables.size() * sizeof(ScoreTable));
-  if (!chunks.empty()) std::memcpy(w + v.off_chunks, chunks.data(), chunks.size() * sizeof(ScoreChunk));
-  if (!cands.empty()) std::memcpy(w + v.off_cand, cands.data(), cands.size() * sizeof(ScoreCand));
   if (!runs.empty()) std::memcpy(w + v.off_runs, runs.data(), runs.size() * sizeof(ScoreRun));
-  for (size_t rn = 0; rn < runs.size(); ++rn)
-    for (int x = runs[rn].cand_begin; x < runs[rn].cand_end; ++x)
-      w[v.off_cand_run + x] = static_cast<int32_t>(rn);
+  if (!ranges.empty()) std::memcpy(w + v.off_ranges, ranges.data(), ranges.size() * sizeof(ScoreRange));
   if (!table_map.empty()) std::memcpy(w + v.off_table_map, table_map.data(), table_map.size() * 4);
   out->max_pages = max_pages;
   out->off_partials = align_up(4 * static_cast<size_t>(off), 256);
-  out->off_kbar = align_up(out->off_partials + 4 * chunks.size() * D, 256);
-  out->off_urot = align_up(out->off_kbar + 4 * cands.size() * D, 256);
+  out->off_kbar = align_up(out->off_partials + 4 * static_cast<size_t>(n_chunks) * D, 256);
+  out->off_urot = align_up(out->off_kbar + 4 * static_cast<size_t>(n_cand) * D, 256);
   out->total = align_up(out->off_urot + 4 * runs.size() * D, 256);
   return RK_OK;
 }

@@ -621,6 +621,10 @@ __device__ __forceinline__ void block_exclusive_scan(int v, int& excl, int& tota
   __syncthreads();  // warp_tot is reused by the next scan
 }
 
+// Each thread owns a contiguous slice of the request's positions, so the
+// picks come out in ascending order from two block scans (equal values
+// before the slice, picks before the slice).  Histogram updates are
+// aggregated over the lanes of a warp that hit the same bin.
 __global__ void __launch_bounds__(kImpSelectThreads)
     importance_select_kernel(const __grid_constant__ ImpArgs a) {
   __shared__ uint32_t hist[256];
@@ -634,15 +638,22 @@ __global__ void __launch_bounds__(kImpSelectThreads)
   if (k <= 0 || !a.tokens) return;
   int32_t* out = a.tokens + (static_cast<int64_t>(layer) * a.n_req + r) * a.top_k;
   const bool all = k >= L;
+  const int lane = threadIdx.x & 31;
+  const int per = (L + kImpSelectThreads - 1) / kImpSelectThreads;
+  const int p0 = threadIdx.x * per, p1 = min(L, p0 + per);
   uint32_t prefix = 0, mask = 0;
   int need = k;
   if (!all) {
     for (int shift = 24; shift >= 0; shift -= 8) {
       for (int x = threadIdx.x; x < 256; x += blockDim.x) hist[x] = 0u;
       __syncthreads();
-      for (int pos = threadIdx.x; pos < L; pos += blockDim.x) {
-        const uint32_t bits = __float_as_uint(imp[pos]);
-        if ((bits & mask) == prefix) atomicAdd(&hist[(bits >> shift) & 255u], 1u);
+      for (int j = 0; j < per; ++j) {  // uniform trip count: every lane takes part
+        const int pos = p0 + j;
+        const uint32_t bits = pos < p1 ? __float_as_uint(imp[pos]) : 0u;
+        const bool take = pos < p1 && (bits & mask) == prefix;
+        const uint32_t bin = (bits >> shift) & 255u;
+        const uint32_t peers = __match_any_sync(0xffffffffu, take ? bin : 256u + lane);
+        if (take && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
       }
       __syncthreads();
       if (threadIdx.x == 0) {
@@ -661,22 +672,28 @@ __global__ void __launch_bounds__(kImpSelectThreads)
       __syncthreads();  // s_pick is rewritten by the next pass
     }
   }
-  // prefix now holds the k-th value's bits; take every value above it and the
-  // first `need` positions equal to it, in ascending position order
-  int eq_base = 0, out_base = 0;
-  for (int c0 = 0; c0 < L; c0 += blockDim.x) {
-    const int pos = c0 + threadIdx.x;
-    const bool in = pos < L;
-    const uint32_t bits = in ? __float_as_uint(imp[pos]) : 0u;
-    const int eq = (in && !all && bits == prefix) ? 1 : 0;
-    int eq_excl, eq_tot;
-    block_exclusive_scan(eq, eq_excl, eq_tot, warp_tot);
-    const bool sel = in && (all || bits > prefix || (eq && eq_base + eq_excl < need));
-    int s_excl, s_tot;
-    block_exclusive_scan(sel ? 1 : 0, s_excl, s_tot, warp_tot);
-    if (sel && out_base + s_excl < k) out[out_base + s_excl] = pos;  // never past k
-    eq_base += eq_tot;
-    out_base += s_tot;
+  // prefix holds the k-th value's bits: every value above it is picked, and
+  // the first `need` positions whose value equals it
+  int n_gt = 0, n_eq = 0;
+  for (int pos = p0; pos < p1; ++pos) {
+    const uint32_t bits = __float_as_uint(imp[pos]);
+    n_gt += (all || bits > prefix) ? 1 : 0;
+    n_eq += (!all && bits == prefix) ? 1 : 0;
+  }
+  int eq_before, eq_tot;
+  block_exclusive_scan(n_eq, eq_before, eq_tot, warp_tot);
+  const int take_eq = max(0, min(n_eq, need - eq_before));
+  int sel_before, sel_tot;
+  block_exclusive_scan(n_gt + take_eq, sel_before, sel_tot, warp_tot);
+  int o = sel_before, eq_seen = 0;
+  for (int pos = p0; pos < p1 && o < k; ++pos) {
+    const uint32_t bits = __float_as_uint(imp[pos]);
+    bool sel = all || bits > prefix;
+    if (!sel && bits == prefix && eq_seen < take_eq) {
+      sel = true;
+      ++eq_seen;
+    }
+    if (sel) out[o++] = pos;
   }
 }
 

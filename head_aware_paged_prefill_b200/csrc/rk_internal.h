@@ -110,7 +110,7 @@ struct PrefillLaunchArgs {
 // ---- retrieval page scoring (host image read by the scoring kernels)
 
 constexpr int kScoreChunkRows = 64;   // query rows summed by one CTA
-constexpr int kScorePagesPerCta = 8;  // candidate pages per CTA (one warp each)
+constexpr int kScorePagesPerCta = 16;  // candidate pages per CTA (one warp each)
 constexpr int kScoreMaxCand = 4096;   // candidate pages of one table
 constexpr int kScoreMaxTopK = 64;
 
@@ -119,28 +119,29 @@ struct ScoreTable {  // one retrieval table that has rows
   int32_t q_row0;    // layer * T + cu[r]: packed q row of the request's position 0
   int32_t head0;     // first q head of the kv head
   int32_t n_rows;    // computed rows (uncached positions)
-  int32_t chunk_begin, chunk_end;  // its query chunks
+  int32_t chunk_begin, chunk_end;  // its query chunks (kScoreChunkRows rows of one range each)
   int32_t cand_begin, cand_end;    // its candidate pages (ascending page)
   int32_t run_begin, run_end;      // its runs of candidates sharing one delta
+  int32_t range_begin, range_end;  // its row ranges (the request's uncached rows, merged)
+  int32_t req_len;
+  int32_t pad[3];
+};
+struct ScoreRun {  // candidates [cand_begin, cand_end): consecutive pages of one cached segment
+  int32_t cand_begin, cand_end, delta;
+  int32_t first_page;  // request page of the run's first candidate
+  int32_t phys_base;   // its physical page (the run's pages are consecutive ids)
+  int32_t req_len;     // length of the request (keys of its last page)
   int32_t pad[2];
 };
-struct ScoreChunk {  // rows [row_begin, row_begin + n_rows) of one table
-  int32_t st, row_begin, n_rows, pad;
-};
-struct ScoreCand {  // a candidate page of a table
-  int32_t page, phys, delta, n_valid;
-};
-struct ScoreRun {  // candidates [cand_begin, cand_end) relocated by delta
-  int32_t cand_begin, cand_end, delta, pad;
+struct ScoreRange {  // request-local rows [begin, end)
+  int32_t begin, end;
 };
 struct ScoreView {
   int32_t n_st, n_chunks, n_cand, n_runs, n_page_blocks, n_tables, top_k;
-  int32_t hq, g;
+  int32_t hq, g, n_ranges;
   int32_t off_tables;     // ScoreTable[n_st]
-  int32_t off_chunks;     // ScoreChunk[n_chunks]
-  int32_t off_cand;       // ScoreCand[n_cand]
   int32_t off_runs;       // ScoreRun[n_runs]
-  int32_t off_cand_run;   // int32[n_cand]: run of each candidate
+  int32_t off_ranges;     // ScoreRange[n_ranges]
   int32_t off_table_map;  // int32[n_tables]: score table of a table, -1 if none
   int32_t words;
 };

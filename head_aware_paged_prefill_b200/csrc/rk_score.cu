@@ -14,15 +14,20 @@
 //   picks    = the top k candidate pages (cached, starting at or before the
 //              last row), ties to the lower page, ascending page order.
 //
+// The host describes a table's candidates by runs (the pages of one cached
+// segment that start at or before the last row) and its query chunks by
+// the request's uncached row ranges; the kernels expand both.
 // Two launches:
 //   1. streaming (HBM bound): the first CTAs each sum the queries of a
 //      64-row chunk of one table over the kv head's q heads (fp32, fixed
-//      order, 16-byte loads); the others average the stored keys of 8
+//      order, 16-byte loads); the others average the stored keys of 16
 //      candidate pages, one warp per page;
 //   2. one CTA per table: u from the table's chunk sums (in chunk order),
 //      R(-delta) u of every run (into the workspace), one warp per candidate
-//      for its dot product, then a bitonic sort in shared memory of (score,
-//      page) keys; the first k, in ascending page order, are the picks.
+//      for its dot product, then the picks: each candidate's rank is the
+//      number of (score, page) keys above its own (up to 2048 candidates;
+//      a bitonic sort in shared memory above that); the first k, in
+//      ascending page order.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -42,7 +47,7 @@ struct ScoreFreqs {
   double f[64];  // theta^(-2m/D), m < D/2
 };
 
-constexpr int kStreamThreads = 256;
+constexpr int kStreamThreads = 512;
 static_assert(kStreamThreads == 32 * kScorePagesPerCta, "one warp per page");
 
 // 1. query chunk sums and candidate key means.
@@ -61,16 +66,34 @@ __global__ void __launch_bounds__(kStreamThreads)
   __shared__ float acc_s[S][D];
   const int n_chunks = sv->n_chunks;
   if (static_cast<int>(blockIdx.x) < n_chunks) {
-    const ScoreChunk ch = reinterpret_cast<const ScoreChunk*>(sv_arr(sv, sv->off_chunks))[blockIdx.x];
-    const ScoreTable st = reinterpret_cast<const ScoreTable*>(sv_arr(sv, sv->off_tables))[ch.st];
+    const ScoreTable* tabs = reinterpret_cast<const ScoreTable*>(sv_arr(sv, sv->off_tables));
+    const ScoreRange* rgs = reinterpret_cast<const ScoreRange*>(sv_arr(sv, sv->off_ranges));
+    const int b = blockIdx.x;
+    int lo = 0, hi = sv->n_st;  // last table with chunk_begin <= b
+    while (hi - lo > 1) {
+      const int m = (lo + hi) >> 1;
+      if (tabs[m].chunk_begin <= b) lo = m; else hi = m;
+    }
+    const ScoreTable st = tabs[lo];
+    int lc = b - st.chunk_begin, row_begin = 0, n_rows = 0;
+    for (int x = st.range_begin; x < st.range_end; ++x) {
+      const int len = rgs[x].end - rgs[x].begin;
+      const int nck = (len + kScoreChunkRows - 1) / kScoreChunkRows;
+      if (lc < nck) {
+        row_begin = rgs[x].begin + lc * kScoreChunkRows;
+        n_rows = min(kScoreChunkRows, rgs[x].end - row_begin);
+        break;
+      }
+      lc -= nck;
+    }
     const int g = sv->g, hq = sv->hq;
     const int cg = threadIdx.x % CG, slot = threadIdx.x / CG;
-    const int n_pairs = ch.n_rows * g;
+    const int n_pairs = n_rows * g;
     float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll 4
     for (int pr = slot; pr < n_pairs; pr += S) {
       const int i = pr / g, h = pr - i * g;
-      const int64_t row = static_cast<int64_t>(st.q_row0) + ch.row_begin + i;
+      const int64_t row = static_cast<int64_t>(st.q_row0) + row_begin + i;
       const uint4 raw =
           *reinterpret_cast<const uint4*>(q + (row * hq + st.head0 + h) * D + cg * 8);
       const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
@@ -94,13 +117,22 @@ __global__ void __launch_bounds__(kStreamThreads)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cand = (blockIdx.x - n_chunks) * kScorePagesPerCta + warp;
   if (cand >= sv->n_cand) return;
-  const ScoreCand cd = reinterpret_cast<const ScoreCand*>(sv_arr(sv, sv->off_cand))[cand];
-  const __nv_bfloat16* base = k_store + (static_cast<int64_t>(cd.phys) * P) * D + lane * CPL;
+  const ScoreRun* runs = reinterpret_cast<const ScoreRun*>(sv_arr(sv, sv->off_runs));
+  int lo = 0, hi = sv->n_runs;  // last run with cand_begin <= cand
+  while (hi - lo > 1) {
+    const int m = (lo + hi) >> 1;
+    if (runs[m].cand_begin <= cand) lo = m; else hi = m;
+  }
+  const ScoreRun rn = runs[lo];
+  const int page = rn.first_page + (cand - rn.cand_begin);
+  const int n_valid = min(P, rn.req_len - page * P);
+  const int64_t phys = static_cast<int64_t>(rn.phys_base) + (cand - rn.cand_begin);
+  const __nv_bfloat16* base = k_store + (phys * P) * D + lane * CPL;
   float acc[CPL];
 #pragma unroll
   for (int k = 0; k < CPL; ++k) acc[k] = 0.f;
 #pragma unroll 8
-  for (int r = 0; r < cd.n_valid; ++r) {
+  for (int r = 0; r < n_valid; ++r) {
     const __nv_bfloat16* kr = base + static_cast<int64_t>(r) * D;
     if constexpr (CPL == 4) {
       const uint2 raw = *reinterpret_cast<const uint2*>(kr);
@@ -116,7 +148,7 @@ __global__ void __launch_bounds__(kStreamThreads)
       acc[1] += x.y;
     }
   }
-  const float inv = 1.f / static_cast<float>(cd.n_valid);
+  const float inv = 1.f / static_cast<float>(n_valid);
 #pragma unroll
   for (int k = 0; k < CPL; ++k)
     kbar[static_cast<int64_t>(cand) * D + lane * CPL + k] = acc[k] * inv;
@@ -128,6 +160,7 @@ __device__ __forceinline__ uint32_t order_bits(float f) {
 }
 
 constexpr int kRankThreads = 1024;
+constexpr int kRankCount = 2048;  // candidates ranked by counting (a sort above)
 constexpr int kRankBatch = 8;  // candidates a warp loads before reducing
 
 // 2. scores and picks of one table
@@ -154,7 +187,6 @@ __global__ void __launch_bounds__(kRankThreads)
     return;
   }
   const ScoreTable st = reinterpret_cast<const ScoreTable*>(sv_arr(sv, sv->off_tables))[st_idx];
-  const ScoreCand* cands = reinterpret_cast<const ScoreCand*>(sv_arr(sv, sv->off_cand));
   const ScoreRun* runs = reinterpret_cast<const ScoreRun*>(sv_arr(sv, sv->off_runs));
   // u: the table's chunk sums, column c, chunks j, j + R, ... per thread,
   // runs added in order, divided by the row count
@@ -201,8 +233,16 @@ __global__ void __launch_bounds__(kRankThreads)
   {
     constexpr int CPL = D / 32;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int32_t* cand_run = sv_arr(sv, sv->off_cand_run);
     constexpr int NW = kRankThreads / 32;
+    // run of a table-local candidate: the table's runs, by cand_begin
+    auto run_of = [&](int xc) {
+      int lo = st.run_begin, hi = st.run_end;
+      while (hi - lo > 1) {
+        const int m = (lo + hi) >> 1;
+        if (runs[m].cand_begin <= xc) lo = m; else hi = m;
+      }
+      return lo;
+    };
     for (int x0 = warp * kRankBatch; x0 < n; x0 += NW * kRankBatch) {
       float sc[kRankBatch];
 #pragma unroll
@@ -212,7 +252,7 @@ __global__ void __launch_bounds__(kRankThreads)
         if (x < n) {
           const int xc = st.cand_begin + x;
           const float* kb = kbar + static_cast<int64_t>(xc) * D + lane * CPL;
-          const float* ub = urot + static_cast<int64_t>(cand_run[xc]) * D + lane * CPL;
+          const float* ub = urot + static_cast<int64_t>(run_of(xc)) * D + lane * CPL;
 #pragma unroll
           for (int k = 0; k < CPL; ++k) sc[b] = fmaf(ub[k], kb[k], sc[b]);
         }
@@ -226,7 +266,8 @@ __global__ void __launch_bounds__(kRankThreads)
 #pragma unroll
         for (int b = 1; b < kRankBatch; ++b) mine = lane == b ? sc[b] : mine;
         const int x = x0 + lane, xc = st.cand_begin + x;
-        const int pg = cands[xc].page;
+        const ScoreRun& rn = runs[run_of(xc)];
+        const int pg = rn.first_page + (xc - rn.cand_begin);
         if (out_scores && pg < scores_stride) out_scores[t * scores_stride + pg] = mine;
         const float rank_sc = isnan(mine) ? -INFINITY : mine;  // a NaN score (bad input) ranks last
         s_key[x] = (static_cast<unsigned long long>(order_bits(rank_sc)) << 32) |
@@ -235,27 +276,48 @@ __global__ void __launch_bounds__(kRankThreads)
     }
   }
   __syncthreads();
-  // bitonic sort, descending: higher score first, equal score to the lower page
-  for (int k = 2; k <= n2; k <<= 1)
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = threadIdx.x; i < n2; i += kRankThreads) {
-        const int p = i ^ j;
-        if (p > i) {
-          const unsigned long long a = s_key[i], b = s_key[p];
-          if (((i & k) == 0) ? (a < b) : (a > b)) {
-            s_key[i] = b;
-            s_key[p] = a;
+  const int n_pick = n < top_k ? n : top_k;
+  if (n <= kRankCount) {
+    // rank of a key = the keys above it (keys are distinct: the page is in
+    // the low bits); a candidate is picked if its rank is below n_pick, and
+    // its output slot is the number of picked candidates before it (the
+    // candidates ascend in page)
+    __shared__ int s_picked[kRankCount];
+    for (int x = threadIdx.x; x < n; x += kRankThreads) {
+      const unsigned long long kx = s_key[x];
+      int rank = 0;
+      for (int y = 0; y < n; ++y) rank += s_key[y] > kx ? 1 : 0;
+      s_picked[x] = rank < n_pick ? 1 : 0;
+    }
+    __syncthreads();
+    for (int x = threadIdx.x; x < n; x += kRankThreads) {
+      if (!s_picked[x]) continue;
+      int pos = 0;
+      for (int y = 0; y < x; ++y) pos += s_picked[y];
+      out_pages[t * top_k + pos] = static_cast<int32_t>(~static_cast<uint32_t>(s_key[x]));
+    }
+  } else {
+    // bitonic sort, descending: higher score first, equal score to the lower page
+    for (int k = 2; k <= n2; k <<= 1)
+      for (int j = k >> 1; j > 0; j >>= 1) {
+        for (int i = threadIdx.x; i < n2; i += kRankThreads) {
+          const int p = i ^ j;
+          if (p > i) {
+            const unsigned long long a = s_key[i], b = s_key[p];
+            if (((i & k) == 0) ? (a < b) : (a > b)) {
+              s_key[i] = b;
+              s_key[p] = a;
+            }
           }
         }
+        __syncthreads();
       }
-      __syncthreads();
+    if (threadIdx.x < n_pick) {
+      const uint32_t pg = ~static_cast<uint32_t>(s_key[threadIdx.x]);
+      int pos = 0;
+      for (int x = 0; x < n_pick; ++x) pos += (~static_cast<uint32_t>(s_key[x])) < pg ? 1 : 0;
+      out_pages[t * top_k + pos] = static_cast<int32_t>(pg);
     }
-  const int n_pick = n < top_k ? n : top_k;
-  if (threadIdx.x < n_pick) {
-    const uint32_t pg = ~static_cast<uint32_t>(s_key[threadIdx.x]);
-    int pos = 0;
-    for (int x = 0; x < n_pick; ++x) pos += (~static_cast<uint32_t>(s_key[x])) < pg ? 1 : 0;
-    out_pages[t * top_k + pos] = static_cast<int32_t>(pg);
   }
   if (threadIdx.x == 0) out_count[t] = n_pick;
 }
