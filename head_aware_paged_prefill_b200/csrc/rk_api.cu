@@ -301,7 +301,7 @@ rk_status build_score_plan(const rk_dims* d, const rk_layout* lay, const Derived
   std::vector<ScoreRun> runs;
   std::vector<ScoreRange> ranges;
   std::vector<int32_t> table_map(static_cast<size_t>(dv.n_tables), -1);
-  int64_t max_pages = 0, n_chunks = 0, n_cand = 0, n_units = 0;
+  int64_t max_pages = 0, n_chunks = 0, n_cand = 0;
   for (int r = 0; r < n_req; ++r) {
     const int L = lay->cu_seqlens[r + 1] - lay->cu_seqlens[r];
     max_pages = std::max<int64_t>(max_pages, (L + P - 1) / P);
@@ -352,9 +352,6 @@ rk_status build_score_plan(const rk_dims* d, const rk_layout* lay, const Derived
         }
         st.cand_end = static_cast<int32_t>(n_cand);
         st.run_end = static_cast<int32_t>(runs.size());
-        st.unit_begin = static_cast<int32_t>(n_units);
-        n_units += (st.cand_end - st.cand_begin + kScorePagesPerUnit - 1) / kScorePagesPerUnit;
-        st.unit_end = static_cast<int32_t>(n_units);
         if (st.cand_end - st.cand_begin > kScoreMaxCand) return RK_ERR_CAPACITY;
         table_map[static_cast<size_t>(t)] = static_cast<int32_t>(tables.size());
         tables.push_back(st);
@@ -366,7 +363,7 @@ rk_status build_score_plan(const rk_dims* d, const rk_layout* lay, const Derived
   v.n_chunks = static_cast<int32_t>(n_chunks);
   v.n_cand = static_cast<int32_t>(n_cand);
   v.n_runs = static_cast<int32_t>(runs.size());
-  v.n_page_units = static_cast<int32_t>(n_units);
+  v.n_page_blocks = static_cast<int32_t>((n_cand + kScorePagesPerCta - 1) / kScorePagesPerCta);
   v.n_tables = static_cast<int32_t>(dv.n_tables);
   v.top_k = top_k;
   v.hq = d->num_q_heads;
@@ -383,8 +380,6 @@ rk_status build_score_plan(const rk_dims* d, const rk_layout* lay, const Derived
   off = al4(off + static_cast<int32_t>(ranges.size() * sizeof(ScoreRange) / 4));
   v.off_table_map = off;
   off = al4(off + static_cast<int32_t>(table_map.size()));
-  v.off_done = off;
-  off = al4(off + static_cast<int32_t>(tables.size()));
   v.words = off;
   out->img.assign(static_cast<size_t>(off), 0);
   int32_t* w = out->img.data();

@@ -594,17 +594,38 @@ __global__ void __launch_bounds__(256) importance_reduce_kernel(const __grid_con
 // 4. the top-k tokens of one (request, layer)
 // ---------------------------------------------------------------------------
 
-// Each warp owns a contiguous slice of the request's positions, read 32
-// consecutive positions at a time (coalesced); the picks come out in
-// ascending order from ballots inside the warp and two scans over the warps
-// (equal values before the slice, picks before the slice).  Histogram
-// updates are aggregated over the lanes of a warp that hit the same bin.
+// Exclusive prefix sum over the block (blockDim.x a multiple of 32, <= 1024);
+// every thread gets its own exclusive sum and the block total.
+__device__ __forceinline__ void block_exclusive_scan(int v, int& excl, int& total, int* warp_tot) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_tot[w] = x;
+  __syncthreads();
+  if (w == 0) {
+    int tt = lane < nw ? warp_tot[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, tt, o);
+      if (lane >= o) tt += y;
+    }
+    warp_tot[lane] = tt;
+  }
+  __syncthreads();
+  excl = x - v + (w > 0 ? warp_tot[w - 1] : 0);
+  total = warp_tot[nw - 1];
+  __syncthreads();  // warp_tot is reused by the next scan
+}
+
 __global__ void __launch_bounds__(kImpSelectThreads)
     importance_select_kernel(const __grid_constant__ ImpArgs a) {
-  constexpr int NW = kImpSelectThreads / 32;
   __shared__ uint32_t hist[256];
   __shared__ int s_pick[2];
-  __shared__ int w_eq[NW], w_sel[NW];
+  __shared__ int warp_tot[32];
   const int r = blockIdx.x % a.n_req, layer = blockIdx.x / a.n_req;
   const int t0 = a.cu[r], L = a.cu[r + 1] - t0;
   const float* imp = a.importance + static_cast<int64_t>(layer) * a.total_tokens + t0;
@@ -613,22 +634,15 @@ __global__ void __launch_bounds__(kImpSelectThreads)
   if (k <= 0 || !a.tokens) return;
   int32_t* out = a.tokens + (static_cast<int64_t>(layer) * a.n_req + r) * a.top_k;
   const bool all = k >= L;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int steps = (L + kImpSelectThreads - 1) / kImpSelectThreads;  // 32-position steps per warp
-  const int w0 = warp * steps * 32;
   uint32_t prefix = 0, mask = 0;
   int need = k;
   if (!all) {
     for (int shift = 24; shift >= 0; shift -= 8) {
       for (int x = threadIdx.x; x < 256; x += blockDim.x) hist[x] = 0u;
       __syncthreads();
-      for (int j = 0; j < steps; ++j) {
-        const int pos = w0 + j * 32 + lane;
-        const uint32_t bits = pos < L ? __float_as_uint(imp[pos]) : 0u;
-        const bool take = pos < L && (bits & mask) == prefix;
-        const uint32_t bin = (bits >> shift) & 255u;
-        const uint32_t peers = __match_any_sync(0xffffffffu, take ? bin : 256u + lane);
-        if (take && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+      for (int pos = threadIdx.x; pos < L; pos += blockDim.x) {
+        const uint32_t bits = __float_as_uint(imp[pos]);
+        if ((bits & mask) == prefix) atomicAdd(&hist[(bits >> shift) & 255u], 1u);
       }
       __syncthreads();
       if (threadIdx.x == 0) {
@@ -647,37 +661,22 @@ __global__ void __launch_bounds__(kImpSelectThreads)
       __syncthreads();  // s_pick is rewritten by the next pass
     }
   }
-  // prefix holds the k-th value's bits: every value above it is picked, and
-  // the first `need` positions whose value equals it
-  int n_gt = 0, n_eq = 0;
-  for (int j = 0; j < steps; ++j) {
-    const int pos = w0 + j * 32 + lane;
-    const uint32_t bits = pos < L ? __float_as_uint(imp[pos]) : 0u;
-    n_gt += __popc(__ballot_sync(0xffffffffu, pos < L && (all || bits > prefix)));
-    n_eq += __popc(__ballot_sync(0xffffffffu, pos < L && !all && bits == prefix));
-  }
-  if (lane == 0) w_eq[warp] = n_eq;
-  __syncthreads();
-  int eq_before = 0;
-  for (int w = 0; w < warp; ++w) eq_before += w_eq[w];
-  const int take_eq = max(0, min(n_eq, need - eq_before));
-  if (lane == 0) w_sel[warp] = n_gt + take_eq;
-  __syncthreads();
-  int o = 0;
-  for (int w = 0; w < warp; ++w) o += w_sel[w];
-  int eq_seen = 0;
-  const uint32_t lt = (1u << lane) - 1u;
-  for (int j = 0; j < steps && o < k; ++j) {
-    const int pos = w0 + j * 32 + lane;
-    const uint32_t bits = pos < L ? __float_as_uint(imp[pos]) : 0u;
-    const bool gt = pos < L && (all || bits > prefix);
-    const bool eq = pos < L && !all && bits == prefix;
-    const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
-    const bool sel = gt || (eq && eq_seen + __popc(eqm & lt) < take_eq);
-    const uint32_t selm = __ballot_sync(0xffffffffu, sel);
-    if (sel && o + __popc(selm & lt) < k) out[o + __popc(selm & lt)] = pos;
-    o += __popc(selm);
-    eq_seen += __popc(eqm);
+  // prefix now holds the k-th value's bits; take every value above it and the
+  // first `need` positions equal to it, in ascending position order
+  int eq_base = 0, out_base = 0;
+  for (int c0 = 0; c0 < L; c0 += blockDim.x) {
+    const int pos = c0 + threadIdx.x;
+    const bool in = pos < L;
+    const uint32_t bits = in ? __float_as_uint(imp[pos]) : 0u;
+    const int eq = (in && !all && bits == prefix) ? 1 : 0;
+    int eq_excl, eq_tot;
+    block_exclusive_scan(eq, eq_excl, eq_tot, warp_tot);
+    const bool sel = in && (all || bits > prefix || (eq && eq_base + eq_excl < need));
+    int s_excl, s_tot;
+    block_exclusive_scan(sel ? 1 : 0, s_excl, s_tot, warp_tot);
+    if (sel && out_base + s_excl < k) out[out_base + s_excl] = pos;  // never past k
+    eq_base += eq_tot;
+    out_base += s_tot;
   }
 }
 

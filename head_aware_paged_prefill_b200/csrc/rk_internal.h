@@ -110,7 +110,7 @@ struct PrefillLaunchArgs {
 // ---- retrieval page scoring (host image read by the scoring kernels)
 
 constexpr int kScoreChunkRows = 64;   // query rows summed by one CTA
-constexpr int kScorePagesPerUnit = 4;  // candidate pages per page unit (four warps each)
+constexpr int kScorePagesPerCta = 8;  // candidate pages per CTA (one warp each)
 constexpr int kScoreMaxCand = 4096;   // candidate pages of one table
 constexpr int kScoreMaxTopK = 64;
 
@@ -124,8 +124,7 @@ struct ScoreTable {  // one retrieval table that has rows
   int32_t run_begin, run_end;      // its runs of candidates sharing one delta
   int32_t range_begin, range_end;  // its row ranges (the request's uncached rows, merged)
   int32_t req_len;
-  int32_t unit_begin, unit_end;    // its page units (kScorePagesPerUnit candidates each)
-  int32_t pad;
+  int32_t pad[3];
 };
 struct ScoreRun {  // candidates [cand_begin, cand_end): consecutive pages of one cached segment
   int32_t cand_begin, cand_end, delta;
@@ -138,19 +137,19 @@ struct ScoreRange {  // request-local rows [begin, end)
   int32_t begin, end;
 };
 struct ScoreView {
-  int32_t n_st, n_chunks, n_cand, n_runs, n_page_units, n_tables, top_k;
+  int32_t n_st, n_chunks, n_cand, n_runs, n_page_blocks, n_tables, top_k;
   int32_t hq, g, n_ranges;
   int32_t off_tables;     // ScoreTable[n_st]
   int32_t off_runs;       // ScoreRun[n_runs]
   int32_t off_ranges;     // ScoreRange[n_ranges]
   int32_t off_table_map;  // int32[n_tables]: score table of a table, -1 if none
-  int32_t off_done;       // int32[n_st]: units finished per score table (zero when uploaded)
   int32_t words;
 };
 
-// One persistent launch: query units (64-row chunks) and page units
-// (kScorePagesPerUnit candidates), and each table ranked by the CTA that
-// finishes its last unit.
+// One launch sums the queries of every 64-row chunk (the first n_chunks
+// CTAs) and averages the stored keys of every candidate page (the other
+// CTAs, kScorePagesPerCta pages each); a second, one CTA per table, scores
+// and ranks.
 cudaError_t launch_score(const ScoreView* sv_dev, const ScoreView& sv_host, const void* q,
                          const void* k_store, int D, int P, const double* inv_freq_host,
                          float* partials, float* kbar, float* urot, int32_t* out_pages,
