@@ -121,7 +121,7 @@ def _stream(stream) -> ctypes.c_void_p:
 
 
 class RkDecodeSizes(ctypes.Structure):
-    _fields_ = [("max_splits", ctypes.c_int64), ("workspace_bytes", ctypes.c_int64)]
+    _fields_ = [("n_pieces", ctypes.c_int64), ("workspace_bytes", ctypes.c_int64)]
 
 
 class RkRelocationSizes(ctypes.Structure):

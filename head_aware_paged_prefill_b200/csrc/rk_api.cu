@@ -673,23 +673,90 @@ extern "C" rk_status rk_score_retrieval_pages(const rk_dims* dims, const rk_layo
 
 namespace rk {
 namespace {
+void importance_table_pages(const rk_dims* d, const rk_layout* lay, const Derived& dv, int r,
+                            int lh, int64_t t, std::vector<int>* out);
+
 struct DecodePlan {
-  int max_splits = 0;
-  size_t off_req_len = 0, off_part_o = 0, off_part_ml = 0, total = 0;
+  int64_t n_pieces = 0;
+  int n_cta = 0, per = 0;
+  int64_t total = 0;                // decode pages of all tables
+  std::vector<int32_t> upload;      // req_len [n_req], then DecodeTable [n_tables]
+  size_t off_req_len = 0, off_tables = 0, off_part_o = 0, off_part_ml = 0, bytes = 0;
 };
-rk_status plan_decode(const rk_dims* d, const Derived& dv, DecodePlan* out) {
+
+// The decode row of request r is its last position.  A table reads the
+// entries of its page table (importance_table_pages: the class rule of the
+// select kernel) from the first whose last key is at or after the row's
+// first visible key; a table whose row set does not hold the row reads
+// nothing.  The tables' decode pages, concatenated, are cut into n_cta
+// equal ranges, one per CTA (2 per SM), so every CTA streams the same
+// number of pages; a range that spans tables gives one partial result per
+// (table, CTA) piece.
+rk_status plan_decode(const rk_dims* d, const rk_layout* lay, const Derived& dv, DecodePlan* out) {
   const int g = d->num_q_heads / d->num_kv_heads;
   if (g > kDecodeMaxG || dv.n_lh > kDecodeMaxLh) return RK_ERR_INVALID_ARG;
-  int64_t max_pages = 0;
-  for (int r = 0; r < d->n_req; ++r)
-    max_pages = std::max<int64_t>(max_pages, dv.page_prefix[r + 1] - dv.page_prefix[r]);
-  out->max_splits = static_cast<int>((max_pages + kDecodePages - 1) / kDecodePages);
-  const size_t slots = static_cast<size_t>(dv.n_tables) * out->max_splits * g;
-  // the first 256 bytes hold the device error word, then the request lengths
+  const int P = d->page_size, hkv = d->num_kv_heads, W = lay->class_window[RK_LOCAL];
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    sms = 148;  // sizes only: the launch queries the device again
+  cudaGetLastError();
+  const size_t nt = static_cast<size_t>(dv.n_tables);
+  std::vector<DecodeTable> tabs(nt);
+  std::vector<int> pages;
+  int64_t total = 0;
+  for (int r = 0; r < d->n_req; ++r) {
+    const int L = lay->cu_seqlens[r + 1] - lay->cu_seqlens[r];
+    const int row = L - 1;
+    bool last_unc = false;  // the request's last position is uncached
+    if (L > 0)
+      for (int s = dv.seg_indptr[r]; s < dv.seg_indptr[r + 1]; ++s)
+        if (lay->segments[s].logical_start + lay->segments[s].len == L) last_unc = !lay->segments[s].cached;
+    for (int layer = 0; layer < d->n_layers; ++layer)
+      for (int kvh = 0; kvh < hkv; ++kvh) {
+        const int lh = layer * hkv + kvh;
+        const int64_t t = (static_cast<int64_t>(r) * d->n_layers + layer) * hkv + kvh;
+        DecodeTable& dt = tabs[static_cast<size_t>(t)];
+        dt.g0 = static_cast<int32_t>(total);
+        const int cls = lay->class_map[lh];
+        const bool has_row = L > 0 && (cls == RK_GLOBAL || cls == RK_DENSE || last_unc);
+        importance_table_pages(d, lay, dv, r, lh, t, &pages);
+        dt.n_e = static_cast<int32_t>(pages.size());
+        if (!has_row || pages.empty()) continue;
+        const int lo = cls == RK_LOCAL ? row - W + 1 : 0;
+        int first = 0;
+        while (first < dt.n_e && pages[first] + std::min(P, L - pages[first]) - 1 < lo) ++first;
+        dt.first = first;
+        dt.n_dec = dt.n_e - first;
+        total += dt.n_dec;
+      }
+  }
+  if (total >= kMaxI32) return RK_ERR_INVALID_ARG;
+  out->total = total;
+  out->n_cta = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(2 * sms, total)));
+  out->per = static_cast<int>(std::max<int64_t>(1, (total + out->n_cta - 1) / out->n_cta));
+  out->n_cta = static_cast<int>(std::max<int64_t>(1, (total + out->per - 1) / out->per));
+  int64_t pieces = 0;
+  for (DecodeTable& dt : tabs) {
+    dt.piece_base = static_cast<int32_t>(pieces);
+    if (dt.n_dec == 0) continue;
+    dt.c_first = dt.g0 / out->per;
+    dt.n_pieces = (dt.g0 + dt.n_dec - 1) / out->per - dt.c_first + 1;
+    pieces += dt.n_pieces;
+  }
+  out->n_pieces = pieces;
+  const int n_req = d->n_req;
+  const size_t rl_words = align_up(static_cast<size_t>(n_req), 4);
+  out->upload.assign(rl_words + nt * (sizeof(DecodeTable) / 4), 0);
+  for (int r = 0; r < n_req; ++r) out->upload[r] = lay->cu_seqlens[r + 1] - lay->cu_seqlens[r];
+  std::memcpy(out->upload.data() + rl_words, tabs.data(), nt * sizeof(DecodeTable));
+  // the first 256 bytes hold the device error word, then the upload, then
+  // one partial (o [G][D], (m, l) [G]) per piece
   out->off_req_len = 256;
-  out->off_part_o = align_up(out->off_req_len + 4 * static_cast<size_t>(d->n_req), 256);
-  out->off_part_ml = align_up(out->off_part_o + 4 * slots * d->head_dim, 256);
-  out->total = align_up(out->off_part_ml + 8 * slots, 256);
+  out->off_tables = out->off_req_len + 4 * rl_words;
+  out->off_part_o = align_up(out->off_req_len + 4 * out->upload.size(), 256);
+  out->off_part_ml = align_up(out->off_part_o + 4 * static_cast<size_t>(pieces) * g * d->head_dim, 256);
+  out->bytes = align_up(out->off_part_ml + 8 * static_cast<size_t>(pieces) * g, 256);
   return RK_OK;
 }
 }  // namespace
@@ -703,9 +770,9 @@ extern "C" rk_status rk_decode_query_sizes(const rk_dims* dims, const rk_layout*
   Derived dv;
   if ((st = check_layout(dims, layout, &dv)) != RK_OK) return st;
   DecodePlan plan;
-  if ((st = plan_decode(dims, dv, &plan)) != RK_OK) return st;
-  out->max_splits = plan.max_splits;
-  out->workspace_bytes = static_cast<int64_t>(plan.total);
+  if ((st = plan_decode(dims, layout, dv, &plan)) != RK_OK) return st;
+  out->n_pieces = plan.n_pieces;
+  out->workspace_bytes = static_cast<int64_t>(plan.bytes);
   return RK_OK;
 }
 
@@ -719,7 +786,7 @@ extern "C" rk_status rk_segpaged_decode(const rk_dims* dims, const rk_layout* la
   Derived dv;
   if ((st = check_layout(dims, layout, &dv)) != RK_OK) return st;
   DecodePlan plan;
-  if ((st = plan_decode(dims, dv, &plan)) != RK_OK) return st;
+  if ((st = plan_decode(dims, layout, dv, &plan)) != RK_OK) return st;
   if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return RK_ERR_INVALID_ARG;
   if (!q || !k_pool || !v_pool || !vis || !o || !workspace || !vis->entries ||
       !vis->entry_start || !vis->entry_count || !vis->ranges || !vis->range_start ||
@@ -730,14 +797,11 @@ extern "C" rk_status rk_segpaged_decode(const rk_dims* dims, const rk_layout* la
     return RK_ERR_INVALID_ARG;
   if (vis->entry_capacity < dv.entry_capacity || vis->range_capacity < dv.range_capacity)
     return RK_ERR_CAPACITY;
-  if (workspace_bytes < plan.total) return RK_ERR_CAPACITY;
+  if (workspace_bytes < plan.bytes) return RK_ERR_CAPACITY;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  std::vector<int32_t> req_len(static_cast<size_t>(dims->n_req));
-  for (int r = 0; r < dims->n_req; ++r)
-    req_len[r] = layout->cu_seqlens[r + 1] - layout->cu_seqlens[r];
   if (cudaMemsetAsync(ws, 0, 256, s) != cudaSuccess ||
-      cudaMemcpyAsync(ws + plan.off_req_len, req_len.data(), 4 * req_len.size(),
+      cudaMemcpyAsync(ws + plan.off_req_len, plan.upload.data(), 4 * plan.upload.size(),
                       cudaMemcpyHostToDevice, s) != cudaSuccess)
     return RK_ERR_CUDA;
   DecodeLaunchArgs a{};
@@ -751,6 +815,7 @@ extern "C" rk_status rk_segpaged_decode(const rk_dims* dims, const rk_layout* la
   a.range_start = vis->range_start;
   a.range_count = vis->range_count;
   a.req_len = reinterpret_cast<const int32_t*>(ws + plan.off_req_len);
+  a.tables = reinterpret_cast<const DecodeTable*>(ws + plan.off_tables);
   a.o = o;
   a.lse = lse;
   a.part_o = reinterpret_cast<float*>(ws + plan.off_part_o);
@@ -762,7 +827,9 @@ extern "C" rk_status rk_segpaged_decode(const rk_dims* dims, const rk_layout* la
   a.hkv = dims->num_kv_heads;
   a.d = dims->head_dim;
   a.p = dims->page_size;
-  a.max_splits = plan.max_splits;
+  a.n_cta = plan.n_cta;
+  a.per = plan.per;
+  a.total = static_cast<int>(plan.total);
   a.window = layout->class_window[RK_LOCAL];
   a.softmax_scale = softmax_scale;
   a.cls = layout->class_map;

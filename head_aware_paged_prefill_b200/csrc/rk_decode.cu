@@ -8,14 +8,18 @@
 // does.
 //
 // HBM bound: every visible key and value is read once per kv head, for all
-// G q heads of the group.  Split-K flash decode:
-//   1. one CTA per (table, split of kDecodePages pages); each warp streams
-//      its own 16-key slices through a private cp.async ring and runs
-//      Q K^T and P V of the GQA group as warp-level bf16 MMAs (the G heads
-//      are the rows of a 16-row tile), with its own online softmax; the
-//      warps merge once at the end and the split writes (o, m, l);
-//   2. one CTA per table merges its splits: o = sum_s o_s 2^(m_s - M) / L,
-//      lse = (M + log2 L) ln 2, written as bf16 / fp32.
+// G q heads of the group.  Split-K flash decode with balanced splits:
+//   1. the tables' decode pages, concatenated in table order, are cut on the
+//      host into equal ranges, one per CTA (two CTAs per SM, one wave), so
+//      every CTA streams the same number of pages.  A CTA walks its range
+//      table by table; each piece (the range's part in one table) is
+//      streamed by the CTA's warps, each through a private cp.async ring of
+//      16-key slices, running Q K^T and P V of the GQA group as warp-level
+//      bf16 MMAs (the G heads are the rows of a 16-row tile) with its own
+//      online softmax; the warps merge at the piece's end and the piece
+//      writes (o, m, l);
+//   2. one CTA per table merges its pieces in order: o = sum_s o_s
+//      2^(m_s - M) / L, lse = (M + log2 L) ln 2, written as bf16 / fp32.
 // The MMAs are there to cut instruction issue (the CUDA-core form of the
 // same dot products issued ~5x more instructions per byte and reached a
 // third of the HBM bandwidth); the bound stays the HBM stream.  Warp-level
@@ -50,12 +54,13 @@ struct DecodeArgs {
   const int32_t* range_start;
   const int32_t* range_count;
   const int32_t* req_len;  // [n_req]
+  const DecodeTable* tables;  // [n_tables]
   __nv_bfloat16* o;  // [n_layers][n_req][hq][d]
   float* lse;        // [n_layers][hq][n_req] or null
-  float* part_o;     // [n_tables][max_splits][g][d]
-  float* part_ml;    // [n_tables][max_splits][g][2]
+  float* part_o;     // [pieces][g][d]
+  float* part_ml;    // [pieces][g][2]
   int64_t n_pages;
-  int n_req, n_layers, hq, hkv, g, p, max_splits, window;
+  int n_req, n_layers, hq, hkv, g, p, n_cta, per, total, window;
   float scale_log2;  // softmax scale * log2(e)
   int8_t cls[kDecodeMaxLh];
   int32_t* error_word;
@@ -109,49 +114,8 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-// The entries a decode row reads: from the first whose last key is at or
-// after lo (entries are in ascending logical_pos; a local table's list covers
-// the windows of all its rows, the decode row needs only its own) to the
-// table's end.  A warp-wide search: each round probes 32 entries and keeps
-// the interval between the last probe before lo and the first after it.
-// Every lane returns the same index.
-__device__ __forceinline__ int first_entry_at(const rk_entry* en, int n, int lo, int lane) {
-  int a = 0, b = n;  // the answer lies in [a, b] (b = n: no such entry)
-  while (a < b) {
-    const int step = (b - a + 30) / 31;  // probe 31 sits at or past b
-    const int p = a + lane * step;
-    bool at = true;
-    if (p < b) {
-      const rk_entry e = en[p];
-      at = e.logical_pos + e.n_valid - 1 >= lo;
-    }
-    const int f = __ffs(__ballot_sync(0xffffffffu, at)) - 1;
-    if (f == 0) return a;
-    const int nb = min(a + f * step, b);
-    a = a + (f - 1) * step + 1;
-    b = nb;
-  }
-  return b;
-}
-
-// This table's decode entries [first, n_e) cut into n_split balanced splits
-// of at most kDecodePages pages (`per` each, the last one shorter).
-struct DecodeSplits {
-  int first, n_split, per;
-};
-__device__ __forceinline__ DecodeSplits decode_splits(const DecodeArgs& a, int t, int cls, int lo,
-                                                      int lane) {
-  const int n_e = a.entry_count[t];
-  DecodeSplits d;
-  d.first = cls == RK_LOCAL && lo > 0 ? first_entry_at(a.entries + a.entry_start[t], n_e, lo, lane)
-                                      : 0;
-  const int n_vis = n_e - d.first;
-  d.n_split = (n_vis + kDecodePages - 1) / kDecodePages;
-  d.per = d.n_split > 0 ? (n_vis + d.n_split - 1) / d.n_split : 0;
-  return d;
-}
-
-// 1. one split of one table.  The split's pages are cut into 16-key slices
+// 1. one piece: entries [e0, e0 + n_ent) of table t's page table, result
+// into partial `part`.  The piece's pages are cut into 16-key slices
 // (P / 16 per page); warp w takes slices w, w + NW, ... and streams them
 // through its own ring of kDecodeStages shared-memory buffers by cp.async,
 // so the warps never wait for one another inside the loop.  Per slice:
@@ -162,33 +126,25 @@ __device__ __forceinline__ DecodeSplits decode_splits(const DecodeArgs& a, int t
 // Rows of K and V are stored with their 16-byte chunks permuted (chunk c of
 // key k at c ^ (k & 7)), so that the eight rows each ldmatrix reads fall in
 // distinct banks.  At the end the warps' (m, l, o) are merged in shared
-// memory and the split writes (o, m, l).
+// memory and the piece writes (o, m, l).
 template <int D, int G>
-__global__ void __launch_bounds__(kDecodeThreads)
-    decode_split_kernel(const __grid_constant__ DecodeArgs a) {
+__device__ void decode_piece(const DecodeArgs& a, int t, int e0, int n_ent, int64_t part,
+                             uint8_t* smem) {
   constexpr int NW = kDecodeThreads / 32;
   constexpr int KS = D / 16;      // 16-column steps of Q K^T; pairs of 8-column tiles of P V
   constexpr int CHUNKS = D / 8;   // 16-byte chunks of a key row
   constexpr int SLICE = 16 * D;   // elements of one slice of K (or V)
-  extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gq = lane >> 2, tq = lane & 3;  // fragment row (q head) and column pair
   const int P = a.p;
-  const int t = blockIdx.x, split = blockIdx.y;
   const int kvh = t % a.hkv, layer = (t / a.hkv) % a.n_layers, r = t / (a.hkv * a.n_layers);
-  const int n_e = a.entry_count[t], e_first = a.entry_start[t];
-  const int64_t part = static_cast<int64_t>(t) * a.max_splits + split;
+  const int e_first = a.entry_start[t];
   const int row = a.req_len[r] - 1;  // the request's last position
-  // the row must belong to the table's row set (else the combine skips it too)
-  const int rc = a.range_count[t];
-  if (n_e == 0 || rc == 0 || a.ranges[a.range_start[t] + rc - 1].end != row + 1) return;
   const int cls = a.cls[layer * a.hkv + kvh];
   const int lo = cls == RK_LOCAL ? row - a.window + 1 : 0;  // first visible key
-  const DecodeSplits ds = decode_splits(a, t, cls, lo, lane);
-  if (split >= ds.n_split) return;
-  const int e0 = ds.first + split * ds.per;
+  __syncthreads();  // the previous piece's merge is done with the shared memory
   const int spp = P / 16;
-  const int n_slices = (min(n_e, e0 + ds.per) - e0) * spp;
+  const int n_slices = n_ent * spp;
   const int my_n = warp < n_slices ? (n_slices - warp + NW - 1) / NW : 0;
   __nv_bfloat16* ring =
       reinterpret_cast<__nv_bfloat16*>(smem) + warp * (kDecodeStages * 2 * SLICE);
@@ -349,30 +305,57 @@ __global__ void __launch_bounds__(kDecodeThreads)
   }
 }
 
-// 2. merge the splits of one table
+// 1'. the CTA's range [c per, (c + 1) per) of the concatenated decode pages,
+// piece by piece (the range's part in each table it crosses)
+template <int D, int G>
+__global__ void __launch_bounds__(kDecodeThreads)
+    decode_split_kernel(const __grid_constant__ DecodeArgs a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int c = blockIdx.x, n_tables = a.n_req * a.n_layers * a.hkv;
+  int a0 = c * a.per;
+  const int a1 = min(a.total, a0 + a.per);
+  int lo = 0, hi = n_tables;  // last table with g0 <= a0
+  while (hi - lo > 1) {
+    const int m = (lo + hi) >> 1;
+    if (a.tables[m].g0 <= a0) lo = m; else hi = m;
+  }
+  int t = lo;
+  while (a0 < a1) {
+    while (t < n_tables && a.tables[t].g0 + a.tables[t].n_dec <= a0) ++t;
+    if (t >= n_tables) break;
+    const DecodeTable dt = a.tables[t];
+    const int end = min(a1, dt.g0 + dt.n_dec);
+    const int64_t part = static_cast<int64_t>(dt.piece_base) + (c - dt.c_first);
+    if (a.entry_count[t] == dt.n_e) {
+      decode_piece<D, G>(a, t, dt.first + (a0 - dt.g0), end - a0, part, smem);
+    } else {  // page tables of another layout: an empty partial, flagged
+      if (threadIdx.x == 0) atomicOr(a.error_word, static_cast<int>(RK_DEV_CAPACITY));
+      for (int x = threadIdx.x; x < G * D; x += kDecodeThreads) a.part_o[part * G * D + x] = 0.f;
+      for (int x = threadIdx.x; x < G; x += kDecodeThreads) {
+        a.part_ml[(part * G + x) * 2] = -INFINITY;
+        a.part_ml[(part * G + x) * 2 + 1] = 0.f;
+      }
+    }
+    a0 = end;
+  }
+}
+
+// 2. merge the pieces of one table, in order
 template <int D, int G>
 __global__ void __launch_bounds__(kDecodeThreads)
     decode_combine_kernel(const __grid_constant__ DecodeArgs a) {
   const int t = blockIdx.x;
   const int kvh = t % a.hkv, layer = (t / a.hkv) % a.n_layers, r = t / (a.hkv * a.n_layers);
-  const int n_e = a.entry_count[t];
-  const int row = a.req_len[r] - 1;
-  {
-    const int rc = a.range_count[t];
-    if (n_e == 0 || rc == 0 || a.ranges[a.range_start[t] + rc - 1].end != row + 1)
-      return;  // the request's last position is not a row of this table
-  }
-  const int cls = a.cls[layer * a.hkv + kvh];
-  const int lo = cls == RK_LOCAL ? row - a.window + 1 : 0;
-  const int n_split = decode_splits(a, t, cls, lo, threadIdx.x & 31).n_split;
-  const int64_t base = static_cast<int64_t>(t) * a.max_splits;
+  const DecodeTable dt = a.tables[t];
+  if (dt.n_dec == 0) return;  // the request's last position is not a row of this table
+  const int64_t base = dt.piece_base;
   for (int x = threadIdx.x; x < G * D; x += kDecodeThreads) {
     const int h = x / D, c = x % D;
     float M = -INFINITY;
-    for (int s = 0; s < n_split; ++s) M = fmaxf(M, a.part_ml[((base + s) * G + h) * 2]);
+    for (int s = 0; s < dt.n_pieces; ++s) M = fmaxf(M, a.part_ml[((base + s) * G + h) * 2]);
     float L = 0.f, acc = 0.f;
     if (M != -INFINITY) {
-      for (int s = 0; s < n_split; ++s) {
+      for (int s = 0; s < dt.n_pieces; ++s) {
         const float m = a.part_ml[((base + s) * G + h) * 2];
         if (m == -INFINITY) continue;
         const float f = exp2f(m - M);
@@ -400,7 +383,7 @@ cudaError_t launch_decode_typed(const DecodeArgs& a, int n_tables, cudaStream_t 
   cudaError_t e = cudaFuncSetAttribute(split, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  split<<<dim3(n_tables, a.max_splits), kDecodeThreads, smem, stream>>>(a);
+  split<<<a.n_cta, kDecodeThreads, smem, stream>>>(a);
   decode_combine_kernel<D, G><<<n_tables, kDecodeThreads, 0, stream>>>(a);
   return cudaGetLastError();
 }
@@ -419,6 +402,7 @@ cudaError_t launch_decode(const DecodeLaunchArgs& in, cudaStream_t stream) {
   a.range_start = in.range_start;
   a.range_count = in.range_count;
   a.req_len = in.req_len;
+  a.tables = in.tables;
   a.o = static_cast<__nv_bfloat16*>(in.o);
   a.lse = in.lse;
   a.part_o = in.part_o;
@@ -430,13 +414,15 @@ cudaError_t launch_decode(const DecodeLaunchArgs& in, cudaStream_t stream) {
   a.hkv = in.hkv;
   a.g = in.hq / in.hkv;
   a.p = in.p;
-  a.max_splits = in.max_splits;
+  a.n_cta = in.n_cta;
+  a.per = in.per;
+  a.total = in.total;
   a.window = in.window;
   a.scale_log2 = in.softmax_scale * 1.4426950408889634f;
   for (int k = 0; k < in.n_layers * in.hkv; ++k) a.cls[k] = in.cls[k];
   a.error_word = in.error_word;
   const int n_tables = in.n_req * in.n_layers * in.hkv;
-  if (n_tables == 0 || in.max_splits == 0) return cudaSuccess;
+  if (n_tables == 0 || in.total == 0) return cudaSuccess;
   const int G = a.g;
 #define RK_DECODE_CASE(DD, GG) \
   if (in.d == DD && G == GG) return launch_decode_typed<DD, GG>(a, n_tables, stream);

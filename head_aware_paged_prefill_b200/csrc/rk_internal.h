@@ -158,9 +158,19 @@ cudaError_t launch_score(const ScoreView* sv_dev, const ScoreView& sv_host, cons
 
 // ---- paged decode
 
-constexpr int kDecodePages = 64;    // pages per split of a table
 constexpr int kDecodeMaxLh = 1024;  // layers x kv heads per call
 constexpr int kDecodeMaxG = 8;      // q heads per kv head
+
+struct DecodeTable {  // one table's decode work (host-computed, uploaded)
+  int32_t g0;          // its first page in the concatenated decode pages of all tables
+  int32_t first;       // its first decode entry (page-table index)
+  int32_t n_dec;       // decode entries (0: the table reads nothing)
+  int32_t n_e;         // page-table entries the host expects (checked on the device)
+  int32_t piece_base;  // its first partial result
+  int32_t c_first;     // the CTA of its first piece
+  int32_t n_pieces;    // pieces (consecutive CTAs)
+  int32_t pad;
+};
 
 struct DecodeLaunchArgs {
   const void* q;  // bf16 [n_layers][n_req][hq][d]
@@ -172,13 +182,14 @@ struct DecodeLaunchArgs {
   const rk_range* ranges;
   const int32_t* range_start;
   const int32_t* range_count;
-  const int32_t* req_len;  // device [n_req]
+  const int32_t* req_len;      // device [n_req]
+  const DecodeTable* tables;   // device [n_tables]
   void* o;     // bf16 [n_layers][n_req][hq][d]
   float* lse;  // fp32 [n_layers][hq][n_req] or null
   float* part_o;
   float* part_ml;
   int64_t n_pages;
-  int n_req, n_layers, hq, hkv, d, p, max_splits, window;
+  int n_req, n_layers, hq, hkv, d, p, n_cta, per, total, window;
   float softmax_scale;
   const int8_t* cls;  // host [n_layers * hkv]
   int32_t* error_word;

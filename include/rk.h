@@ -356,7 +356,8 @@ rk_status rk_score_retrieval_pages(const rk_dims* dims, const rk_layout* layout,
  * layout.  bf16 in, fp32 scores and accumulation, bf16 out. */
 
 typedef struct {
-  int64_t max_splits;      /* splits of the longest table (<= 64 pages each) */
+  int64_t n_pieces;        /* partial results: the tables' decode pages are cut into equal
+                              per-CTA ranges, one partial per (table, range) piece */
   int64_t workspace_bytes; /* device workspace for rk_segpaged_decode */
 } rk_decode_sizes;
 
