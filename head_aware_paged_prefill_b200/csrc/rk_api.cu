@@ -184,6 +184,20 @@ void build_layout_image(const rk_dims* d, const rk_layout* lay, const Derived& d
   for (int r = 0; r < d->n_req; ++r)
     max_pages = std::max(max_pages, dv.page_prefix[r + 1] - dv.page_prefix[r]);
   v.max_table_pages = max_pages;
+  {
+    // work-list groups: (request, layer) pairs, a power of two of them so
+    // that each gets an equal share of the cost buckets; past
+    // kMaxBucketGroups one group (plain longest-first order)
+    const int64_t n_groups = static_cast<int64_t>(d->n_req) * d->n_layers;
+    int groups = 1;
+    if (n_groups > 1 && n_groups <= kMaxBucketGroups)
+      while (groups < n_groups) groups <<= 1;
+    const int bpg = kCostBuckets / groups;
+    const int ept = kKeysPerTile / d->page_size;
+    const int max_cost = (max_pages + ept - 1) / ept + 1;
+    v.bucket_groups = groups;
+    v.cost_width = std::max(1, (max_cost + 1 + bpg - 1) / bpg);
+  }
   int32_t off = static_cast<int32_t>((sizeof(LayoutView) + 3) / 4);
   int32_t* w = img->data();
   v.off_seg = off;

@@ -14,8 +14,12 @@ namespace rk {
 constexpr int kRowsPerTile = 128;  // query rows per Q tile (one TMEM lane per row)
 constexpr int kKeysPerTile = 128;  // keys per KV tile (N of the QK^T MMA)
 // Work items are ordered by cost (KV tiles) in this many buckets, longest
-// first; costs past the last bucket (over 256K keys) share it.
+// first; costs past the last bucket share it.  With several requests or
+// layers the buckets are split between (request, layer) groups, taken one
+// group after another, so the items that run side by side read the pages of
+// few tables (their K / V stays in L2).
 constexpr int kCostBuckets = 2048;
+constexpr int kMaxBucketGroups = 256;
 
 // Workspace header (first 256 bytes of the workspace).
 struct WsHeader {
@@ -56,6 +60,12 @@ struct LayoutView {
   int32_t window;                     // class_window[RK_LOCAL]
   int32_t item_capacity;
   int32_t max_table_pages;            // max_r ceil(L_r / P)
+  // work-list order: bucket_groups groups of kCostBuckets / bucket_groups
+  // cost buckets each (group = request x n_layers + layer when bucket_groups
+  // > 1, else one group), longest first inside a group, cost_width KV tiles
+  // per bucket
+  int32_t bucket_groups;
+  int32_t cost_width;
   // written by the select kernel (the host uploads them as zero each call)
   int32_t error;       // RK_DEV_* bits raised while selecting
   int32_t done_count;  // CTAs of the select kernel that finished their table

@@ -77,9 +77,14 @@ __device__ __forceinline__ int warp_claim(int* hist, int b, bool valid) {
   return base + rank;
 }
 
-// cost bucket of an item: bucket 0 holds the longest
-__device__ __forceinline__ int cost_bucket(int cost) {
-  return kCostBuckets - 1 - min(max(cost, 0), kCostBuckets - 1);
+// bucket of an item: groups in order ((request, layer) groups when the
+// layout has several), the longest first inside a group
+__device__ __forceinline__ int item_bucket(const LayoutView* lv, int req, int layer, int cost) {
+  const int groups = lv->bucket_groups;
+  const int bpg = kCostBuckets / groups;
+  const int g = groups > 1 ? req * lv->n_layers + layer : 0;
+  const int c = min(max(cost, 0) / lv->cost_width, bpg - 1);
+  return g * bpg + (bpg - 1 - c);
 }
 
 // index of the first of n entries whose key exceeds v (keys ascending)
@@ -270,7 +275,7 @@ __global__ void __launch_bounds__(kSelectThreads)
         it.table = t;
         it.cost = (e_hi - e_lo + ept - 1) / ept;
         items_tmp[first + x] = it;
-        bucket = cost_bucket(it.cost);
+        bucket = item_bucket(lv, r, layer, it.cost);
       }
       warp_claim(hist, bucket, bucket >= 0);
     }
@@ -322,7 +327,8 @@ __global__ void __launch_bounds__(kSelectThreads)
         for (int b = 0; b < kScatterBatch; ++b) {
           const int x = base + b * kSelectThreads + threadIdx.x;
           const bool v = x < total;
-          const int pos = warp_claim(hist, v ? cost_bucket(it[b].cost) : 0, v);
+          const int pos =
+              warp_claim(hist, v ? item_bucket(lv, it[b].req, it[b].layer, it[b].cost) : 0, v);
           if (v) items[pos] = it[b];
         }
       }
@@ -352,7 +358,8 @@ __global__ void __launch_bounds__(kSelectThreads)
   for (int round = 0; round < rounds; ++round) {
     const int x = round * kSelectThreads + threadIdx.x;
     const bool v = x < n_it;
-    warp_claim(hist, v ? cost_bucket(items_tmp[first + x].cost) : 0, v);
+    const Item* ix = items_tmp + first + x;
+    warp_claim(hist, v ? item_bucket(lv, ix->req, ix->layer, ix->cost) : 0, v);
   }
   __syncthreads();
   // this table's run of each bucket
@@ -364,7 +371,7 @@ __global__ void __launch_bounds__(kSelectThreads)
     const bool v = x < n_it;
     Item it;
     if (v) it = items_tmp[first + x];
-    const int pos = warp_claim(hist, v ? cost_bucket(it.cost) : 0, v);
+    const int pos = warp_claim(hist, v ? item_bucket(lv, it.req, it.layer, it.cost) : 0, v);
     if (v) items[pos] = it;
   }
 }

@@ -1,5 +1,6 @@
 """The attention work list the selection builds in the workspace: a
-permutation of the per-table items, longest first.  Small lists are sorted by
+permutation of the per-table items, longest first inside each (request,
+layer) group, the groups one after another.  Small lists are sorted by
 the selection kernel's last CTA, large ones by the per-table scatter launch;
 both are checked.  White-box: reads the workspace through its internal map
 (a 256-byte header, then the sorted list, then the unsorted list)."""
@@ -46,9 +47,24 @@ def _check(lay, expect_large=None):
     # a permutation of the per-table items
     key = lambda a: np.lexsort(a.T[::-1])
     assert np.array_equal(items[key(items)], tmp[key(tmp)])
-    # longest first (costs past the last bucket share it)
-    c = np.minimum(items[:, 11], COST_BUCKETS - 1)
-    assert np.all(c[:-1] >= c[1:])
+    # groups in order, longest first inside a group (costs past the last
+    # bucket of a group share it): a group is one (request, layer) when the
+    # layout has several (up to 256), the buckets split evenly between a
+    # power of two of groups
+    n_groups = lay.n_req * lay.n_layers
+    groups = 1
+    if 1 < n_groups <= 256:
+        while groups < n_groups:
+            groups *= 2
+    bpg = COST_BUCKETS // groups
+    ept = 128 // lay.p
+    max_pages = max(-(-lay.req_len(r) // lay.p) for r in range(lay.n_req))
+    max_cost = -(-max_pages // ept) + 1
+    width = max(1, -(-(max_cost + 1) // bpg))
+    g = items[:, 9] * lay.n_layers + items[:, 8] if groups > 1 else np.zeros(len(items), np.int64)
+    c = np.minimum(items[:, 11] // width, bpg - 1)
+    order = g * bpg + (bpg - 1 - c)
+    assert np.all(order[:-1] <= order[1:])
     # every item of a table lies in that table and has a cost of its entries
     assert np.all(items[:, 4] >= items[:, 3])
     assert np.all(items[:, 6] >= 1) and np.all(items[:, 6] <= 2)
