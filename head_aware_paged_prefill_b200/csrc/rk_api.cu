@@ -394,6 +394,8 @@ rk_status build_score_plan(const rk_dims* d, const rk_layout* lay, const Derived
   off = al4(off + static_cast<int32_t>(ranges.size() * sizeof(ScoreRange) / 4));
   v.off_table_map = off;
   off = al4(off + static_cast<int32_t>(table_map.size()));
+  v.off_done = off;
+  off = al4(off + static_cast<int32_t>(tables.size()));
   v.words = off;
   out->img.assign(static_cast<size_t>(off), 0);
   int32_t* w = out->img.data();
@@ -405,7 +407,7 @@ rk_status build_score_plan(const rk_dims* d, const rk_layout* lay, const Derived
   out->max_pages = max_pages;
   out->off_partials = align_up(4 * static_cast<size_t>(off), 256);
   out->off_kbar = align_up(out->off_partials + 4 * static_cast<size_t>(n_chunks) * D, 256);
-  out->off_urot = align_up(out->off_kbar + 4 * static_cast<size_t>(n_cand) * D, 256);
+  out->off_urot = align_up(out->off_kbar + 4 * static_cast<size_t>(n_cand), 256);  // kbar: the scores
   out->total = align_up(out->off_urot + 4 * runs.size() * D, 256);
   return RK_OK;
 }

@@ -153,16 +153,16 @@ struct ScoreView {
   int32_t off_runs;       // ScoreRun[n_runs]
   int32_t off_ranges;     // ScoreRange[n_ranges]
   int32_t off_table_map;  // int32[n_tables]: score table of a table, -1 if none
+  int32_t off_done;       // int32[n_st]: query chunks finished per score table (zero when uploaded)
   int32_t words;
 };
 
-// One launch sums the queries of every 64-row chunk (the first n_chunks
-// CTAs) and averages the stored keys of every candidate page (the other
-// CTAs, kScorePagesPerCta pages each); a second, one CTA per table, scores
-// and ranks.
+// Three launches: query chunk sums (the last chunk of a table forms the
+// rotated u of its runs), page scores (key means dotted with their run's
+// rotated u), and the picks, one CTA per table.
 cudaError_t launch_score(const ScoreView* sv_dev, const ScoreView& sv_host, const void* q,
                          const void* k_store, int D, int P, const double* inv_freq_host,
-                         float* partials, float* kbar, float* urot, int32_t* out_pages,
+                         float* partials, float* scores, float* urot, int32_t* out_pages,
                          int32_t* out_count, float* out_scores, int64_t scores_stride,
                          cudaStream_t stream);
 
