@@ -366,7 +366,7 @@ def _bench_scoring(torch, lay, q, k_store, dev, flush, stream, reps, peaks, peak
     nbytes = metrics.scoring_bytes(lay_r)
     gbs = nbytes / (t * 1e-3) / 1e9
     n_tables = int((out.count > 0).sum().item())
-    return {"bound": "hbm", "kernel": "score_query + score_pages + score_topk",
+    return {"bound": "hbm", "kernel": "score_query + score_page + score_pick",
             "workload": "the same layer, every kv head a retrieval head, top 16",
             "tables": n_tables, "bytes": nbytes, "achieved": gbs,
             "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
