@@ -407,7 +407,8 @@ rk_status build_score_plan(const rk_dims* d, const rk_layout* lay, const Derived
   out->max_pages = max_pages;
   out->off_partials = align_up(4 * static_cast<size_t>(off), 256);
   out->off_kbar = align_up(out->off_partials + 4 * static_cast<size_t>(n_chunks) * D, 256);
-  out->off_urot = align_up(out->off_kbar + 4 * static_cast<size_t>(n_cand), 256);  // kbar: the scores
+  // kbar: the scores (4 bytes each), then the rank keys (8 bytes each)
+  out->off_urot = align_up(out->off_kbar + 4 * static_cast<size_t>(n_cand + 1) + 8 * static_cast<size_t>(n_cand), 256);
   out->total = align_up(out->off_urot + 4 * runs.size() * D, 256);
   return RK_OK;
 }

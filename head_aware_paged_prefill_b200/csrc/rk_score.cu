@@ -24,10 +24,15 @@
 //      writes R(-delta) u for each of the table's runs;
 //   2. pages (HBM bound): one warp per candidate page sums the page's
 //      stored keys and takes the dot product of their mean with its run's
-//      rotated u at once, so the page's score leaves the launch;
-//   3. picks, one CTA per table: each candidate's rank is the number of
-//      (score, page) keys above its own (up to 2048 candidates; a bitonic
-//      sort above that); the first k, in ascending page order.
+//      rotated u at once, so the page's score and its rank key leave the
+//      launch;
+//   3. picks, one CTA per table: the k largest (score, page) keys, found
+//      by a radix select on the 64-bit key a byte at a time, written in
+//      ascending page order by a block-wide scan.
+// Launches 2 and 3 are programmatic dependents of the one before: the page
+// launch starts while the query launch still streams and waits for it only
+// before it reads the rotated u, and the pick launch waits before it reads
+// the scores.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -50,7 +55,6 @@ struct ScoreFreqs {
 constexpr int kQueryThreads = 256;
 constexpr int kPageThreads = 32 * kScorePagesPerCta;  // one warp per page
 constexpr int kPickThreads = 1024;
-constexpr int kRankCount = 2048;  // candidates ranked by counting (a sort above)
 
 // Last index in [lo, hi) whose key is <= x (the keys ascend; lo's is <= x).
 template <typename F>
@@ -61,6 +65,14 @@ __device__ __forceinline__ int last_at_most(int lo, int hi, int x, F key) {
   }
   return lo;
 }
+
+// Programmatic dependent launch: let the next launch on the stream begin,
+// and wait until the launch before has completed with its writes visible
+// (a no-op when this launch was not made a dependent).
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 __device__ __forceinline__ uint32_t order_bits(float f) {
   const uint32_t b = __float_as_uint(f);
@@ -78,6 +90,7 @@ __global__ void __launch_bounds__(kQueryThreads)
   __shared__ float acc_s[S][D];
   __shared__ float u[D];
   __shared__ int s_last;
+  pdl_launch_dependents();  // the page launch streams its keys meanwhile
   const ScoreTable* tabs = reinterpret_cast<const ScoreTable*>(sv_arr(sv, sv->off_tables));
   const ScoreRange* rgs = reinterpret_cast<const ScoreRange*>(sv_arr(sv, sv->off_ranges));
   const ScoreRun* runs = reinterpret_cast<const ScoreRun*>(sv_arr(sv, sv->off_runs));
@@ -133,8 +146,16 @@ __global__ void __launch_bounds__(kQueryThreads)
   {
     const int c = threadIdx.x % D, j = threadIdx.x / D;
     float t = 0.f;
-    for (int k = st.chunk_begin + j; k < st.chunk_end; k += R)
-      t += __ldcg(partials + static_cast<int64_t>(k) * D + c);
+    for (int k0 = st.chunk_begin + j; k0 < st.chunk_end; k0 += 8 * R) {
+      float v[8];  // eight loads in flight, added in chunk order
+#pragma unroll
+      for (int x = 0; x < 8; ++x) {
+        const int k = k0 + x * R;
+        v[x] = k < st.chunk_end ? __ldcg(partials + static_cast<int64_t>(k) * D + c) : 0.f;
+      }
+#pragma unroll
+      for (int x = 0; x < 8; ++x) t += v[x];
+    }
     acc_s[j][c] = t;
   }
   __syncthreads();
@@ -169,8 +190,10 @@ __global__ void __launch_bounds__(kQueryThreads)
 template <int D>
 __global__ void __launch_bounds__(kPageThreads)
     score_page_kernel(const ScoreView* __restrict__ sv, const __nv_bfloat16* __restrict__ k_store,
-                      int P, const float* __restrict__ urot, float* __restrict__ scores) {
+                      int P, const float* __restrict__ urot, float* __restrict__ scores,
+                      unsigned long long* __restrict__ keys) {
   constexpr int CPL = D / 32;
+  pdl_launch_dependents();  // the pick launch waits for this one to complete
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cand = blockIdx.x * kScorePagesPerCta + warp;
   if (cand >= sv->n_cand) return;
@@ -184,23 +207,51 @@ __global__ void __launch_bounds__(kPageThreads)
   float acc[CPL];
 #pragma unroll
   for (int k = 0; k < CPL; ++k) acc[k] = 0.f;
-#pragma unroll 8
-  for (int r = 0; r < n_valid; ++r) {
-    const __nv_bfloat16* kr = base + static_cast<int64_t>(r) * D;
+  // rows in batches of 16 loads in flight (two rounds for a 64-key page),
+  // added in row order
+  for (int r0 = 0; r0 < n_valid; r0 += 16) {
     if constexpr (CPL == 4) {
-      const uint2 raw = *reinterpret_cast<const uint2*>(kr);
-      const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
-      const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
-      acc[0] += x.x;
-      acc[1] += x.y;
-      acc[2] += y.x;
-      acc[3] += y.y;
+      uint2 raw[16];
+      if (r0 + 16 <= n_valid) {
+#pragma unroll
+        for (int x = 0; x < 16; ++x)
+          raw[x] = *reinterpret_cast<const uint2*>(base + static_cast<int64_t>(r0 + x) * D);
+      } else {
+#pragma unroll
+        for (int x = 0; x < 16; ++x)
+          raw[x] = r0 + x < n_valid ? *reinterpret_cast<const uint2*>(base + static_cast<int64_t>(r0 + x) * D)
+                                    : make_uint2(0u, 0u);
+      }
+#pragma unroll
+      for (int x = 0; x < 16; ++x) {
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw[x].x));
+        const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw[x].y));
+        acc[0] += a.x;
+        acc[1] += a.y;
+        acc[2] += b.x;
+        acc[3] += b.y;
+      }
     } else {
-      const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(kr));
-      acc[0] += x.x;
-      acc[1] += x.y;
+      uint32_t raw[16];
+      if (r0 + 16 <= n_valid) {
+#pragma unroll
+        for (int x = 0; x < 16; ++x)
+          raw[x] = *reinterpret_cast<const uint32_t*>(base + static_cast<int64_t>(r0 + x) * D);
+      } else {
+#pragma unroll
+        for (int x = 0; x < 16; ++x)
+          raw[x] = r0 + x < n_valid ? *reinterpret_cast<const uint32_t*>(base + static_cast<int64_t>(r0 + x) * D)
+                                    : 0u;
+      }
+#pragma unroll
+      for (int x = 0; x < 16; ++x) {
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw[x]));
+        acc[0] += a.x;
+        acc[1] += a.y;
+      }
     }
   }
+  pdl_wait();  // the query launch's rotated u
   const float inv = 1.f / static_cast<float>(n_valid);
   const float* ub = urot + static_cast<int64_t>(rn) * D + lane * CPL;
   float sc = 0.f;
@@ -208,85 +259,125 @@ __global__ void __launch_bounds__(kPageThreads)
   for (int k = 0; k < CPL; ++k) sc = fmaf(ub[k], acc[k] * inv, sc);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sc += __shfl_xor_sync(0xffffffffu, sc, o);
-  if (lane == 0) scores[cand] = sc;
+  if (lane == 0) {
+    scores[cand] = sc;
+    const float rank_sc = isnan(sc) ? -INFINITY : sc;  // a NaN score (bad input) ranks last
+    keys[cand] = (static_cast<unsigned long long>(order_bits(rank_sc)) << 32) |
+                 static_cast<uint32_t>(~static_cast<uint32_t>(page));
+  }
 }
 
 // 3. the picks of one table from its candidates' scores
 __global__ void __launch_bounds__(kPickThreads)
     score_pick_kernel(const ScoreView* __restrict__ sv, const float* __restrict__ scores,
-                      int32_t* __restrict__ out_pages, int32_t* __restrict__ out_count,
+                      const unsigned long long* __restrict__ keys, int32_t* __restrict__ out_pages,
+                      int32_t* __restrict__ out_count,
                       float* __restrict__ out_scores, int64_t scores_stride) {
   __shared__ unsigned long long s_key[kScoreMaxCand];
-  __shared__ int s_picked[kRankCount];
+  __shared__ int s_hist[256];
+  __shared__ int s_sel[3];
+  __shared__ int s_warp[kPickThreads / 32];
   const int t = blockIdx.x;
   const int top_k = sv->top_k;
   const int st_idx = sv_arr(sv, sv->off_table_map)[t];
   if (out_scores)
     for (int64_t c = threadIdx.x; c < scores_stride; c += kPickThreads)
       out_scores[t * scores_stride + c] = __int_as_float(0x7fc00000);  // NaN
+  // the plan (uploaded before the first launch) is read before the wait
+  ScoreTable st{};
+  if (st_idx >= 0) st = reinterpret_cast<const ScoreTable*>(sv_arr(sv, sv->off_tables))[st_idx];
+  const int n = st_idx >= 0 ? st.cand_end - st.cand_begin : 0;
+  pdl_wait();  // the page launch's scores and keys
   if (st_idx < 0) {
     if (threadIdx.x == 0) out_count[t] = 0;
     return;
   }
-  const ScoreTable st = reinterpret_cast<const ScoreTable*>(sv_arr(sv, sv->off_tables))[st_idx];
-  const ScoreRun* runs = reinterpret_cast<const ScoreRun*>(sv_arr(sv, sv->off_runs));
-  const int n = st.cand_end - st.cand_begin;
-  int n2 = 1;
-  while (n2 < n) n2 <<= 1;
-  for (int x = n + threadIdx.x; x < n2; x += kPickThreads) s_key[x] = 0;  // padding sorts last
   if (out_scores) __syncthreads();  // the NaN fill lands before the scores
   for (int x = threadIdx.x; x < n; x += kPickThreads) {
-    const int xc = st.cand_begin + x;
-    const ScoreRun& ru = runs[last_at_most(st.run_begin, st.run_end, xc,
-                                           [&](int m) { return runs[m].cand_begin; })];
-    const int pg = ru.first_page + (xc - ru.cand_begin);
-    const float sc = scores[xc];
-    if (out_scores && pg < scores_stride) out_scores[t * scores_stride + pg] = sc;
-    const float rank_sc = isnan(sc) ? -INFINITY : sc;  // a NaN score (bad input) ranks last
-    s_key[x] = (static_cast<unsigned long long>(order_bits(rank_sc)) << 32) |
-               static_cast<uint32_t>(~static_cast<uint32_t>(pg));
+    const unsigned long long key = keys[st.cand_begin + x];
+    s_key[x] = key;
+    const uint32_t pg = ~static_cast<uint32_t>(key);
+    if (out_scores && pg < scores_stride) out_scores[t * scores_stride + pg] = scores[st.cand_begin + x];
   }
   __syncthreads();
   const int n_pick = n < top_k ? n : top_k;
-  if (n <= kRankCount) {
-    // rank of a key = the keys above it (keys are distinct: the page is in
-    // the low bits); a candidate is picked if its rank is below n_pick, and
-    // its output slot is the number of picked candidates before it (the
-    // candidates ascend in page)
-    for (int x = threadIdx.x; x < n; x += kPickThreads) {
-      const unsigned long long kx = s_key[x];
-      int rank = 0;
-      for (int y = 0; y < n; ++y) rank += s_key[y] > kx ? 1 : 0;
-      s_picked[x] = rank < n_pick ? 1 : 0;
-    }
-    __syncthreads();
-    for (int x = threadIdx.x; x < n; x += kPickThreads) {
-      if (!s_picked[x]) continue;
-      int pos = 0;
-      for (int y = 0; y < x; ++y) pos += s_picked[y];
-      out_pages[t * top_k + pos] = static_cast<int32_t>(~static_cast<uint32_t>(s_key[x]));
-    }
-  } else {
-    // bitonic sort, descending: higher score first, equal score to the lower page
-    for (int k = 2; k <= n2; k <<= 1)
-      for (int j = k >> 1; j > 0; j >>= 1) {
-        for (int i = threadIdx.x; i < n2; i += kPickThreads) {
-          const int p = i ^ j;
-          if (p > i) {
-            const unsigned long long a = s_key[i], b = s_key[p];
-            if (((i & k) == 0) ? (a < b) : (a > b)) {
-              s_key[i] = b;
-              s_key[p] = a;
+  {
+    // the picks are the n_pick largest keys (distinct: the page is in the
+    // low bits), found by a radix select from the top byte down: prefix /
+    // mask hold the decided high bits of the threshold, `need` the picks
+    // still to take among keys matching them; a key is picked when its
+    // decided bits reach the prefix.  The select stops as soon as the
+    // keys matching the prefix are exactly the picks still needed.
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    unsigned long long prefix = 0ull, mask = 0ull;
+    int need = n_pick;
+    for (int shift = 56; shift >= 0 && need > 0; shift -= 8) {
+      if (threadIdx.x < 256) s_hist[threadIdx.x] = 0;
+      __syncthreads();
+      for (int x = threadIdx.x; x < n; x += kPickThreads) {
+        const unsigned long long kx = s_key[x];
+        if ((kx & mask) == prefix) atomicAdd(&s_hist[(kx >> shift) & 255u], 1);
+      }
+      __syncthreads();
+      if (w == 0) {
+        // lane l holds digits 255 - 8l down to 248 - 8l (descending)
+        int c[8], loc = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          c[j] = s_hist[255 - 8 * lane - j];
+          loc += c[j];
+        }
+        int incl = loc;
+        for (int o = 1; o < 32; o <<= 1) {
+          const int u = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += u;
+        }
+        int above = incl - loc;  // keys matching the prefix with a larger digit
+        if (above < need && need <= incl) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            if (above + c[j] >= need) {
+              s_sel[0] = 255 - 8 * lane - j;
+              s_sel[1] = above;
+              s_sel[2] = c[j];
+              break;
             }
+            above += c[j];
           }
         }
-        __syncthreads();
       }
-    if (threadIdx.x < n_pick) {
-      const uint32_t pg = ~static_cast<uint32_t>(s_key[threadIdx.x]);
-      int pos = 0;
-      for (int x = 0; x < n_pick; ++x) pos += (~static_cast<uint32_t>(s_key[x])) < pg ? 1 : 0;
-      out_pages[t * top_k + pos] = static_cast<int32_t>(pg);
+      __syncthreads();
+      const int d = s_sel[0], above = s_sel[1], cnt = s_sel[2];
+      prefix |= static_cast<unsigned long long>(d) << shift;
+      mask |= 255ull << shift;
+      need -= above;
+      if (cnt == need) need = 0;  // every key matching the prefix is a pick
+      __syncthreads();           // s_hist and s_sel are reused
+    }
+    // output slot = picked candidates before it (the candidates ascend in
+    // page): ballots within a warp, the warps' counts scanned by warp 0
+    int placed = 0;
+    for (int base = 0; base < n; base += kPickThreads) {
+      const int x = base + threadIdx.x;
+      const bool f = x < n && (s_key[x] & mask) >= prefix;
+      const unsigned m = __ballot_sync(0xffffffffu, f);
+      if (lane == 0) s_warp[w] = __popc(m);
+      __syncthreads();
+      if (w == 0) {
+        int v = s_warp[lane];
+        for (int o = 1; o < 32; o <<= 1) {
+          const int u = __shfl_up_sync(0xffffffffu, v, o);
+          if (lane >= o) v += u;
+        }
+        s_warp[lane] = v;  // inclusive prefix over the warps
+      }
+      __syncthreads();
+      if (f) {
+        const int pos = placed + (w ? s_warp[w - 1] : 0) + __popc(m & ((1u << lane) - 1u));
+        out_pages[t * top_k + pos] = static_cast<int32_t>(~static_cast<uint32_t>(s_key[x]));
+      }
+      placed += s_warp[kPickThreads / 32 - 1];
+      __syncthreads();
     }
   }
   if (threadIdx.x == 0) out_count[t] = n_pick;
@@ -309,15 +400,34 @@ cudaError_t launch_score(const ScoreView* sv_dev, const ScoreView& sv_host, cons
     else
       score_query_kernel<64><<<sv_host.n_chunks, kQueryThreads, 0, stream>>>(sv_dev, f, qb, partials, urot);
   }
+  // the scores, then (8-byte aligned) the rank keys, share one workspace slot
+  auto* keys = reinterpret_cast<unsigned long long*>(
+      scores + ((static_cast<int64_t>(sv_host.n_cand) + 1) & ~static_cast<int64_t>(1)));
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg{};
+  cfg.stream = stream;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaSuccess;
   if (sv_host.n_page_blocks > 0) {
-    if (D == 128)
-      score_page_kernel<128><<<sv_host.n_page_blocks, kPageThreads, 0, stream>>>(sv_dev, kb, P, urot, scores);
-    else
-      score_page_kernel<64><<<sv_host.n_page_blocks, kPageThreads, 0, stream>>>(sv_dev, kb, P, urot, scores);
+    cfg.gridDim = dim3(sv_host.n_page_blocks);
+    cfg.blockDim = dim3(kPageThreads);
+    e = D == 128 ? cudaLaunchKernelEx(&cfg, score_page_kernel<128>, sv_dev, kb, P,
+                                      static_cast<const float*>(urot), scores, keys)
+                 : cudaLaunchKernelEx(&cfg, score_page_kernel<64>, sv_dev, kb, P,
+                                      static_cast<const float*>(urot), scores, keys);
+    if (e != cudaSuccess) return e;
   }
-  if (sv_host.n_tables > 0)
-    score_pick_kernel<<<sv_host.n_tables, kPickThreads, 0, stream>>>(sv_dev, scores, out_pages, out_count,
-                                                                     out_scores, scores_stride);
+  if (sv_host.n_tables > 0) {
+    cfg.gridDim = dim3(sv_host.n_tables);
+    cfg.blockDim = dim3(kPickThreads);
+    e = cudaLaunchKernelEx(&cfg, score_pick_kernel, sv_dev, static_cast<const float*>(scores),
+                           static_cast<const unsigned long long*>(keys), out_pages, out_count,
+                           out_scores, scores_stride);
+    if (e != cudaSuccess) return e;
+  }
   return cudaGetLastError();
 }
 

@@ -126,3 +126,33 @@ def test_scored_lists_drive_attention():
     idx = [torch.from_numpy(rows[:, c]).long().cuda() for c in (0, 2, 1)]
     got = o[idx[0], idx[1], idx[2]].double().cpu().numpy()
     assert_close(got, o_ref, "scored retrieval o")
+
+
+def _retrieval_layout(seg_len, n_seg, tail, p=16, hq=2, hkv=1, d=64):
+    segs = [(f"c{i}", seg_len, 0, True) for i in range(n_seg)] + [("tail", tail, 0, False)]
+    return synth._make_layout(n_layers=1, hq=hq, hkv=hkv, d=d, p=p, theta=1e4, requests=[segs],
+                              class_map=[synth.RETRIEVAL] * hkv, window=0)
+
+
+@pytest.mark.parametrize("top_k", [1, 7, 64])
+def test_score_ties_go_to_the_lower_pages(top_k):
+    """Zero queries make every candidate's score exactly zero: the picks are
+    then decided by the page alone (ties to the lower page), so every byte
+    of the (score, page) key takes part in the selection."""
+    lay = _retrieval_layout(1024, 3, 64, hkv=2, hq=4)
+    q, k, _ = synth.tiny_workload(lay, seed=31).materialize("cuda")
+    q.zero_()
+    out = _run(lay, q, k, top_k)
+    for t in range(lay.n_tables):
+        assert out.count[t].item() == top_k
+        assert out.pages[t, :top_k].cpu().numpy().tolist() == list(range(top_k))
+        assert (out.scores[t, :192] == 0).all()
+
+
+@pytest.mark.parametrize("n_seg,top_k", [(9, 16), (16, 64)])
+def test_score_thousands_of_candidates(n_seg, top_k):
+    """2304 and 4096 (the most a table takes) candidate pages of 16 keys."""
+    lay = _retrieval_layout(4096, n_seg, 128)
+    wl = synth.tiny_workload(lay, seed=32 + n_seg)
+    q, k, _ = wl.materialize("cpu")
+    assert _check(lay, q, k, top_k, f"{n_seg * 256} candidates") == 1
