@@ -396,6 +396,10 @@ rk_status build_score_plan(const rk_dims* d, const rk_layout* lay, const Derived
   off = al4(off + static_cast<int32_t>(table_map.size()));
   v.off_done = off;
   off = al4(off + static_cast<int32_t>(tables.size()));
+  v.off_chunk_table = off;
+  off = al4(off + v.n_chunks);
+  v.off_block_run = off;
+  off = al4(off + v.n_page_blocks);
   v.words = off;
   out->img.assign(static_cast<size_t>(off), 0);
   int32_t* w = out->img.data();
@@ -404,6 +408,16 @@ rk_status build_score_plan(const rk_dims* d, const rk_layout* lay, const Derived
   if (!runs.empty()) std::memcpy(w + v.off_runs, runs.data(), runs.size() * sizeof(ScoreRun));
   if (!ranges.empty()) std::memcpy(w + v.off_ranges, ranges.data(), ranges.size() * sizeof(ScoreRange));
   if (!table_map.empty()) std::memcpy(w + v.off_table_map, table_map.data(), table_map.size() * 4);
+  // the lookups the kernels would otherwise search for: a chunk's table and
+  // the run holding a page block's first candidate (runs are never empty)
+  for (int32_t i = 0; i < v.n_st; ++i)
+    for (int32_t c = tables[static_cast<size_t>(i)].chunk_begin; c < tables[static_cast<size_t>(i)].chunk_end; ++c)
+      w[v.off_chunk_table + c] = i;
+  for (int32_t b = 0, rn = 0; b < v.n_page_blocks; ++b) {
+    const int32_t first = b * kScorePagesPerCta;
+    while (rn + 1 < v.n_runs && runs[static_cast<size_t>(rn) + 1].cand_begin <= first) ++rn;
+    w[v.off_block_run + b] = rn;
+  }
   out->max_pages = max_pages;
   out->off_partials = align_up(4 * static_cast<size_t>(off), 256);
   out->off_kbar = align_up(out->off_partials + 4 * static_cast<size_t>(n_chunks) * D, 256);

@@ -154,6 +154,8 @@ struct ScoreView {
   int32_t off_ranges;     // ScoreRange[n_ranges]
   int32_t off_table_map;  // int32[n_tables]: score table of a table, -1 if none
   int32_t off_done;       // int32[n_st]: query chunks finished per score table (zero when uploaded)
+  int32_t off_chunk_table;  // int32[n_chunks]: score table of each query chunk
+  int32_t off_block_run;    // int32[n_page_blocks]: run of each page block's first candidate
   int32_t words;
 };
 

@@ -56,16 +56,6 @@ constexpr int kQueryThreads = 256;
 constexpr int kPageThreads = 32 * kScorePagesPerCta;  // one warp per page
 constexpr int kPickThreads = 1024;
 
-// Last index in [lo, hi) whose key is <= x (the keys ascend; lo's is <= x).
-template <typename F>
-__device__ __forceinline__ int last_at_most(int lo, int hi, int x, F key) {
-  while (hi - lo > 1) {
-    const int m = (lo + hi) >> 1;
-    if (key(m) <= x) lo = m; else hi = m;
-  }
-  return lo;
-}
-
 // Programmatic dependent launch: let the next launch on the stream begin,
 // and wait until the launch before has completed with its writes visible
 // (a no-op when this launch was not made a dependent).
@@ -96,7 +86,7 @@ __global__ void __launch_bounds__(kQueryThreads)
   const ScoreRun* runs = reinterpret_cast<const ScoreRun*>(sv_arr(sv, sv->off_runs));
   int* done = const_cast<int*>(sv_arr(sv, sv->off_done));  // zeros in the uploaded image
   const int b = blockIdx.x;
-  const int st_idx = last_at_most(0, sv->n_st, b, [&](int m) { return tabs[m].chunk_begin; });
+  const int st_idx = sv_arr(sv, sv->off_chunk_table)[b];
   const ScoreTable st = tabs[st_idx];
   int lc = b - st.chunk_begin, row_begin = 0, n_rows = 0;
   for (int x = st.range_begin; x < st.range_end; ++x) {
@@ -198,7 +188,9 @@ __global__ void __launch_bounds__(kPageThreads)
   const int cand = blockIdx.x * kScorePagesPerCta + warp;
   if (cand >= sv->n_cand) return;
   const ScoreRun* runs = reinterpret_cast<const ScoreRun*>(sv_arr(sv, sv->off_runs));
-  const int rn = last_at_most(0, sv->n_runs, cand, [&](int m) { return runs[m].cand_begin; });
+  // the run of the block's first candidate, then forward to this warp's
+  int rn = sv_arr(sv, sv->off_block_run)[blockIdx.x];
+  while (rn + 1 < sv->n_runs && runs[rn + 1].cand_begin <= cand) ++rn;
   const ScoreRun ru = runs[rn];
   const int page = ru.first_page + (cand - ru.cand_begin);
   const int n_valid = min(P, ru.req_len - page * P);
